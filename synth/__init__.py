@@ -1,0 +1,248 @@
+"""Seeded synthetic inputs for the sparse latent-MoE decode layer step.
+
+This package only draws random numbers (see ``synth.c`` for the generator's definition).
+It holds none of the layer's arithmetic, so the CPU oracle and the CUDA path can both take
+their inputs from it without sharing any code of the method.
+
+Workloads (the five shapes the layer is exercised on):
+
+=================  ====================================================================
+name               shape
+=================  ====================================================================
+tiny_b1            H=512, L=256, E=64, k=4, I=256, I_s=256, B=1
+full_b1            H=7168, L=2048, E=896, k=16, I=1024, I_s=2048, B=1
+full_b2            full size, B=2; token 1 = bf16(token 0 + 0.1 N(0,1))
+full_b16           full size, B=16, independent N(0,1) tokens
+full_b64_skewed    full size, B=64; 32 hot router rows get beta * u added (u ~ N(0,1/H)),
+                   timed over 32 layers of distinct weights
+=================  ====================================================================
+
+Value recipe: tokens bf16 ~ N(0,1); router, W_dn, W_up bf16 ~ N(0, 1/fan_in); MXFP4 codes
+uniform 4-bit; E8M0 scale bytes 127 + U{-6..-2}.  Kimi K3's layer (896 experts, 16
+active, MXFP4 weights) is described on "Hyper Optimizing Kimi K3 in vLLM" coverage pages
+(jetabc.cn, section "为什么一条请求会慢"); all dimensions come from the workload table.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libsynth.so")
+_SRC = os.path.join(_HERE, "synth.c")
+
+
+def build(force: bool = False) -> str:
+    """Compile libsynth.so next to its source (gcc, OpenMP)."""
+    if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", _SRC, "-o", _SO, "-lm"])
+    return _SO
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_SO)
+        u64, u32, dbl = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_double
+        vp = ctypes.c_void_p
+        L.synth_key.argtypes = [u64, u64, u64]
+        L.synth_key.restype = u64
+        L.synth_draw.argtypes = [u64, u64]
+        L.synth_draw.restype = u64
+        L.synth_normal.argtypes = [u64, u64]
+        L.synth_normal.restype = dbl
+        L.synth_bf16_from_double.argtypes = [dbl]
+        L.synth_bf16_from_double.restype = ctypes.c_uint16
+        L.synth_bytes.argtypes = [u64, u64, u64, vp]
+        L.synth_scales.argtypes = [u64, u64, u64, u32, u32, vp]
+        L.synth_normal_bf16.argtypes = [u64, u64, u64, dbl, vp]
+        L.synth_normal_f64.argtypes = [u64, u64, u64, dbl, vp]
+        L.synth_router_rows.argtypes = [u64, u64, u64, dbl, vp, dbl, vp, vp]
+        L.synth_perturb_bf16.argtypes = [u64, u64, vp, dbl, vp]
+        L.synth_choose.argtypes = [u64, u32, u32, vp]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+# tensor ids of the generator's streams
+T_ROUTER, T_W_DN, T_W_UP = 1, 2, 3
+T_GATE_Q, T_GATE_S, T_UP_Q, T_UP_S, T_DOWN_Q, T_DOWN_S = 4, 5, 6, 7, 8, 9
+T_SH_GATE_Q, T_SH_GATE_S, T_SH_UP_Q, T_SH_UP_S, T_SH_DOWN_Q, T_SH_DOWN_S = 10, 11, 12, 13, 14, 15
+T_X, T_X_NOISE, T_HOT_SET, T_HOT_BIAS = 16, 17, 18, 19
+
+SCALE_LO, SCALE_COUNT = 121, 5  # E8M0 bytes 127 + U{-6..-2}
+
+
+@dataclass(frozen=True)
+class Dims:
+    hidden: int        # H
+    latent: int        # L
+    n_experts: int     # E
+    top_k: int         # k
+    expert_inter: int  # I
+    shared_inter: int  # I_s (one shared expert)
+
+    def expert_bytes(self) -> int:
+        H, L, I = self.hidden, self.latent, self.expert_inter
+        return 2 * (I * L // 2 + I * L // 32) + (L * I // 2 + L * I // 32)
+
+    def fixed_bytes(self) -> int:
+        """Bytes of the weights every step reads whatever the routing: router, W_dn, W_up, shared."""
+        H, L, E, Is = self.hidden, self.latent, self.n_experts, self.shared_inter
+        shared = 2 * (Is * H // 2 + Is * H // 32) + (H * Is // 2 + H * Is // 32)
+        return 2 * (E * H + L * H + H * L) + shared
+
+
+TINY = Dims(hidden=512, latent=256, n_experts=64, top_k=4, expert_inter=256, shared_inter=256)
+FULL = Dims(hidden=7168, latent=2048, n_experts=896, top_k=16, expert_inter=1024, shared_inter=2048)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    dims: Dims
+    batch: int
+    seed: int
+    tokens: str = "normal"        # "normal" | "perturbed" (token b>0 = token 0 + eps*N(0,1))
+    perturb_eps: float = 0.1
+    hot_experts: int = 0          # router rows that get beta * u added
+    hot_beta: float = 0.0
+    layers: int = 1               # distinct seeded layers the bench cycles through
+    description: str = ""
+
+
+# beta for the skewed workload: the first value of the grid 4, 8, 12, ... whose hot share of
+# the 32 layers x 64 tokens x 16 selections (seed 1004) lies in [0.45, 0.55] (it is 0.452);
+# found by tests/golden/calibrate_hot_bias.py and re-checked by tests/test_synth.py.
+HOT_BETA_B64 = 20.0
+
+WORKLOADS = {
+    "tiny_b1": Workload("tiny_b1", TINY, 1, 1000, description="tiny latent-MoE layer, B=1"),
+    "full_b1": Workload("full_b1", FULL, 1, 1001, description="full-size layer, B=1"),
+    "full_b2": Workload("full_b2", FULL, 2, 1002, tokens="perturbed",
+                        description="full-size layer, B=2, token 1 = token 0 + 0.1 N(0,1)"),
+    "full_b16": Workload("full_b16", FULL, 16, 1003, description="full-size layer, B=16, independent tokens"),
+    "full_b64_skewed": Workload("full_b64_skewed", FULL, 64, 1004, hot_experts=32, hot_beta=HOT_BETA_B64,
+                                layers=32, description="full-size layer, B=64, 32 hot experts, 32 layers"),
+}
+
+
+def _normal_bf16(key: int, n: int, sigma: float, start: int = 0) -> np.ndarray:
+    out = np.empty(n, dtype=np.uint16)
+    lib().synth_normal_bf16(key, start, n, sigma, _ptr(out))
+    return out
+
+
+def _bytes(key: int, n: int, start: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+    if out is None:
+        out = np.empty(n, dtype=np.uint8)
+    lib().synth_bytes(key, start, n, _ptr(out))
+    return out
+
+
+def _scales(key: int, n: int, start: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+    if out is None:
+        out = np.empty(n, dtype=np.uint8)
+    lib().synth_scales(key, start, n, SCALE_LO, SCALE_COUNT, _ptr(out))
+    return out
+
+
+def hot_set(w: Workload, layer: int) -> np.ndarray:
+    """Sorted indices of the hot experts of one layer (empty if the workload has none)."""
+    if w.hot_experts == 0:
+        return np.zeros(0, dtype=np.int64)
+    E = w.dims.n_experts
+    perm = np.empty(E, dtype=np.uint32)
+    lib().synth_choose(lib().synth_key(w.seed, layer, T_HOT_SET), E, w.hot_experts, _ptr(perm))
+    return np.sort(perm[: w.hot_experts].astype(np.int64))
+
+
+def router_weights(w: Workload, layer: int, beta: float | None = None) -> np.ndarray:
+    """Router rows, bf16 bits [E, H]; hot rows carry beta * u (u ~ N(0,1/H), one vector per layer)."""
+    d = w.dims
+    E, H = d.n_experts, d.hidden
+    beta = w.hot_beta if beta is None else beta
+    out = np.empty((E, H), dtype=np.uint16)
+    key = lib().synth_key(w.seed, layer, T_ROUTER)
+    hot = np.zeros(E, dtype=np.uint8)
+    bias = np.zeros(H, dtype=np.float64)
+    if w.hot_experts:
+        hot[hot_set(w, layer)] = 1
+        lib().synth_normal_f64(lib().synth_key(w.seed, layer, T_HOT_BIAS), 0, H, 1.0 / np.sqrt(H), _ptr(bias))
+    lib().synth_router_rows(key, E, H, 1.0 / np.sqrt(H), _ptr(hot), float(beta), _ptr(bias), _ptr(out))
+    return out
+
+
+def layer_weights(w: Workload, layer: int = 0, beta: float | None = None) -> dict:
+    """All weights of one layer as numpy arrays (bf16 as uint16 bits, MXFP4 as uint8).
+
+    Layout (row-major): router [E,H]; w_down_lat [L,H]; w_up_lat [H,L];
+    gate/up codes [E,I,L/2] + scales [E,I,L/32]; down codes [E,L,I/2] + scales [E,L,I/32];
+    shared gate/up codes [I_s,H/2] + scales [I_s,H/32]; shared down [H,I_s/2] + [H,I_s/32].
+    Packed FP4: element 2j in the low nibble of byte j, element 2j+1 in the high nibble.
+    """
+    d = w.dims
+    H, L, E, I, Is = d.hidden, d.latent, d.n_experts, d.expert_inter, d.shared_inter
+    k = lambda t: lib().synth_key(w.seed, layer, t)
+    W = {}
+    W["router"] = router_weights(w, layer, beta)
+    W["w_down_lat"] = _normal_bf16(k(T_W_DN), L * H, 1.0 / np.sqrt(H)).reshape(L, H)
+    W["w_up_lat"] = _normal_bf16(k(T_W_UP), H * L, 1.0 / np.sqrt(L)).reshape(H, L)
+    W["gate_q"] = _bytes(k(T_GATE_Q), E * I * L // 2).reshape(E, I, L // 2)
+    W["gate_s"] = _scales(k(T_GATE_S), E * I * L // 32).reshape(E, I, L // 32)
+    W["up_q"] = _bytes(k(T_UP_Q), E * I * L // 2).reshape(E, I, L // 2)
+    W["up_s"] = _scales(k(T_UP_S), E * I * L // 32).reshape(E, I, L // 32)
+    W["down_q"] = _bytes(k(T_DOWN_Q), E * L * I // 2).reshape(E, L, I // 2)
+    W["down_s"] = _scales(k(T_DOWN_S), E * L * I // 32).reshape(E, L, I // 32)
+    W["sh_gate_q"] = _bytes(k(T_SH_GATE_Q), Is * H // 2).reshape(Is, H // 2)
+    W["sh_gate_s"] = _scales(k(T_SH_GATE_S), Is * H // 32).reshape(Is, H // 32)
+    W["sh_up_q"] = _bytes(k(T_SH_UP_Q), Is * H // 2).reshape(Is, H // 2)
+    W["sh_up_s"] = _scales(k(T_SH_UP_S), Is * H // 32).reshape(Is, H // 32)
+    W["sh_down_q"] = _bytes(k(T_SH_DOWN_Q), H * Is // 2).reshape(H, Is // 2)
+    W["sh_down_s"] = _scales(k(T_SH_DOWN_S), H * Is // 32).reshape(H, Is // 32)
+    return W
+
+
+WEIGHT_NAMES = ("router", "w_down_lat", "w_up_lat", "gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s",
+                "sh_gate_q", "sh_gate_s", "sh_up_q", "sh_up_s", "sh_down_q", "sh_down_s")
+
+
+def tokens(w: Workload, step: int = 0, batch: int | None = None) -> np.ndarray:
+    """Decode-step activations x, bf16 bits [B, H] ~ N(0,1).  `step` selects a fresh draw."""
+    d = w.dims
+    B = w.batch if batch is None else batch
+    H = d.hidden
+    key = lib().synth_key(w.seed, 1_000_000 + step, T_X)
+    if w.tokens == "normal":
+        return _normal_bf16(key, B * H, 1.0).reshape(B, H)
+    x = np.empty((B, H), dtype=np.uint16)
+    x[0] = _normal_bf16(key, H, 1.0)
+    for b in range(1, B):
+        nk = lib().synth_key(w.seed, 1_000_000 + step, T_X_NOISE + 100 * b)
+        lib().synth_perturb_bf16(nk, H, _ptr(x[0]), w.perturb_eps, _ptr(x[b]))
+    return x
+
+
+def bf16_to_f32(a: np.ndarray) -> np.ndarray:
+    """bf16 bits (uint16) -> float32 values (exact)."""
+    return (a.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16(a: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bits, round to nearest even."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
