@@ -1,0 +1,389 @@
+#!/usr/bin/env python3
+"""Benchmark of the sparse latent-MoE decode layer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one decode layer step (router, top-k, latent down-projection, routed MXFP4 experts,
+combine, up-projection, shared expert) for one batch of tokens.  The timed region replays a
+CUDA graph of exactly K steps that cycles through `--layers` layers of distinct seeded weights
+(32 by default, ~99 GB), so every step streams its weights from HBM: the per-step working set
+(>= 148 MB) exceeds the 126 MB L2 and the same layer returns only after 31 others.  Rank 0
+prints one JSON line.  Under torchrun every rank runs an independent replica (the step does
+not shard; no collective touches the data path); value = all ranks' steps / max time.
+
+--impl reference times the CPU oracle (the plain fp64 C implementation) on this host's cores
+for a bounded sample of the same workload; it is the baseline the driver divides by.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE layer-steps/s & µs/step at B=1..64; achieved HBM GB/s vs B200 peak"
+UNIT = "layer-steps/s"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="full_b1", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--layers", type=int, default=0, help="distinct layers cycled through (default 32)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
+    return p.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# byte accounting (algorithmic bytes: every weight byte the step must read once, plus tokens)
+
+def kernel_bytes(d: synth.Dims, unique_experts: float, B: int) -> dict:
+    H, L, E, I, Is = d.hidden, d.latent, d.n_experts, d.expert_inter, d.shared_inter
+    fp4 = lambda n, k: n * k // 2 + n * k // 32
+    return {
+        "router_dn": 2 * E * H + 2 * L * H + 2 * B * H,
+        "topk": 4 * B * E,
+        "expert_gate_up": unique_experts * 2 * fp4(I, L),
+        "expert_down": unique_experts * fp4(L, I),
+        "combine": 4 * B * d.top_k * L,
+        "up": 2 * H * L + 2 * B * H,
+        "shared_gate_up": 2 * fp4(Is, H),
+        "shared_down": fp4(H, Is),
+    }
+
+
+def step_bytes(d: synth.Dims, unique_experts: float, B: int) -> float:
+    """Algorithmic HBM bytes of one step: fixed weights + touched experts + tokens in and out."""
+    return d.fixed_bytes() + unique_experts * d.expert_bytes() + 2 * 2 * B * d.hidden
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks during the timed region
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    rows.append(f)
+        except OSError:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        busy = [s for s in sm if smax and s > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = json.load(open(p))["hbm_gbs"]
+        return float(v), "measured (MEASURED_PEAKS.json hbm_gbs, copy)"
+    except Exception:
+        return 6650.0, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle timing (the baseline; also the reference arm)
+
+def cpu_oracle_rate(w: synth.Workload, seconds: float):
+    import oracle
+    W = synth.layer_weights(w, 0)
+    x = synth.tokens(w)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.step(w.dims, W, x)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n} oracle steps of {w.name} layer 0 (B={w.batch}, all {w.batch} tokens), {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    w = synth.WORKLOADS[args.workload]
+    import oracle
+    W = synth.layer_weights(w, 0)
+    x = synth.tokens(w)
+    t0 = time.perf_counter()
+    for _ in range(max(args.warmup, 1)):
+        oracle.step(w.dims, W, x)
+    est = (time.perf_counter() - t0) / max(args.warmup, 1)
+    # bounded sample: at most ~150 s of timed oracle steps whatever K is
+    n = max(1, min(args.steps, int(150.0 / max(est, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        oracle.step(w.dims, W, x)
+    dt = time.perf_counter() - t0
+    v = n / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": n,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "layers": 1},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": f"{n} timed oracle steps (of {args.steps} requested, capped at ~150 s) of "
+                                       f"{w.name} layer 0 after {args.warmup} warm-up"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# our arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    rank, local_rank, world = dist_env()
+    import torch
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    from moe_decode_layer_moedec_b200 import FLAG_SKIP_SCALE_CHECK, LayerDims, MoeDecodeLayer
+
+    w = synth.WORKLOADS[args.workload]
+    d = w.dims
+    B = w.batch
+    n_layers = args.layers or (32 if d is synth.FULL else 4)
+    dims = LayerDims(d.hidden, d.latent, d.n_experts, d.top_k, d.expert_inter, d.shared_inter, 1)
+
+    # weights of n_layers distinct layers, resident in HBM (created once, outside any timing)
+    t0 = time.time()
+    layers, dev_weights = [], []
+    for l in range(n_layers):
+        W = synth.layer_weights(w, l)
+        Wd = {}
+        for k, v in W.items():
+            t = torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v)
+            Wd[k] = t.to(f"cuda:{local_rank}", non_blocking=False)
+        del W
+        flags = 0 if l == 0 else FLAG_SKIP_SCALE_CHECK  # layer 0 runs the create-time scale scan
+        layers.append(MoeDecodeLayer(dims, Wd, max_batch=B, flags=flags))
+        dev_weights.append(Wd)
+        if rank == 0 and (l % 8 == 7 or l == n_layers - 1):
+            log(f"[bench] {l + 1}/{n_layers} layers resident ({time.time() - t0:.0f} s)")
+    x_host = torch.from_numpy(synth.tokens(w).view(np.int16)).pin_memory()
+    x = x_host.to(f"cuda:{local_rank}")
+    out = torch.empty_like(x)
+    stream = torch.cuda.Stream()
+
+    # routing of every layer (outside the timed region) -> unique experts touched per step
+    uniq = []
+    with torch.cuda.stream(stream):
+        for L_ in layers:
+            L_.step(x, out=out, stream=stream)
+            idx, _ = L_.routing(B, stream=stream)
+            uniq.append(len(np.unique(idx.cpu().numpy())))
+    torch.cuda.synchronize()
+    unique_mean = float(np.mean(uniq))
+
+    def capture(n_steps, first):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            for i in range(n_steps):
+                layers[(first + i) % n_layers].step(x, out=out, stream=stream)
+        return g
+
+    # eager warm-up (module load, caches) then the graphs
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            layers[i % n_layers].step(x, out=out, stream=stream)
+    torch.cuda.synchronize()
+    g_warm = capture(max(args.warmup, 1), 0)
+    g_main = capture(args.steps, args.warmup)
+    for L_ in layers:
+        L_.profile(True)
+    g_prof = capture(args.steps, args.warmup)
+    for L_ in layers:
+        L_.profile(False)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g_warm.replay()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        with torch.cuda.stream(stream):
+            g_main.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    clocks = clk.summary()
+    if dist:
+        t = torch.tensor([ms], device=f"cuda:{local_rank}", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * args.steps / (ms / 1e3)
+
+    # per-kernel durations: a second replay of the same K steps with an event pair around every
+    # kernel on the stream it runs on (main or side stream)
+    g_warm.replay()
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        g_prof.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms_prof = ev0.elapsed_time(ev1)
+    per_kernel = {}
+    for L_ in layers:
+        for name, (kms, n) in L_.profile_read().items():
+            a, b = per_kernel.get(name, (0.0, 0))
+            per_kernel[name] = (a + kms, b + n)
+    kb = kernel_bytes(d, unique_mean, B)
+    peak, peak_src = measured_peak_hbm()
+    dom = max(per_kernel, key=lambda k: per_kernel[k][0])
+    dom_ms, dom_n = per_kernel[dom]
+    dom_avg_s = dom_ms / 1e3 / max(dom_n, 1)
+    achieved = kb[dom] / dom_avg_s / 1e9
+    kernels_table = {k: {"avg_us": 1e3 * v[0] / max(v[1], 1), "launches": v[1],
+                         "share": v[0] / max(sum(x[0] for x in per_kernel.values()), 1e-12),
+                         "gbs": kb[k] / (v[0] / 1e3 / max(v[1], 1)) / 1e9 if v[0] > 0 else None}
+                     for k, v in per_kernel.items()}
+
+    # end to end through the public API: pinned host tokens in, step, result back to pinned host
+    out_host = torch.empty_like(x_host).pin_memory()
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            x.copy_(x_host, non_blocking=True)
+            layers[i % n_layers].step(x, out=out, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            x.copy_(x_host, non_blocking=True)
+            layers[i % n_layers].step(x, out=out, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=f"cuda:{local_rank}", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * args.steps / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_rate(w, args.cpu_seconds)
+
+    sb = step_bytes(d, unique_mean, B)
+    kps = layers[0].kernels_per_step(B)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "hidden": d.hidden, "latent": d.latent, "experts": d.n_experts,
+                       "top_k": d.top_k, "layers_cycled": n_layers, "unique_experts_per_step": unique_mean,
+                       "l2": "inputs larger than L2: each step streams one of %d distinct layers (>= 148 MB)" % n_layers,
+                       "arith": "MXFP4/bf16 weights, fp16/bf16 tensor-core MMA with fp32 accumulation, fp64 router",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "us_per_step": 1e3 * ms_per_step,
+            "step_hbm": {"bytes_per_step": sb, "gbs": sb / (ms_per_step / 1e3) / 1e9,
+                         "frac": sb / (ms_per_step / 1e3) / 1e9 / peak, "peak_gbs": peak, "peak": peak_src},
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x_host.numel() * 2),
+                    "d2h_bytes_per_step": int(out_host.numel() * 2)},
+            "gpu_launches": kps * args.steps,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "bytes_per_launch": kb[dom],
+                         "avg_launch_us": dom_avg_s * 1e6, "peak_source": peak_src},
+            "kernels": kernels_table,
+            "profiled_pass_ms_per_step": ms_prof / args.steps,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    del g_main, g_prof, g_warm
+    for L_ in layers:
+        L_.close()
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

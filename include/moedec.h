@@ -1,0 +1,179 @@
+/*
+ * moedec.h -- C ABI of the B200 (sm_100a) sparse latent-MoE decode layer step.
+ *
+ * The operation.  One decode step of one MoE layer of a Kimi-K3-shaped model: E routed
+ * experts with top-k active per token, MXFP4 expert weights, a latent space of width L
+ * below the hidden width H, and one always-on shared expert.  Kimi K3 has 896 experts with
+ * 16 active per token and stores its weights as MXFP4 ("快是可以生成的，可信只能证明（vLLM
+ * 重写 Kimi K3 解码路径，以及怎么放心合并 Agent 写的内核）", section 为什么一条请求会慢).
+ * The step's parts -- router scoring, the latent projection, the routed experts, the shared
+ * expert on its own stream -- are the ones that page lists (section 他们换掉了什么), and
+ * decode at small batch is bounded by streaming the weights from HBM (same page, section
+ * 为什么一条请求会慢; "NVIDIA uses a 12,000-line Megakernel to optimize Kimi K3 inference…",
+ * section 为什么解码优化比训练优化更难).  For tokens x[b] (bf16, width H):
+ *
+ *   logit[b,e] = fp32( sum_j R[e,j] x[b,j] )    exact products, fp64 accumulation
+ *   s[b,e]     = fp32( 1 / (1 + exp(-logit)) )  (evaluated in fp64)
+ *   idx[b,:]   = the top_k experts by s, the lower index first among equal s
+ *   w[b,r]     = s_r / (fp32 sum of the k selected s, in rank order)
+ *   h          = W_dn x[b]                       (H -> L)
+ *   ylat       = sum_r w[b,r] * D_e( silu(G_e h) * (U_e h) ),  e = idx[b,r]
+ *   out[b]     = bf16( W_up ylat + SD( silu(SG x[b]) * (SU x[b]) ) )   (L -> H, one rounding)
+ *
+ * Number formats.  bf16 values are passed as their 16-bit patterns (uint16_t).  An MXFP4
+ * matrix [N, K] (OCP Microscaling Formats v1.0) is two arrays: codes uint8 [N][K/2], element
+ * 2j in the low nibble of byte j and 2j+1 in the high nibble, and E8M0 scale bytes uint8
+ * [N][K/32], one per 32-element block along K; element = E2M1(code) * 2^(scale - 127).
+ *
+ * Conventions for every call:
+ *   - Every pointer is a CUDA device pointer unless the argument says "host".
+ *   - Arrays are dense and row-major; every weight pointer is 16-byte aligned.
+ *   - A stream argument is a cudaStream_t passed as void*; NULL is the legacy default stream.
+ *   - Calls return MOEDEC_OK (0) or a negative moedec_status; they never abort the process.
+ *   - A handle is not thread-safe: one host thread at a time, one step in flight per handle
+ *     (steps of one handle issued on one stream are ordered by that stream).
+ */
+#ifndef MOEDEC_H
+#define MOEDEC_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define MOEDEC_API __declspec(dllexport)
+#else
+#define MOEDEC_API __attribute__((visibility("default")))
+#endif
+
+#define MOEDEC_ABI_VERSION 1
+
+typedef enum moedec_status {
+    MOEDEC_OK = 0,
+    MOEDEC_ERR_INVALID_ARG = -1,  /* NULL handle/pointer, misaligned pointer, batch < 0, bad abi_version */
+    MOEDEC_ERR_UNSUPPORTED = -2,  /* dimensions or batch outside what this build handles (see moedec_create) */
+    MOEDEC_ERR_CUDA = -3,         /* a CUDA runtime call failed; the CUDA error is kept in the handle */
+    MOEDEC_ERR_OOM = -4,          /* workspace allocation failed */
+    MOEDEC_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (reported by the next call) */
+    MOEDEC_ERR_DEVICE = -6        /* a kernel recorded an internal error word (reported by the next call) */
+} moedec_status;
+
+/* Config flags. */
+#define MOEDEC_FLAG_TAPS 1u            /* also materialise the fp32 `up` tap (W_up ylat) for tests */
+#define MOEDEC_FLAG_SKIP_SCALE_CHECK 2u /* skip moedec_create's scan of the E8M0 scale bytes */
+
+typedef struct moedec_config {
+    int32_t abi_version;  /* MOEDEC_ABI_VERSION */
+    int32_t hidden;       /* H: multiple of 128 */
+    int32_t latent;       /* L: multiple of 128 */
+    int32_t n_experts;    /* E: 1..1024 */
+    int32_t top_k;        /* k: 1..min(E, 32) */
+    int32_t expert_inter; /* I: multiple of 128 */
+    int32_t shared_inter; /* I_s: multiple of 128 (ignored when n_shared == 0) */
+    int32_t n_shared;     /* 0 or 1 shared expert */
+    int32_t max_batch;    /* largest B a step will be called with: 1..64 */
+    uint32_t flags;       /* MOEDEC_FLAG_* */
+} moedec_config;
+
+/*
+ * Weights of one layer.  All device pointers, borrowed: the caller keeps them alive and
+ * unchanged for the handle's lifetime (they are read with non-coherent loads).  Shapes:
+ *   router     bf16 [E][H]          w_down_lat bf16 [L][H]        w_up_lat bf16 [H][L]
+ *   gate_q/up_q    [E][I][L/2]      gate_s/up_s    [E][I][L/32]
+ *   down_q         [E][L][I/2]      down_s         [E][L][I/32]
+ *   sh_gate_q/sh_up_q [I_s][H/2]    sh_gate_s/sh_up_s [I_s][H/32]
+ *   sh_down_q      [H][I_s/2]       sh_down_s      [H][I_s/32]
+ * The sh_* pointers may be NULL when n_shared == 0.
+ */
+typedef struct moedec_weights {
+    const uint16_t *router, *w_down_lat, *w_up_lat;
+    const uint8_t *gate_q, *gate_s, *up_q, *up_s, *down_q, *down_s;
+    const uint8_t *sh_gate_q, *sh_gate_s, *sh_up_q, *sh_up_s, *sh_down_q, *sh_down_s;
+} moedec_weights;
+
+typedef struct moedec_handle moedec_handle;
+
+/*
+ * Create a handle for one layer on the current CUDA device.
+ *   cfg, w      host pointers to the config and the weight-pointer table (copied).
+ *   out         host pointer that receives the new handle (set to NULL on failure).
+ * Allocates the step workspace for cfg->max_batch tokens, a side stream and two events.
+ * Unless MOEDEC_FLAG_SKIP_SCALE_CHECK is set it scans every E8M0 scale byte once (one device
+ * kernel and one synchronisation): the tensor-core expert kernels fold the block scale into
+ * fp16 weights, which is exact for scale bytes 104..140 (2^-23 .. 2^13); any byte outside that
+ * range gives MOEDEC_ERR_UNSUPPORTED.
+ * Errors: INVALID_ARG (NULL, misaligned, abi_version), UNSUPPORTED (dimensions), OOM, CUDA.
+ */
+MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, moedec_handle **out);
+
+/*
+ * One layer step: out[b] for b < batch from x[b].
+ *   x       bf16 [batch][H], device, 16-byte aligned; read only.
+ *   batch   0..max_batch (0 is a no-op that still reports pending device errors).
+ *   out     bf16 [batch][H], device, 16-byte aligned; must not overlap x.
+ *   stream  the caller's stream; all work is ordered after prior work on it and the call
+ *           returns without synchronising.  Work also runs on the handle's side stream,
+ *           forked from and joined back into `stream` with events, so the step can be
+ *           captured into a CUDA graph on `stream`.
+ * Errors: INVALID_ARG, UNSUPPORTED (batch > max_batch), CUDA (launch failure).  Errors that
+ * kernels record on the device (TIMEOUT/DEVICE) are reported by the next synchronising call,
+ * moedec_get_routing or moedec_get_taps, which also clear them.
+ */
+MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint16_t *out, void *stream);
+
+/* Release the workspace, side stream and events (synchronises the side stream). NULL is a no-op. */
+MOEDEC_API int moedec_destroy(moedec_handle *h);
+
+/*
+ * Routing of the last step, copied on `stream` into caller device buffers:
+ *   idx  int32 [batch][top_k] expert indices in rank order (score descending, lower index first)
+ *   w    fp32  [batch][top_k] routing weights in the same order
+ * Either pointer may be NULL.  batch must equal the last step's batch.  Synchronises `stream`
+ * and reports (then clears) any device-side error word of earlier steps: TIMEOUT or DEVICE.
+ */
+MOEDEC_API int moedec_get_routing(moedec_handle *h, int32_t *idx, float *w, int batch, void *stream);
+
+/*
+ * Intermediate values of the last step (test taps), copied on `stream` into caller device buffers:
+ *   logits fp32 [batch][E]   h    fp32 [batch][L]   ylat fp32 [batch][L]
+ *   sh     fp32 [batch][H]   up   fp32 [batch][H] (W_up ylat; only with MOEDEC_FLAG_TAPS)
+ * Any pointer may be NULL.  `up` non-NULL without MOEDEC_FLAG_TAPS gives INVALID_ARG.
+ * Synchronises `stream` and reports device-side errors like moedec_get_routing.
+ */
+MOEDEC_API int moedec_get_taps(moedec_handle *h, float *logits, float *hlat, float *ylat, float *sh, float *up,
+                               int batch, void *stream);
+
+/*
+ * Launch counters (host values): launches[i] counts the kernels of variant i issued by this
+ * handle since creation; i = 0 SMALL (batch <= 2), 1 SPLITK (batch >= 3).  n_variants in/out.
+ */
+MOEDEC_API int moedec_get_launch_counts(moedec_handle *h, uint64_t *launches, int *n_variants);
+
+/* Kernels issued per step by the current build (so a timed loop can count its launches). */
+MOEDEC_API int moedec_kernels_per_step(moedec_handle *h, int batch);
+
+/* Last CUDA error string recorded by the handle ("" if none); static storage of the handle. */
+MOEDEC_API const char *moedec_last_cuda_error(moedec_handle *h);
+
+/*
+ * Per-kernel timing.  While enabled, every kernel a step launches is bracketed by a pair of CUDA
+ * events recorded on the stream that kernel runs on (the caller's stream or the side stream).
+ * moedec_profile_read synchronises both streams and returns, per kernel kind i < *n:
+ *   total_ms[i]  summed event-measured duration of its launches since enabling (host array)
+ *   launches[i]  number of its launches (host array)
+ *   names[i]     static name of the kind (host array of const char*), may be NULL
+ * *n is in/out (array capacity in, number of kinds out).  Enabling again resets the sums.
+ */
+MOEDEC_API int moedec_profile_enable(moedec_handle *h, int enable);
+MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t *launches, const char **names, int *n);
+
+/* Human-readable name of a status code (static storage). */
+MOEDEC_API const char *moedec_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEDEC_H */

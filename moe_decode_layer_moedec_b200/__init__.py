@@ -1,0 +1,202 @@
+"""Python binding of libmoedec.so, the B200 (sm_100a) sparse latent-MoE decode layer step.
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.  PyTorch
+is used for device memory and streams.  There is no CPU path: if the shared library is missing
+or cannot be loaded, importing this package raises.
+
+    layer = MoeDecodeLayer(dims, weights, max_batch=64)   # weights: dict of CUDA tensors
+    out = layer.step(x)                                   # x: bf16 [B, H] on the same device
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoedec.so")
+
+ABI_VERSION = 1
+FLAG_TAPS = 1
+FLAG_SKIP_SCALE_CHECK = 2
+STATUS = {0: "MOEDEC_OK", -1: "MOEDEC_ERR_INVALID_ARG", -2: "MOEDEC_ERR_UNSUPPORTED", -3: "MOEDEC_ERR_CUDA",
+          -4: "MOEDEC_ERR_OOM", -5: "MOEDEC_ERR_TIMEOUT", -6: "MOEDEC_ERR_DEVICE"}
+WEIGHT_NAMES = ("router", "w_down_lat", "w_up_lat", "gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s",
+                "sh_gate_q", "sh_gate_s", "sh_up_q", "sh_up_s", "sh_down_q", "sh_down_s")
+
+
+class MoedecError(RuntimeError):
+    def __init__(self, call: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{call} failed: {STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("abi_version", ctypes.c_int32), ("hidden", ctypes.c_int32), ("latent", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("expert_inter", ctypes.c_int32),
+                ("shared_inter", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("max_batch", ctypes.c_int32),
+                ("flags", ctypes.c_uint32)]
+
+
+class _Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_NAMES]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with `python -m moe_decode_layer_moedec_b200.build` "
+                          "(nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    lib.moedec_create.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), ctypes.POINTER(vp)]
+    lib.moedec_create.restype = i32
+    lib.moedec_step.argtypes = [vp, vp, i32, vp, vp]
+    lib.moedec_step.restype = i32
+    lib.moedec_destroy.argtypes = [vp]
+    lib.moedec_destroy.restype = i32
+    lib.moedec_get_routing.argtypes = [vp, vp, vp, i32, vp]
+    lib.moedec_get_routing.restype = i32
+    lib.moedec_get_taps.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp]
+    lib.moedec_get_taps.restype = i32
+    lib.moedec_get_launch_counts.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(i32)]
+    lib.moedec_get_launch_counts.restype = i32
+    lib.moedec_profile_enable.argtypes = [vp, i32]
+    lib.moedec_profile_enable.restype = i32
+    lib.moedec_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64),
+                                        ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(i32)]
+    lib.moedec_profile_read.restype = i32
+    lib.moedec_kernels_per_step.argtypes = [vp, i32]
+    lib.moedec_kernels_per_step.restype = i32
+    lib.moedec_last_cuda_error.argtypes = [vp]
+    lib.moedec_last_cuda_error.restype = ctypes.c_char_p
+    lib.moedec_status_string.argtypes = [i32]
+    lib.moedec_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+lib = _load()
+
+
+@dataclass(frozen=True)
+class LayerDims:
+    hidden: int
+    latent: int
+    n_experts: int
+    top_k: int
+    expert_inter: int
+    shared_inter: int
+    n_shared: int = 1
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+class MoeDecodeLayer:
+    """One MoE layer's decode step on the current CUDA device (a moedec handle).
+
+    `weights` maps the names in WEIGHT_NAMES to contiguous CUDA tensors: bf16 matrices as
+    torch.bfloat16 or torch.uint16/int16 bit patterns, MXFP4 codes and E8M0 scales as uint8.
+    The tensors are borrowed: keep them alive and unchanged while the layer exists.
+    """
+
+    def __init__(self, dims: LayerDims, weights: dict, max_batch: int, flags: int = 0):
+        self.dims = dims
+        self.max_batch = max_batch
+        self.flags = flags
+        self._weights = {n: weights.get(n) for n in WEIGHT_NAMES}  # keep the tensors alive
+        for n, t in self._weights.items():
+            if t is not None and not t.is_contiguous():
+                raise ValueError(f"weight {n} must be contiguous")
+        cfg = _Config(ABI_VERSION, dims.hidden, dims.latent, dims.n_experts, dims.top_k, dims.expert_inter,
+                      dims.shared_inter, dims.n_shared, max_batch, flags)
+        w = _Weights(*[_ptr(self._weights[n]) for n in WEIGHT_NAMES])
+        h = ctypes.c_void_p()
+        rc = lib.moedec_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))
+        if rc != 0:
+            raise MoedecError("moedec_create", rc)
+        self._h = h
+
+    def _check(self, call: str, rc: int):
+        if rc != 0:
+            detail = lib.moedec_last_cuda_error(self._h).decode() if self._h else ""
+            raise MoedecError(call, rc, detail)
+
+    def step(self, x, out=None, stream=None):
+        """out[b] = layer(x[b]) for x bf16 [B, H] on the device; asynchronous on `stream`."""
+        import torch
+        B = x.shape[0]
+        if out is None:
+            out = torch.empty((B, self.dims.hidden), dtype=x.dtype, device=x.device)
+        assert x.is_contiguous() and out.is_contiguous()
+        self._check("moedec_step", lib.moedec_step(self._h, _ptr(x), B, _ptr(out), _stream_ptr(stream)))
+        return out
+
+    def step_ptr(self, x_ptr: int, batch: int, out_ptr: int, stream_ptr: int):
+        self._check("moedec_step", lib.moedec_step(self._h, x_ptr, batch, out_ptr, stream_ptr))
+
+    def routing(self, batch: int, stream=None):
+        """(idx int32 [B, k], w fp32 [B, k]) of the last step, in rank order."""
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        idx = torch.empty((batch, self.dims.top_k), dtype=torch.int32, device=dev)
+        w = torch.empty((batch, self.dims.top_k), dtype=torch.float32, device=dev)
+        self._check("moedec_get_routing", lib.moedec_get_routing(self._h, _ptr(idx), _ptr(w), batch, _stream_ptr(stream)))
+        return idx, w
+
+    def taps(self, batch: int, stream=None) -> dict:
+        """fp32 intermediates of the last step: logits [B,E], h/ylat [B,L], sh (and up with FLAG_TAPS) [B,H]."""
+        import torch
+        d = self.dims
+        dev = torch.device("cuda", torch.cuda.current_device())
+        f = lambda *s: torch.empty(s, dtype=torch.float32, device=dev)
+        r = dict(logits=f(batch, d.n_experts), h=f(batch, d.latent), ylat=f(batch, d.latent), sh=f(batch, d.hidden))
+        if self.flags & FLAG_TAPS:
+            r["up"] = f(batch, d.hidden)
+        self._check("moedec_get_taps", lib.moedec_get_taps(self._h, _ptr(r["logits"]), _ptr(r["h"]), _ptr(r["ylat"]),
+                                                           _ptr(r["sh"]), _ptr(r.get("up")), batch, _stream_ptr(stream)))
+        return r
+
+    def launch_counts(self):
+        arr = (ctypes.c_uint64 * 2)()
+        n = ctypes.c_int(2)
+        self._check("moedec_get_launch_counts", lib.moedec_get_launch_counts(self._h, arr, ctypes.byref(n)))
+        return {"small": int(arr[0]), "splitk": int(arr[1])}
+
+    def profile(self, enable: bool = True):
+        """Bracket every kernel of later steps with CUDA events on its own stream (resets the sums)."""
+        self._check("moedec_profile_enable", lib.moedec_profile_enable(self._h, 1 if enable else 0))
+
+    def profile_read(self) -> dict:
+        """{kernel name: (total ms, launches)} since profile(True); synchronises."""
+        cap = 16
+        ms = (ctypes.c_double * cap)()
+        cnt = (ctypes.c_uint64 * cap)()
+        names = (ctypes.c_char_p * cap)()
+        n = ctypes.c_int(cap)
+        self._check("moedec_profile_read", lib.moedec_profile_read(self._h, ms, cnt, names, ctypes.byref(n)))
+        return {names[i].decode(): (float(ms[i]), int(cnt[i])) for i in range(n.value)}
+
+    def kernels_per_step(self, batch: int) -> int:
+        return int(lib.moedec_kernels_per_step(self._h, batch))
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib.moedec_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

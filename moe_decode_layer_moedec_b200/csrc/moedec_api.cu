@@ -1,0 +1,396 @@
+// moedec_api.cu -- the C ABI: argument checks, workspace, side stream, launch order.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/moedec.h"
+#include "moedec_internal.h"
+
+using namespace moedec;
+
+struct moedec_handle {
+    moedec_config cfg;
+    Dims d;
+    Weights w;
+    Plan p;
+    Work ws;
+    void *buf = nullptr;
+    size_t buf_bytes = 0;
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    int device = 0, n_sm = 0;
+    int last_batch = 0;
+    uint64_t launches[2] = {0, 0};
+    char cuda_error[256] = {0};
+    // per-kernel event timing (moedec_profile_enable)
+    bool profiling = false;
+    struct Mark {
+        int kind;
+        cudaEvent_t start, stop;
+    };
+    std::vector<Mark> marks;      // recorded, not yet read
+    std::vector<cudaEvent_t> pool;  // free events
+    double prof_ms[16] = {0};
+    uint64_t prof_n[16] = {0};
+};
+
+namespace {
+
+int record_cuda(moedec_handle *h, cudaError_t e) {
+    if (e == cudaSuccess) return MOEDEC_OK;
+    if (h) snprintf(h->cuda_error, sizeof(h->cuda_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return e == cudaErrorMemoryAllocation ? MOEDEC_ERR_OOM : MOEDEC_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int krange_for(int K) { return K % 512 == 0 ? 512 : K % 256 == 0 ? 256 : 128; }
+
+SplitPlan split(int rows, int rows_per_block, int K) {
+    SplitPlan s;
+    s.blocks = (rows + rows_per_block - 1) / rows_per_block;
+    s.krange = krange_for(K);
+    s.splits = K / s.krange;
+    return s;
+}
+
+// carve aligned sub-buffers from one allocation
+struct Carver {
+    char *base;
+    size_t off = 0;
+    template <class T>
+    T *take(size_t n) {
+        off = (off + 255) & ~(size_t)255;
+        T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += n * sizeof(T);
+        return p;
+    }
+};
+
+void layout(moedec_handle *h, char *base) {
+    const Dims &d = h->d;
+    const size_t B = (size_t)d.max_batch;
+    const Plan &p = h->p;
+    Carver c{base};
+    Work &w = h->ws;
+    w.rt_part = c.take<double>((size_t)p.rt.splits * B * d.E);
+    w.logits = c.take<float>(B * d.E);
+    w.dn_part = c.take<float>((size_t)p.dn.splits * B * d.L);
+    w.h = c.take<float>(B * d.L);
+    w.h_shift = c.take<int>(B);
+    w.idx = c.take<int>(B * d.k);
+    w.wts = c.take<float>(B * d.k);
+    w.n_active = c.take<int>(1);
+    w.active_e = c.take<int>(d.E);
+    w.active_cnt = c.take<int>(d.E);
+    w.active_off = c.take<int>(d.E);
+    w.entries = c.take<int>(B * d.k);
+    w.a = c.take<float>(B * d.k * d.I);
+    w.a_amax = c.take<unsigned>(B * d.k);
+    w.y = c.take<float>(B * d.k * d.L);
+    w.ylat = c.take<float>(B * d.L);
+    w.sgu_part = c.take<float>((size_t)p.sgu.splits * B * 2 * d.Is);
+    w.sh_a = c.take<float>(B * d.Is);
+    w.sd_part = c.take<float>((size_t)p.sd.splits * B * d.H);
+    w.sh = c.take<float>(B * d.H);
+    w.up_part = c.take<float>((size_t)p.up.splits * B * d.H);
+    w.up_tap = (h->cfg.flags & MOEDEC_FLAG_TAPS) ? c.take<float>(B * d.H) : nullptr;
+    w.tickets = c.take<unsigned>((size_t)p.n_tickets);
+    w.err = c.take<unsigned>(1);
+    h->buf_bytes = c.off;
+}
+
+int check_scales(moedec_handle *h) {
+    const Dims &d = h->d;
+    unsigned *bad = nullptr;
+    cudaError_t e = cudaMalloc(&bad, sizeof(unsigned));
+    if (e != cudaSuccess) return record_cuda(h, e);
+    struct {
+        const uint8_t *p;
+        size_t n;
+    } arrs[] = {
+        {h->w.gate_s, (size_t)d.E * d.I * (d.L / 32)}, {h->w.up_s, (size_t)d.E * d.I * (d.L / 32)},
+        {h->w.down_s, (size_t)d.E * d.L * (d.I / 32)}, {h->w.sh_gate_s, d.n_shared ? (size_t)d.Is * (d.H / 32) : 0},
+        {h->w.sh_up_s, d.n_shared ? (size_t)d.Is * (d.H / 32) : 0}, {h->w.sh_down_s, d.n_shared ? (size_t)d.H * (d.Is / 32) : 0},
+    };
+    unsigned host_bad = 0;
+    e = cudaMemsetAsync(bad, 0, sizeof(unsigned), h->side);
+    for (auto &a : arrs)
+        if (e == cudaSuccess) e = launch_scale_check(a.p, a.n, bad, h->side);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&host_bad, bad, sizeof(unsigned), cudaMemcpyDeviceToHost, h->side);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(h->side);
+    cudaFree(bad);
+    if (e != cudaSuccess) return record_cuda(h, e);
+    return host_bad ? MOEDEC_ERR_UNSUPPORTED : MOEDEC_OK;
+}
+
+enum KernelKind { K_ROUTER_DN, K_TOPK, K_EXPERT_GU, K_EXPERT_DOWN, K_COMBINE, K_UP, K_SHARED_GU, K_SHARED_DOWN, K_COUNT };
+const char *const kKernelNames[K_COUNT] = {"router_dn", "topk", "expert_gate_up", "expert_down",
+                                           "combine", "up", "shared_gate_up", "shared_down"};
+
+cudaEvent_t pool_get(moedec_handle *h) {
+    if (!h->pool.empty()) {
+        cudaEvent_t e = h->pool.back();
+        h->pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Launch `fn` on `s`; when profiling, bracket it with an event pair on the same stream.
+template <class F>
+cudaError_t timed(moedec_handle *h, int kind, cudaStream_t s, F fn) {
+    if (!h->profiling) return fn();
+    cudaEvent_t a = pool_get(h), b = pool_get(h);
+    if (!a || !b) return cudaErrorMemoryAllocation;
+    cudaError_t e = cudaEventRecord(a, s);
+    if (e == cudaSuccess) e = fn();
+    if (e == cudaSuccess) e = cudaEventRecord(b, s);
+    if (e == cudaSuccess) h->marks.push_back({kind, a, b});
+    return e;
+}
+
+int read_device_error(moedec_handle *h, cudaStream_t s) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, h->ws.err, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return record_cuda(h, e);
+    if (v == 0) return MOEDEC_OK;
+    cudaMemsetAsync(h->ws.err, 0, sizeof(unsigned), s);
+    cudaStreamSynchronize(s);
+    return (v & kErrTimeout) ? MOEDEC_ERR_TIMEOUT : MOEDEC_ERR_DEVICE;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOEDEC_API const char *moedec_status_string(int status) {
+    switch (status) {
+        case MOEDEC_OK: return "MOEDEC_OK";
+        case MOEDEC_ERR_INVALID_ARG: return "MOEDEC_ERR_INVALID_ARG";
+        case MOEDEC_ERR_UNSUPPORTED: return "MOEDEC_ERR_UNSUPPORTED";
+        case MOEDEC_ERR_CUDA: return "MOEDEC_ERR_CUDA";
+        case MOEDEC_ERR_OOM: return "MOEDEC_ERR_OOM";
+        case MOEDEC_ERR_TIMEOUT: return "MOEDEC_ERR_TIMEOUT";
+        case MOEDEC_ERR_DEVICE: return "MOEDEC_ERR_DEVICE";
+        default: return "MOEDEC_ERR_UNKNOWN";
+    }
+}
+
+MOEDEC_API const char *moedec_last_cuda_error(moedec_handle *h) { return h ? h->cuda_error : ""; }
+
+MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, moedec_handle **out) {
+    if (!out) return MOEDEC_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!cfg || !w || cfg->abi_version != MOEDEC_ABI_VERSION) return MOEDEC_ERR_INVALID_ARG;
+    const moedec_config &c = *cfg;
+    if (c.hidden <= 0 || c.latent <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.expert_inter <= 0 || c.max_batch <= 0 ||
+        (c.n_shared != 0 && c.n_shared != 1) || (c.n_shared && c.shared_inter <= 0))
+        return MOEDEC_ERR_INVALID_ARG;
+    if (c.hidden % 128 || c.latent % 128 || c.expert_inter % 128 || (c.n_shared && c.shared_inter % 128) ||
+        c.n_experts > kMaxExperts || c.top_k > c.n_experts || c.top_k > kMaxTopK || c.max_batch > kMaxBatch)
+        return MOEDEC_ERR_UNSUPPORTED;
+    const void *ptrs[] = {w->router, w->w_down_lat, w->w_up_lat, w->gate_q, w->gate_s, w->up_q, w->up_s, w->down_q, w->down_s};
+    for (const void *p : ptrs)
+        if (!p || !aligned16(p)) return MOEDEC_ERR_INVALID_ARG;
+    if (c.n_shared) {
+        const void *sp[] = {w->sh_gate_q, w->sh_gate_s, w->sh_up_q, w->sh_up_s, w->sh_down_q, w->sh_down_s};
+        for (const void *p : sp)
+            if (!p || !aligned16(p)) return MOEDEC_ERR_INVALID_ARG;
+    }
+    moedec_handle *h = new (std::nothrow) moedec_handle();
+    if (!h) return MOEDEC_ERR_OOM;
+    h->cfg = c;
+    h->d = Dims{c.hidden, c.latent, c.n_experts, c.top_k, c.expert_inter, c.n_shared ? c.shared_inter : 128,
+                c.n_shared, c.max_batch};
+    h->w = Weights{w->router, w->w_down_lat, w->w_up_lat, w->gate_q, w->gate_s, w->up_q, w->up_s, w->down_q, w->down_s,
+                   w->sh_gate_q, w->sh_gate_s, w->sh_up_q, w->sh_up_s, w->sh_down_q, w->sh_down_s};
+    const Dims &d = h->d;
+    Plan &p = h->p;
+    p.rt = split(d.E, kRouterRows, d.H);
+    p.dn = split(d.L, kDenseRows, d.H);
+    p.up = split(d.H, kDenseRows, d.L);
+    p.sgu = split(d.Is, kDenseRows, d.H);
+    p.sd = split(d.H, kDenseRows, d.Is);
+    p.ticket_rt = 0;
+    p.ticket_dn = p.ticket_rt + p.rt.blocks;
+    p.ticket_up = p.ticket_dn + p.dn.blocks;
+    p.ticket_sgu = p.ticket_up + p.up.blocks;
+    p.ticket_sd = p.ticket_sgu + p.sgu.blocks;
+    p.ticket_topk = p.ticket_sd + p.sd.blocks;
+    p.n_tickets = p.ticket_topk + 1;
+
+    int rc = MOEDEC_OK;
+    cudaError_t e = cudaGetDevice(&h->device);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device);
+    if (e == cudaSuccess) e = init_kernel_attributes();
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
+    if (e == cudaSuccess) {
+        layout(h, nullptr);
+        e = cudaMalloc(&h->buf, h->buf_bytes);
+    }
+    if (e == cudaSuccess) {
+        layout(h, static_cast<char *>(h->buf));
+        e = cudaMemsetAsync(h->buf, 0, h->buf_bytes, h->side);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(h->side);
+    }
+    if (e != cudaSuccess) rc = record_cuda(h, e);
+    if (rc == MOEDEC_OK && !(c.flags & MOEDEC_FLAG_SKIP_SCALE_CHECK)) rc = check_scales(h);
+    if (rc != MOEDEC_OK) {
+        moedec_destroy(h);
+        return rc;
+    }
+    *out = h;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_destroy(moedec_handle *h) {
+    if (!h) return MOEDEC_OK;
+    if (h->side) cudaStreamSynchronize(h->side);
+    for (auto &m : h->marks) {
+        cudaEventSynchronize(m.stop);
+        cudaEventDestroy(m.start);
+        cudaEventDestroy(m.stop);
+    }
+    for (auto e : h->pool) cudaEventDestroy(e);
+    if (h->buf) cudaFree(h->buf);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->side) cudaStreamDestroy(h->side);
+    delete h;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint16_t *out, void *stream) {
+    if (!h || batch < 0) return MOEDEC_ERR_INVALID_ARG;
+    if (batch > h->d.max_batch) return MOEDEC_ERR_UNSUPPORTED;
+    if (batch == 0) return MOEDEC_OK;
+    if (!x || !out || !aligned16(x) || !aligned16(out)) return MOEDEC_ERR_INVALID_ARG;
+    const size_t bytes = (size_t)batch * h->d.H * 2;
+    const char *xb = reinterpret_cast<const char *>(x), *ob = reinterpret_cast<const char *>(out);
+    if (xb < ob + bytes && ob < xb + bytes) return MOEDEC_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    StepArgs a;
+    a.d = h->d;
+    a.w = h->w;
+    a.ws = h->ws;
+    a.p = h->p;
+    a.x = x;
+    a.out = out;
+    a.B = batch;
+    cudaError_t e = cudaSuccess;
+    if (h->d.n_shared) {
+        e = cudaEventRecord(h->ev_fork, s);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
+        if (e == cudaSuccess) e = timed(h, K_SHARED_GU, h->side, [&] { return launch_shared_gate_up(a, h->side); });
+        if (e == cudaSuccess) e = timed(h, K_SHARED_DOWN, h->side, [&] { return launch_shared_down(a, h->side); });
+        if (e == cudaSuccess) e = cudaEventRecord(h->ev_join, h->side);
+    }
+    if (e == cudaSuccess) e = timed(h, K_ROUTER_DN, s, [&] { return launch_router_dn(a, s); });
+    if (e == cudaSuccess) e = timed(h, K_TOPK, s, [&] { return launch_topk(a, s); });
+    if (e == cudaSuccess) e = timed(h, K_EXPERT_GU, s, [&] { return launch_expert_gate_up(a, s, h->n_sm); });
+    if (e == cudaSuccess) e = timed(h, K_EXPERT_DOWN, s, [&] { return launch_expert_down(a, s, h->n_sm); });
+    if (e == cudaSuccess) e = timed(h, K_COMBINE, s, [&] { return launch_combine(a, s); });
+    if (e == cudaSuccess && h->d.n_shared) e = cudaStreamWaitEvent(s, h->ev_join, 0);
+    if (e == cudaSuccess) e = timed(h, K_UP, s, [&] { return launch_up(a, s); });
+    if (e != cudaSuccess) return record_cuda(h, e);
+    h->launches[batch <= 2 ? 0 : 1] += (uint64_t)kernels_per_step(h->d);
+    h->last_batch = batch;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_get_routing(moedec_handle *h, int32_t *idx, float *w, int batch, void *stream) {
+    if (!h || batch != h->last_batch || batch <= 0) return MOEDEC_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)batch * h->d.k;
+    cudaError_t e = cudaSuccess;
+    if (idx) e = cudaMemcpyAsync(idx, h->ws.idx, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess && w) e = cudaMemcpyAsync(w, h->ws.wts, n * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return record_cuda(h, e);
+    return read_device_error(h, s);
+}
+
+MOEDEC_API int moedec_get_taps(moedec_handle *h, float *logits, float *hlat, float *ylat, float *sh, float *up, int batch,
+                               void *stream) {
+    if (!h || batch != h->last_batch || batch <= 0) return MOEDEC_ERR_INVALID_ARG;
+    if (up && !h->ws.up_tap) return MOEDEC_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Dims &d = h->d;
+    const size_t B = (size_t)batch;
+    struct {
+        void *dst;
+        const void *src;
+        size_t bytes;
+    } cp[] = {{logits, h->ws.logits, B * d.E * 4}, {hlat, h->ws.h, B * d.L * 4}, {ylat, h->ws.ylat, B * d.L * 4},
+              {sh, h->ws.sh, B * d.H * 4}, {up, h->ws.up_tap, B * d.H * 4}};
+    cudaError_t e = cudaSuccess;
+    if (sh && !d.n_shared) e = cudaMemsetAsync(sh, 0, B * d.H * 4, s);
+    for (auto &c : cp) {
+        if (!c.dst || e != cudaSuccess) continue;
+        if (c.src == h->ws.sh && !d.n_shared) continue;
+        e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyDeviceToDevice, s);
+    }
+    if (e != cudaSuccess) return record_cuda(h, e);
+    return read_device_error(h, s);
+}
+
+MOEDEC_API int moedec_get_launch_counts(moedec_handle *h, uint64_t *launches, int *n_variants) {
+    if (!h || !launches || !n_variants || *n_variants < 1) return MOEDEC_ERR_INVALID_ARG;
+    const int n = *n_variants < 2 ? *n_variants : 2;
+    for (int i = 0; i < n; ++i) launches[i] = h->launches[i];
+    *n_variants = 2;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_profile_enable(moedec_handle *h, int enable) {
+    if (!h) return MOEDEC_ERR_INVALID_ARG;
+    for (auto &m : h->marks) {
+        cudaEventSynchronize(m.stop);
+        h->pool.push_back(m.start);
+        h->pool.push_back(m.stop);
+    }
+    h->marks.clear();
+    for (int i = 0; i < K_COUNT; ++i) {
+        h->prof_ms[i] = 0.0;
+        h->prof_n[i] = 0;
+    }
+    h->profiling = enable != 0;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t *launches, const char **names, int *n) {
+    if (!h || !n || *n < 0) return MOEDEC_ERR_INVALID_ARG;
+    for (auto &m : h->marks) {
+        cudaError_t e = cudaEventSynchronize(m.stop);
+        float ms = 0.0f;
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, m.start, m.stop);
+        if (e != cudaSuccess) return record_cuda(h, e);
+        h->prof_ms[m.kind] += ms;
+        h->prof_n[m.kind] += 1;
+        h->pool.push_back(m.start);
+        h->pool.push_back(m.stop);
+    }
+    h->marks.clear();
+    const int cap = *n;
+    for (int i = 0; i < K_COUNT && i < cap; ++i) {
+        if (total_ms) total_ms[i] = h->prof_ms[i];
+        if (launches) launches[i] = h->prof_n[i];
+        if (names) names[i] = kKernelNames[i];
+    }
+    *n = K_COUNT;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_kernels_per_step(moedec_handle *h, int batch) {
+    if (!h || batch <= 0) return 0;
+    return kernels_per_step(h->d);
+}
+
+}  // extern "C"

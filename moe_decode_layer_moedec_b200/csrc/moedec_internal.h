@@ -1,0 +1,95 @@
+// moedec_internal.h -- parameter blocks shared by the host orchestration and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moedec {
+
+constexpr int kMaxBatch = 64;      // token masks of the routing buckets are one 64-bit word
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;  // one top-k thread per expert
+constexpr int kDenseWarps = 8;     // dense split-K kernels: 8 warps x 16 rows = 128 rows per CTA
+constexpr int kDenseRows = 128;
+constexpr int kRouterRows = 64;    // router CTA: 8 warps x 8 rows (fp64 m8n8k4)
+constexpr int kExpertWarps = 4;    // expert kernels: 4 warps x 16 rows per item
+constexpr int kExpertRows = 64;
+constexpr int kKChunk = 512;       // activation staging chunk along K
+
+struct Dims {
+    int H, L, E, k, I, Is, n_shared, max_batch;
+};
+
+struct Weights {
+    const uint16_t *router, *w_dn, *w_up;
+    const uint8_t *gate_q, *gate_s, *up_q, *up_s, *down_q, *down_s;
+    const uint8_t *sh_gate_q, *sh_gate_s, *sh_up_q, *sh_up_s, *sh_down_q, *sh_down_s;
+};
+
+// Split-K plan of one dense matrix-vector product: `blocks` row blocks x `splits` K ranges.
+struct SplitPlan {
+    int blocks, splits, krange;
+};
+
+struct Plan {
+    SplitPlan rt, dn, up, sgu, sd;
+    int ticket_rt, ticket_dn, ticket_up, ticket_sgu, ticket_sd, ticket_topk;  // offsets into tickets[]
+    int n_tickets;
+};
+
+// Device workspace of one handle (all sized for max_batch).
+struct Work {
+    double *rt_part;    // [rt.splits][maxB][E]   router partial sums (fp64)
+    float *logits;      // [maxB][E]
+    float *dn_part;     // [dn.splits][maxB][L]
+    float *h;           // [maxB][L]
+    int *h_shift;       // [maxB] fp16 staging exponent of h per token
+    int *idx;           // [maxB][k]
+    float *wts;         // [maxB][k]
+    int *n_active;      // [1]  experts with at least one token
+    int *active_e;      // [E]  their ids, ascending
+    int *active_cnt;    // [E]  tokens per active expert
+    int *active_off;    // [E]  offset of the expert's entries
+    int *entries;       // [maxB*k] entry = b*k + r, grouped by expert, token-ascending inside a group
+    float *a;           // [maxB*k][I]  silu(gate) * up per entry
+    unsigned *a_amax;   // [maxB*k]     max |a| per entry (float bits)
+    float *y;           // [maxB*k][L]  expert output per entry
+    float *ylat;        // [maxB][L]
+    float *sgu_part;    // [sgu.splits][maxB][2*Is] shared gate then up partials
+    float *sh_a;        // [maxB][Is]
+    float *sd_part;     // [sd.splits][maxB][H]
+    float *sh;          // [maxB][H]
+    float *up_part;     // [up.splits][maxB][H]
+    float *up_tap;      // [maxB][H] or nullptr
+    unsigned *tickets;  // [n_tickets]
+    unsigned *err;      // [1] sticky device error word
+};
+
+struct StepArgs {
+    Dims d;
+    Weights w;
+    Work ws;
+    Plan p;
+    const uint16_t *x;  // [B][H]
+    uint16_t *out;      // [B][H]
+    int B;
+};
+
+// error word bits
+constexpr unsigned kErrBucket = 1u;    // routing bucket overflow (internal invariant)
+constexpr unsigned kErrTimeout = 2u;   // a bounded device wait gave up
+
+// host launchers (moedec_kernels.cu)
+cudaError_t launch_router_dn(const StepArgs &a, cudaStream_t s);
+cudaError_t launch_topk(const StepArgs &a, cudaStream_t s);
+cudaError_t launch_expert_gate_up(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t launch_expert_down(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t launch_combine(const StepArgs &a, cudaStream_t s);
+cudaError_t launch_up(const StepArgs &a, cudaStream_t s);
+cudaError_t launch_shared_gate_up(const StepArgs &a, cudaStream_t s);
+cudaError_t launch_shared_down(const StepArgs &a, cudaStream_t s);
+cudaError_t launch_scale_check(const uint8_t *s, size_t n, unsigned *bad, cudaStream_t st);
+int kernels_per_step(const Dims &d);
+cudaError_t init_kernel_attributes();
+
+}  // namespace moedec

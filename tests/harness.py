@@ -1,0 +1,70 @@
+"""Helpers shared by the GPU tests: upload seeded weights, run the layer, compare with the oracle."""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+
+TOL_REL_L2 = 5e-3       # relative L2 error bound of every float output
+TOL_MAX_REL = 1e-2      # max |err| <= TOL_MAX_REL * max |ref|
+
+
+def to_device(arr: np.ndarray, device="cuda"):
+    import torch
+    if arr.dtype == np.uint16:
+        return torch.from_numpy(arr.view(np.int16)).to(device)
+    return torch.from_numpy(arr).to(device)
+
+
+def upload_weights(W: dict, device="cuda") -> dict:
+    return {k: to_device(np.ascontiguousarray(v), device) for k, v in W.items()}
+
+
+def layer_dims(d: synth.Dims):
+    from moe_decode_layer_moedec_b200 import LayerDims
+    return LayerDims(d.hidden, d.latent, d.n_experts, d.top_k, d.expert_inter, d.shared_inter, 1)
+
+
+def bf16_tensor_to_f32(t) -> np.ndarray:
+    return synth.bf16_to_f32(t.cpu().numpy().view(np.uint16))
+
+
+def rel_errors(got: np.ndarray, ref: np.ndarray):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = got - ref
+    rel_l2 = float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300))
+    max_rel = float(np.abs(err).max() / max(np.abs(ref).max(), 1e-300))
+    return rel_l2, max_rel
+
+
+def assert_close(got, ref, name: str):
+    rel_l2, max_rel = rel_errors(got, ref)
+    assert rel_l2 <= TOL_REL_L2 and max_rel <= TOL_MAX_REL, \
+        f"{name}: relative L2 {rel_l2:.3e} (bound {TOL_REL_L2}), max|err|/max|ref| {max_rel:.3e} (bound {TOL_MAX_REL})"
+    return rel_l2, max_rel
+
+
+def assert_logits_match(got: np.ndarray, ref: np.ndarray, name: str = "logits"):
+    """fp32 logits from fp64 sums: identical except where the exact sum sits within fp64
+    rounding of an fp32 rounding boundary (then they differ by one ulp)."""
+    got = np.asarray(got, dtype=np.float32)
+    ref = np.asarray(ref, dtype=np.float32)
+    diff = got != ref
+    if diff.any():
+        ulps = np.abs(got.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
+        assert ulps[diff].max() <= 1, f"{name}: logits differ by more than one ulp"
+        assert diff.mean() <= 1e-4, f"{name}: {int(diff.sum())} logits differ"
+
+
+def run_layer(layer, x_np: np.ndarray):
+    """One step through the C ABI; returns (out fp32, idx, w, taps dict) as numpy."""
+    import torch
+    x = to_device(x_np)
+    out = layer.step(x)
+    B = x_np.shape[0]
+    idx, w = layer.routing(B)
+    taps = layer.taps(B)
+    torch.cuda.synchronize()
+    return (bf16_tensor_to_f32(out), idx.cpu().numpy(), w.cpu().numpy(),
+            {k: v.cpu().numpy() for k, v in taps.items()})

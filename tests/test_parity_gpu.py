@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA step through the C ABI against the CPU oracle, element by element.
+
+Routing indices must match bit-exactly; every float output (out, and the h / ylat / sh / up
+taps, checked separately because the shared expert dominates the magnitude of out) must meet
+relative L2 <= 5e-3 and max|err| <= 1e-2 * max|ref|.  Sizes: the tiny layer at several batches
+(ragged n-tiles, every token checked) and the full-size layer in the launch configuration the
+bench times (all tokens' routing, sampled tokens' outputs).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.harness import (assert_close, assert_logits_match, layer_dims, rel_errors, run_layer, to_device,
+                           upload_weights)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    assert torch.cuda.is_available()
+    return torch
+
+
+def _make_layer(w, W_dev, max_batch, flags=None):
+    from moe_decode_layer_moedec_b200 import FLAG_TAPS, MoeDecodeLayer
+    return MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=max_batch, flags=FLAG_TAPS if flags is None else flags)
+
+
+def _check_step(w, W, x, layer, tokens=None, check_all_routing=True):
+    out, idx, wts, taps = run_layer(layer, x)
+    B = x.shape[0]
+    if check_all_routing:
+        lg, ridx, rw = oracle.route(W["router"], x, w.dims.top_k)
+        assert np.array_equal(idx, ridx), "routing indices differ from the oracle"
+        np.testing.assert_allclose(wts, rw, rtol=2e-6, atol=0)
+        assert_logits_match(taps["logits"], lg)
+    toks = range(B) if tokens is None else tokens
+    for t in toks:
+        r = oracle.step(w.dims, W, x, tokens=range(t, t + 1))
+        assert np.array_equal(idx[t], r["idx"][0])
+        assert_close(taps["h"][t], r["h"][0], f"h[{t}]")
+        assert_close(taps["ylat"][t], r["ylat"][0], f"ylat[{t}]")
+        assert_close(taps["sh"][t], r["sh"][0], f"sh[{t}]")
+        assert_close(taps["up"][t], r["out"][0] - r["sh"][0], f"up[{t}]")
+        assert_close(out[t], r["out"][0], f"out[{t}]")
+    return out, idx
+
+
+# ---- tiny layer -------------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def tiny(torch_cuda):
+    w = synth.WORKLOADS["tiny_b1"]
+    W = synth.layer_weights(w, 0)
+    return w, W, upload_weights(W)
+
+
+@pytest.mark.parametrize("B", [1, 2, 3, 5, 8, 9, 17, 33, 64])
+def test_tiny_parity(tiny, B):
+    w, W, W_dev = tiny
+    layer = _make_layer(w, W_dev, max_batch=64)
+    x = synth.tokens(w, step=B, batch=B)
+    _check_step(w, W, x, layer)
+
+
+def test_tiny_launch_variant_counts(tiny):
+    w, W, W_dev = tiny
+    layer = _make_layer(w, W_dev, max_batch=16)
+    run_layer(layer, synth.tokens(w, batch=1))
+    run_layer(layer, synth.tokens(w, batch=2))
+    c = layer.launch_counts()
+    assert c["small"] == 2 * layer.kernels_per_step(1) and c["splitk"] == 0
+    run_layer(layer, synth.tokens(w, batch=16))
+    assert layer.launch_counts()["splitk"] == layer.kernels_per_step(16)
+
+
+def test_tiny_deterministic(tiny):
+    w, W, W_dev = tiny
+    layer = _make_layer(w, W_dev, max_batch=8)
+    x = synth.tokens(w, batch=8)
+    a = run_layer(layer, x)
+    b = run_layer(layer, x)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    for k in a[3]:
+        assert np.array_equal(a[3][k], b[3][k]), k
+
+
+def test_tiny_back_to_back_steps_see_their_own_tokens(tiny, torch_cuda):
+    # Several steps queued on one stream with different tokens, then one graph replay of two
+    # steps: every output must match its own token batch (no stale activations).
+    torch = torch_cuda
+    w, W, W_dev = tiny
+    layer = _make_layer(w, W_dev, max_batch=4, flags=0)
+    xs = [synth.tokens(w, step=100 + i, batch=4) for i in range(3)]
+    xd = [to_device(x) for x in xs]
+    outs = [layer.step(x) for x in xd]
+    torch.cuda.synchronize()
+    for x, o in zip(xs, outs):
+        ref = oracle.step(w.dims, W, x)
+        got = synth.bf16_to_f32(o.cpu().numpy().view(np.uint16))
+        assert_close(got, ref["out"], "queued out")
+    g = torch.cuda.CUDAGraph()
+    o1 = torch.empty_like(xd[0])
+    o2 = torch.empty_like(xd[0])
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        layer.step(xd[0], out=o1)
+        layer.step(xd[1], out=o2)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        layer.step(xd[1], out=o1)
+        layer.step(xd[2], out=o2)
+    o1.zero_()
+    o2.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    for x, o in ((xs[1], o1), (xs[2], o2)):
+        ref = oracle.step(w.dims, W, x)
+        assert_close(synth.bf16_to_f32(o.cpu().numpy().view(np.uint16)), ref["out"], "graph out")
+    del g
+
+
+def test_batch_zero_and_limits(tiny, torch_cuda):
+    from moe_decode_layer_moedec_b200 import MoedecError, lib
+    torch = torch_cuda
+    w, W, W_dev = tiny
+    layer = _make_layer(w, W_dev, max_batch=4)
+    x = to_device(synth.tokens(w, batch=8))
+    out = torch.empty_like(x)
+    s = torch.cuda.current_stream().cuda_stream
+    assert lib.moedec_step(layer._h, x.data_ptr(), 0, out.data_ptr(), s) == 0
+    assert lib.moedec_step(layer._h, x.data_ptr(), 5, out.data_ptr(), s) == -2      # > max_batch
+    assert lib.moedec_step(layer._h, x.data_ptr() + 2, 1, out.data_ptr(), s) == -1  # misaligned
+    assert lib.moedec_step(layer._h, x.data_ptr(), 2, x.data_ptr() + 16, s) == -1   # overlapping
+    assert lib.moedec_step(None, x.data_ptr(), 1, out.data_ptr(), s) == -1
+    with pytest.raises(MoedecError):
+        layer.routing(3)  # not the last step's batch
+
+
+def test_create_rejects_bad_config(tiny):
+    from moe_decode_layer_moedec_b200 import MoedecError, MoeDecodeLayer
+    w, W, W_dev = tiny
+    d = layer_dims(w.dims)
+    with pytest.raises(MoedecError, match="UNSUPPORTED"):
+        MoeDecodeLayer(d, W_dev, max_batch=65)
+    bad = dict(W_dev)
+    bad["gate_s"] = W_dev["gate_s"].clone()
+    bad["gate_s"][3, 7, 1] = 150   # scale 2^23: outside the exact fp16 range
+    with pytest.raises(MoedecError, match="UNSUPPORTED"):
+        MoeDecodeLayer(d, bad, max_batch=1)
+    import dataclasses
+    with pytest.raises(MoedecError, match="UNSUPPORTED"):
+        MoeDecodeLayer(dataclasses.replace(d, hidden=500), W_dev, max_batch=1)
+
+
+def test_tiny_tied_router_rows(tiny, torch_cuda):
+    # duplicated router rows give equal logits: the lower expert index must win
+    w, W, W_dev = tiny
+    x = synth.tokens(w, batch=4)
+    lg, idx, _ = oracle.route(W["router"], x, w.dims.top_k)
+    W2 = {k: v.copy() for k, v in W.items()}
+    top = int(idx[0, 0])
+    other = (top + 1) % w.dims.n_experts
+    W2["router"][other] = W["router"][top]
+    W2_dev = dict(W_dev)
+    W2_dev["router"] = to_device(W2["router"])
+    layer = _make_layer(w, W2_dev, max_batch=4)
+    out, gidx, _, _ = run_layer(layer, x)
+    _, ridx, _ = oracle.route(W2["router"], x, w.dims.top_k)
+    assert np.array_equal(gidx, ridx)
+    assert min(top, other) == ridx[0, 0]
+
+
+# ---- full-size layer ----------------------------------------------------------------------------
+
+@pytest.fixture(scope="module")
+def full_layers(torch_cuda):
+    cache = {}
+
+    def get(name, layer_idx=0):
+        key = (name, layer_idx)
+        if key not in cache:
+            cache.clear()  # one full layer (3 GB) resident at a time
+            torch_cuda.cuda.empty_cache()
+            w = synth.WORKLOADS[name]
+            W = synth.layer_weights(w, layer_idx)
+            cache[key] = (w, W, upload_weights(W))
+        return cache[key]
+    return get
+
+
+@pytest.mark.parametrize("name", ["full_b1", "full_b2"])
+def test_full_small_batches_all_tokens(full_layers, name):
+    w, W, W_dev = full_layers(name)
+    layer = _make_layer(w, W_dev, max_batch=w.batch)
+    x = synth.tokens(w)
+    out, idx = _check_step(w, W, x, layer)
+    if name == "full_b2":
+        assert 0 < len(set(idx[0]) & set(idx[1])) < w.dims.top_k
+
+
+def test_full_b16_sampled_tokens(full_layers):
+    w, W, W_dev = full_layers("full_b16")
+    layer = _make_layer(w, W_dev, max_batch=w.batch)
+    x = synth.tokens(w)
+    _check_step(w, W, x, layer, tokens=[0, 7, 15])
+
+
+@pytest.mark.parametrize("layer_idx", [0, 31])
+def test_full_b64_skewed_sampled_tokens(full_layers, layer_idx):
+    w, W, W_dev = full_layers("full_b64_skewed", layer_idx)
+    layer = _make_layer(w, W_dev, max_batch=w.batch)
+    x = synth.tokens(w)
+    _, ridx_all = oracle.route(W["router"], x, w.dims.top_k)[0], oracle.route(W["router"], x, w.dims.top_k)[1]
+    # sample the token with the most hot selections, one with none, and the last token
+    hot = np.isin(ridx_all, synth.hot_set(w, layer_idx)).sum(axis=1)
+    sample = sorted({int(np.argmax(hot)), int(np.argmin(hot)), w.batch - 1})
+    _check_step(w, W, x, layer, tokens=sample)
