@@ -312,6 +312,8 @@ def main():
             per_kernel[name] = (a + kms, b + n)
     kb = kernel_bytes(d, unique_mean, B)
     peak, peak_src = measured_peak_hbm()
+    if not any(v[0] > 0 for v in per_kernel.values()):
+        raise RuntimeError(f"per-kernel profile is empty: {per_kernel}")
     dom = max(per_kernel, key=lambda k: per_kernel[k][0])
     dom_ms, dom_n = per_kernel[dom]
     dom_avg_s = dom_ms / 1e3 / max(dom_n, 1)

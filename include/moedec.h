@@ -164,7 +164,10 @@ MOEDEC_API const char *moedec_last_cuda_error(moedec_handle *h);
  *   total_ms[i]  summed event-measured duration of its launches since enabling (host array)
  *   launches[i]  number of its launches (host array)
  *   names[i]     static name of the kind (host array of const char*), may be NULL
- * *n is in/out (array capacity in, number of kinds out).  Enabling again resets the sums.
+ * *n is in/out (array capacity in, number of kinds out).  enable=1 resets the sums and starts
+ * recording; enable=0 stops recording and keeps what was recorded for moedec_profile_read.  Event
+ * pairs recorded while a stream is being captured become part of the graph and hold the times
+ * of the graph's latest replay.
  */
 MOEDEC_API int moedec_profile_enable(moedec_handle *h, int enable);
 MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t *launches, const char **names, int *n);

@@ -147,9 +147,14 @@ cudaError_t timed(moedec_handle *h, int kind, cudaStream_t s, F fn) {
     if (!h->profiling) return fn();
     cudaEvent_t a = pool_get(h), b = pool_get(h);
     if (!a || !b) return cudaErrorMemoryAllocation;
-    cudaError_t e = cudaEventRecord(a, s);
+    // Under stream capture a plain record only expresses a dependency; an external record
+    // becomes an event-record node that timestamps every replay of the graph.
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    const unsigned flags = (cs == cudaStreamCaptureStatusActive) ? cudaEventRecordExternal : 0u;
+    if (e == cudaSuccess) e = cudaEventRecordWithFlags(a, s, flags);
     if (e == cudaSuccess) e = fn();
-    if (e == cudaSuccess) e = cudaEventRecord(b, s);
+    if (e == cudaSuccess) e = cudaEventRecordWithFlags(b, s, flags);
     if (e == cudaSuccess) h->marks.push_back({kind, a, b});
     return e;
 }
@@ -351,6 +356,10 @@ MOEDEC_API int moedec_get_launch_counts(moedec_handle *h, uint64_t *launches, in
 
 MOEDEC_API int moedec_profile_enable(moedec_handle *h, int enable) {
     if (!h) return MOEDEC_ERR_INVALID_ARG;
+    if (!enable) {  // stop recording; recorded marks stay readable
+        h->profiling = false;
+        return MOEDEC_OK;
+    }
     for (auto &m : h->marks) {
         cudaEventSynchronize(m.stop);
         h->pool.push_back(m.start);
@@ -361,7 +370,7 @@ MOEDEC_API int moedec_profile_enable(moedec_handle *h, int enable) {
         h->prof_ms[i] = 0.0;
         h->prof_n[i] = 0;
     }
-    h->profiling = enable != 0;
+    h->profiling = true;
     return MOEDEC_OK;
 }
 
