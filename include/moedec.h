@@ -172,6 +172,30 @@ MOEDEC_API const char *moedec_last_cuda_error(moedec_handle *h);
 MOEDEC_API int moedec_profile_enable(moedec_handle *h, int enable);
 MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t *launches, const char **names, int *n);
 
+/*
+ * Router logits without any device allocation.  The pages have no counterpart of this call; it
+ * exists for callers that cannot call cudaMalloc: code that runs while its stream is being
+ * captured into a CUDA graph under a no-allocation policy, processes whose device memory is
+ * entirely handed to another allocator, and runtimes with a fixed, pre-planned memory budget.
+ *   router   bf16 [n_experts][hidden], device, 16-byte aligned      x  bf16 [batch][hidden], device, 16-byte aligned
+ *   logits   fp32 [batch][n_experts], device (output)               stream  cudaStream_t as void*
+ * Computes logits[b][e] = fp32(sum_j router[e][j] x[b][j]) exactly as moedec_step does (same
+ * kernel body and split order, so the values equal moedec_get_taps' logits).  Its split-K scratch
+ * is one static 2 MiB device array in the library that every GPU loading the library keeps until
+ * the process exits; the call only clears the ticket words it needs (an async memset on `stream`).
+ * Limit: (hidden / 512) * batch * n_experts * 8 bytes + 4 KiB <= 2 MiB (hidden a multiple of 512;
+ * 256 or 128 when it is not, with proportionally more splits); beyond it the call returns
+ * MOEDEC_ERR_UNSUPPORTED.  With hidden 7168 and 896 experts that allows batch <= 20.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.  All calls
+ * share the one array, so calls that may overlap on the GPU (different streams, or different
+ * host threads) race; serialise them.
+ * Errors: INVALID_ARG (NULL or misaligned pointer, batch < 0, non-positive sizes), UNSUPPORTED
+ * (hidden not a multiple of 128, n_experts > 1024, scratch limit), CUDA.
+ */
+MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, const uint16_t *x, int n_experts, int hidden,
+                                            int batch, float *logits, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 MOEDEC_API const char *moedec_status_string(int status);
 

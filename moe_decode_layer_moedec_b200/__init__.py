@@ -68,6 +68,8 @@ def _load():
     lib.moedec_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64),
                                         ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(i32)]
     lib.moedec_profile_read.restype = i32
+    lib.moedec_router_logits_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.moedec_router_logits_noalloc.restype = i32
     lib.moedec_kernels_per_step.argtypes = [vp, i32]
     lib.moedec_kernels_per_step.restype = i32
     lib.moedec_last_cuda_error.argtypes = [vp]
@@ -200,3 +202,18 @@ class MoeDecodeLayer:
             self.close()
         except Exception:
             pass
+
+
+def router_logits_noalloc(router, x, logits=None, stream=None):
+    """fp32 router logits [B, E] without any device allocation by the library (see include/moedec.h).
+
+    For callers that cannot call cudaMalloc; `logits` may be passed in pre-allocated."""
+    import torch
+    E, H = router.shape
+    B = x.shape[0]
+    if logits is None:
+        logits = torch.empty((B, E), dtype=torch.float32, device=x.device)
+    rc = lib.moedec_router_logits_noalloc(_ptr(router), _ptr(x), E, H, B, _ptr(logits), _stream_ptr(stream))
+    if rc != 0:
+        raise MoedecError("moedec_router_logits_noalloc", rc)
+    return logits

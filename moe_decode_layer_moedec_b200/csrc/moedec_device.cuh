@@ -123,6 +123,11 @@ DEVI uint16_t f32_to_bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
+// Shared-memory swizzle of staged fp16/fp64 activation units: within each group of 16 units of 16
+// bytes, unit u is stored at u ^ bit3(u), so that the four lane quads of a phase hit distinct
+// bank groups (see the staging layouts in moedec_kernels.cu).
+__host__ __device__ __forceinline__ int swz(int u) { return u ^ ((u >> 3) & 1); }
+
 // ---------------------------------------------------------------------------------------------
 // tensor-core MMAs (warp-wide)
 

@@ -18,6 +18,7 @@
 // its weights once with 128-bit loads and keeps the decode tokens on chip.
 #include "moedec_device.cuh"
 #include "moedec_internal.h"
+#include "moedec_router.cuh"
 
 namespace moedec {
 
@@ -27,7 +28,6 @@ namespace moedec {
 // fp16 columns feeding MXFP4 rows: a 128-element round is 16 units of 16 bytes; lane quad q
 // reads units 4q..4q+3.  Unit u is stored at u ^ bit3(u), and the column pitch is 32 bytes mod
 // 128, so the eight lanes of each shared-memory phase hit eight distinct bank groups.
-__host__ __device__ __forceinline__ int swz(int u) { return u ^ ((u >> 3) & 1); }
 __host__ __device__ __forceinline__ int f16_pitch(int kc) { return kc + 16; }   // halfs
 // bf16 columns feeding bf16 rows: lane quad q reads unit 4r + q; pitch 64 bytes mod 128.
 __host__ __device__ __forceinline__ int bf16_pitch(int kc) { return kc + 32; }  // elements
@@ -280,64 +280,6 @@ DEVI void stage_bf16split_from_f32(uint16_t *xs, int pitch, const float *src, si
 // ---------------------------------------------------------------------------------------------
 // K1: router logits (fp64) and h = W_dn x, one grid.  Blocks [0, rt.blocks*rt.splits) are router
 // blocks (64 rows, one K range), the rest W_dn blocks (128 rows, one K range).
-
-DEVI void router_block(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
-    const int E = a.d.E, H = a.d.H, B = a.B, maxB = a.d.max_batch;
-    const int rb = bid / a.p.rt.splits, ks = bid % a.p.rt.splits;
-    const int KR = a.p.rt.krange, k0 = ks * KR;
-    double *xs = reinterpret_cast<double *>(smem);  // [8][KR + 4]: pitch 32 bytes mod 128
-    const int pitch = KR + 4;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int row = rb * kRouterRows + warp * 8 + g;
-    const bool row_ok = row < E;
-    const uint16_t *rrow = a.w.router + (size_t)(row_ok ? row : 0) * H + k0 + 8 * q;
-    const int half_units = KR / 2;  // units of two doubles
-    for (int tg = 0; tg < B; tg += 8) {
-        const int ntok = min(8, B - tg);
-        __syncthreads();
-        for (int i = threadIdx.x; i < 8 * half_units; i += blockDim.x) {
-            const int t = i / half_units, u = i % half_units;
-            double2 v = make_double2(0.0, 0.0);
-            if (t < ntok) {
-                const uint32_t pr = *reinterpret_cast<const uint32_t *>(a.x + (size_t)(tg + t) * H + k0 + 2 * u);
-                v.x = (double)bf16_lo(pr);
-                v.y = (double)bf16_hi(pr);
-            }
-            *reinterpret_cast<double2 *>(xs + (size_t)t * pitch + 2 * swz(u)) = v;
-        }
-        __syncthreads();
-        // m8n8k4 fp64: lane (g,q) holds A[row g][slot q] and B[slot q][token g]; MMA step s of
-        // chunk c maps slot q to k = 32c + 8q + s.
-        double c0 = 0.0, c1 = 0.0;
-        const double *xr = xs + (size_t)g * pitch;
-        for (int c = 0; c < KR / 32; ++c) {
-            const uint4 A = row_ok ? ldg_weights_l1(rrow + 32 * c) : make_uint4(0u, 0u, 0u, 0u);
-            const double av[8] = {bf16_lo(A.x), bf16_hi(A.x), bf16_lo(A.y), bf16_hi(A.y),
-                                  bf16_lo(A.z), bf16_hi(A.z), bf16_lo(A.w), bf16_hi(A.w)};
-            double2 xv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int u = (16 * c + 4 * q + i) ^ (q >> 1);
-                xv[i] = *reinterpret_cast<const double2 *>(xr + 2 * u);
-            }
-#pragma unroll
-            for (int s = 0; s < 8; ++s) mma_f64(c0, c1, av[s], (s & 1) ? xv[s >> 1].y : xv[s >> 1].x);
-        }
-        if (row_ok) {
-            if (2 * q < ntok) a.ws.rt_part[((size_t)ks * maxB + tg + 2 * q) * E + row] = c0;
-            if (2 * q + 1 < ntok) a.ws.rt_part[((size_t)ks * maxB + tg + 2 * q + 1) * E + row] = c1;
-        }
-    }
-    if (cta_ticket_last(a.ws.tickets + a.p.ticket_rt + rb, a.p.rt.splits, s_flag)) {
-        for (int i = threadIdx.x; i < kRouterRows * B; i += blockDim.x) {
-            const int r = rb * kRouterRows + (i % kRouterRows), b = i / kRouterRows;
-            if (r >= E) continue;
-            double s = 0.0;
-            for (int k = 0; k < a.p.rt.splits; ++k) s += __ldcg(a.ws.rt_part + ((size_t)k * maxB + b) * E + r);
-            a.ws.logits[(size_t)b * E + r] = (float)s;
-        }
-    }
-}
 
 template <int NT>
 DEVI void dn_block(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
