@@ -44,6 +44,8 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="full_b1", choices=sorted(synth.WORKLOADS))
     p.add_argument("--layers", type=int, default=0, help="distinct layers cycled through (default 32)")
+    p.add_argument("--schedule", choices=["fused", "multi"], default="fused",
+                   help="one persistent kernel per step (default) or eight stream-ordered kernels")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
     return p.parse_args()
@@ -72,6 +74,8 @@ def kernel_bytes(d: synth.Dims, unique_experts: float, B: int) -> dict:
         "up": 2 * H * L + 2 * B * H,
         "shared_gate_up": 2 * fp4(Is, H),
         "shared_down": fp4(H, Is),
+        "fused_step_splitk": step_bytes(d, unique_experts, B),
+        "fused_step_small": step_bytes(d, unique_experts, B),
     }
 
 
@@ -215,7 +219,7 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
-    from moe_decode_layer_moedec_b200 import FLAG_SKIP_SCALE_CHECK, LayerDims, MoeDecodeLayer
+    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_SKIP_SCALE_CHECK, LayerDims, MoeDecodeLayer
 
     w = synth.WORKLOADS[args.workload]
     d = w.dims
@@ -234,6 +238,8 @@ def main():
             Wd[k] = t.to(f"cuda:{local_rank}", non_blocking=False)
         del W
         flags = 0 if l == 0 else FLAG_SKIP_SCALE_CHECK  # layer 0 runs the create-time scale scan
+        if args.schedule == "multi":
+            flags |= FLAG_MULTI_KERNEL
         layers.append(MoeDecodeLayer(dims, Wd, max_batch=B, flags=flags))
         dev_weights.append(Wd)
         if rank == 0 and (l % 8 == 7 or l == n_layers - 1):
@@ -364,7 +370,7 @@ def main():
                        "top_k": d.top_k, "layers_cycled": n_layers, "unique_experts_per_step": unique_mean,
                        "l2": "inputs larger than L2: each step streams one of %d distinct layers (>= 148 MB)" % n_layers,
                        "arith": "MXFP4/bf16 weights, fp16/bf16 tensor-core MMA with fp32 accumulation, fp64 router",
-                       "parallelism": "replicas" if world > 1 else "single GPU"},
+                       "parallelism": "replicas" if world > 1 else "single GPU", "schedule": args.schedule},
             "us_per_step": 1e3 * ms_per_step,
             "step_hbm": {"bytes_per_step": sb, "gbs": sb / (ms_per_step / 1e3) / 1e9,
                          "frac": sb / (ms_per_step / 1e3) / 1e9 / peak, "peak_gbs": peak, "peak": peak_src},

@@ -63,6 +63,14 @@ typedef enum moedec_status {
 /* Config flags. */
 #define MOEDEC_FLAG_TAPS 1u            /* also materialise the fp32 `up` tap (W_up ylat) for tests */
 #define MOEDEC_FLAG_SKIP_SCALE_CHECK 2u /* skip moedec_create's scan of the E8M0 scale bytes */
+#define MOEDEC_FLAG_TEST_STALL 4u      /* tests only: the fused step's router never publishes its
+                                          logits, so the first wait on them runs out after 20 ms and
+                                          the step reports MOEDEC_ERR_TIMEOUT (no GPU fault, no hang) */
+#define MOEDEC_FLAG_MULTI_KERNEL 8u    /* run each step as eight stream-ordered kernels (shared expert
+                                          on the side stream) instead of one fused persistent kernel */
+#define MOEDEC_FLAG_TRACE 16u          /* fused step: every CTA stamps %globaltimer at its phase
+                                          boundaries (read with moedec_get_trace) */
+#define MOEDEC_TRACE_STAMPS 16         /* stamps per CTA */
 
 typedef struct moedec_config {
     int32_t abi_version;  /* MOEDEC_ABI_VERSION */
@@ -109,7 +117,11 @@ typedef struct moedec_handle moedec_handle;
 MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, moedec_handle **out);
 
 /*
- * One layer step: out[b] for b < batch from x[b].
+ * One layer step: out[b] for b < batch from x[b].  By default the whole step is one persistent
+ * kernel (one CTA per SM, cooperative launch) whose CTAs take the step's work items in dependency
+ * order; every device-side wait in it is bounded (1 s) and a timeout is reported as
+ * MOEDEC_ERR_TIMEOUT by the next synchronising call.  MOEDEC_FLAG_MULTI_KERNEL selects the
+ * stream-ordered schedule instead (same work items, same results up to fp32 rounding order).
  *   x       bf16 [batch][H], device, 16-byte aligned; read only.
  *   batch   0..max_batch (0 is a no-op that still reports pending device errors).
  *   out     bf16 [batch][H], device, 16-byte aligned; must not overlap x.
@@ -147,7 +159,8 @@ MOEDEC_API int moedec_get_taps(moedec_handle *h, float *logits, float *hlat, flo
 
 /*
  * Launch counters (host values): launches[i] counts the kernels of variant i issued by this
- * handle since creation; i = 0 SMALL (batch <= 2), 1 SPLITK (batch >= 3).  n_variants in/out.
+ * handle since creation; i = 0 the small-batch schedule (batch <= 4: full-K work items, no split-K
+ * partials), 1 the split-K schedule (batch >= 5).  n_variants in/out.
  */
 MOEDEC_API int moedec_get_launch_counts(moedec_handle *h, uint64_t *launches, int *n_variants);
 
@@ -195,6 +208,15 @@ MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t 
  */
 MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, const uint16_t *x, int n_experts, int hidden,
                                             int batch, float *logits, void *stream);
+
+/*
+ * Phase timeline of the last fused step (MOEDEC_FLAG_TRACE): host array out[n_cta][MOEDEC_TRACE_STAMPS]
+ * of %globaltimer nanoseconds, stamp i taken by CTA c when it finished phase i (0 start, 1 router,
+ * 2 top-k, 3 W_dn, 4 shared gate/up, 5 routing wait, 6 expert gate/up, 7 shared down, 8 expert down,
+ * 9 W_up, 10 exit; 0 where a phase was skipped).  *n_cta in/out (capacity in rows, CTAs out).
+ * Synchronises `stream`.  INVALID_ARG without MOEDEC_FLAG_TRACE.
+ */
+MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 MOEDEC_API const char *moedec_status_string(int status);

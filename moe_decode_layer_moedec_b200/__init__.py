@@ -19,6 +19,10 @@ LIB_PATH = os.path.join(_HERE, "libmoedec.so")
 ABI_VERSION = 1
 FLAG_TAPS = 1
 FLAG_SKIP_SCALE_CHECK = 2
+FLAG_TEST_STALL = 4
+FLAG_MULTI_KERNEL = 8
+FLAG_TRACE = 16
+TRACE_STAMPS = 16
 STATUS = {0: "MOEDEC_OK", -1: "MOEDEC_ERR_INVALID_ARG", -2: "MOEDEC_ERR_UNSUPPORTED", -3: "MOEDEC_ERR_CUDA",
           -4: "MOEDEC_ERR_OOM", -5: "MOEDEC_ERR_TIMEOUT", -6: "MOEDEC_ERR_DEVICE"}
 WEIGHT_NAMES = ("router", "w_down_lat", "w_up_lat", "gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s",
@@ -70,6 +74,8 @@ def _load():
     lib.moedec_profile_read.restype = i32
     lib.moedec_router_logits_noalloc.argtypes = [vp, vp, i32, i32, i32, vp, vp]
     lib.moedec_router_logits_noalloc.restype = i32
+    lib.moedec_get_trace.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(i32), vp]
+    lib.moedec_get_trace.restype = i32
     lib.moedec_kernels_per_step.argtypes = [vp, i32]
     lib.moedec_kernels_per_step.restype = i32
     lib.moedec_last_cuda_error.argtypes = [vp]
@@ -188,6 +194,14 @@ class MoeDecodeLayer:
         n = ctypes.c_int(cap)
         self._check("moedec_profile_read", lib.moedec_profile_read(self._h, ms, cnt, names, ctypes.byref(n)))
         return {names[i].decode(): (float(ms[i]), int(cnt[i])) for i in range(n.value)}
+
+    def trace(self, stream=None):
+        """Per-CTA phase timestamps (ns) of the last fused step: list of rows (FLAG_TRACE only)."""
+        cap = 1024
+        buf = (ctypes.c_uint64 * (cap * TRACE_STAMPS))()
+        n = ctypes.c_int(cap)
+        self._check("moedec_get_trace", lib.moedec_get_trace(self._h, buf, ctypes.byref(n), _stream_ptr(stream)))
+        return [[int(buf[r * TRACE_STAMPS + i]) for i in range(TRACE_STAMPS)] for r in range(n.value)]
 
     def kernels_per_step(self, batch: int) -> int:
         return int(lib.moedec_kernels_per_step(self._h, batch))

@@ -5,7 +5,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/moedec.h"
+#include "moedec.h"
 #include "moedec_internal.h"
 
 using namespace moedec;
@@ -98,6 +98,8 @@ void layout(moedec_handle *h, char *base) {
     w.up_part = c.take<float>((size_t)p.up.splits * B * d.H);
     w.up_tap = (h->cfg.flags & MOEDEC_FLAG_TAPS) ? c.take<float>(B * d.H) : nullptr;
     w.tickets = c.take<unsigned>((size_t)p.n_tickets);
+    w.ctl = c.take<unsigned>((size_t)p.ctl_words);
+    w.trace = (h->cfg.flags & MOEDEC_FLAG_TRACE) ? c.take<unsigned long long>((size_t)h->n_sm * kTraceStamps) : nullptr;
     w.err = c.take<unsigned>(1);
     h->buf_bytes = c.off;
 }
@@ -126,9 +128,13 @@ int check_scales(moedec_handle *h) {
     return host_bad ? MOEDEC_ERR_UNSUPPORTED : MOEDEC_OK;
 }
 
-enum KernelKind { K_ROUTER_DN, K_TOPK, K_EXPERT_GU, K_EXPERT_DOWN, K_COMBINE, K_UP, K_SHARED_GU, K_SHARED_DOWN, K_COUNT };
-const char *const kKernelNames[K_COUNT] = {"router_dn", "topk", "expert_gate_up", "expert_down",
-                                           "combine", "up", "shared_gate_up", "shared_down"};
+enum KernelKind {
+    K_ROUTER_DN, K_TOPK, K_EXPERT_GU, K_EXPERT_DOWN, K_COMBINE, K_UP, K_SHARED_GU, K_SHARED_DOWN, K_FUSED,
+    K_FUSED_SMALL, K_COUNT
+};
+const char *const kKernelNames[K_COUNT] = {"router_dn", "topk",        "expert_gate_up", "expert_down",
+                                           "combine",   "up",          "shared_gate_up", "shared_down",
+                                           "fused_step_splitk", "fused_step_small"};
 
 cudaEvent_t pool_get(moedec_handle *h) {
     if (!h->pool.empty()) {
@@ -229,11 +235,22 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     p.ticket_sd = p.ticket_sgu + p.sgu.blocks;
     p.ticket_topk = p.ticket_sd + p.sd.blocks;
     p.n_tickets = p.ticket_topk + 1;
+    p.ctl_gu = CTL_FIXED;
+    p.ctl_comb = p.ctl_gu + d.E;
+    p.ctl_ylat = p.ctl_comb + d.max_batch * (d.L / 16);
+    p.ctl_hamax = p.ctl_ylat + d.L / 16;
+    p.ctl_shamax = p.ctl_hamax + d.max_batch;
+    p.ctl_tk = p.ctl_shamax + d.max_batch;
+    p.ctl_tk_words = (d.E + 7) / 8 + d.L / 16 + d.Is / 16 + 2 * (d.H / 16);
+    p.ctl_words = p.ctl_tk + p.ctl_tk_words;
+    p.wait_limit_ns = (c.flags & MOEDEC_FLAG_TEST_STALL) ? 20000000LL : 1000000000LL;
 
     int rc = MOEDEC_OK;
     cudaError_t e = cudaGetDevice(&h->device);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&h->n_sm, cudaDevAttrMultiProcessorCount, h->device);
     if (e == cudaSuccess) e = init_kernel_attributes();
+    if (e == cudaSuccess) e = init_fused_attributes();
+    if (e == cudaSuccess) e = init_fused_small_attributes();
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
@@ -290,7 +307,19 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     a.x = x;
     a.out = out;
     a.B = batch;
+    a.flags = h->cfg.flags;
     cudaError_t e = cudaSuccess;
+    const int variant = batch <= 4 ? 0 : 1;
+    if (!(h->cfg.flags & MOEDEC_FLAG_MULTI_KERNEL)) {
+        if (fused_small_supports(h->d, batch))
+            e = timed(h, K_FUSED_SMALL, s, [&] { return launch_fused_small(a, s, h->n_sm); });
+        else
+            e = timed(h, K_FUSED, s, [&] { return launch_fused(a, s, h->n_sm); });
+        if (e != cudaSuccess) return record_cuda(h, e);
+        h->launches[variant] += 1;
+        h->last_batch = batch;
+        return MOEDEC_OK;
+    }
     if (h->d.n_shared) {
         e = cudaEventRecord(h->ev_fork, s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(h->side, h->ev_fork, 0);
@@ -306,7 +335,7 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     if (e == cudaSuccess && h->d.n_shared) e = cudaStreamWaitEvent(s, h->ev_join, 0);
     if (e == cudaSuccess) e = timed(h, K_UP, s, [&] { return launch_up(a, s); });
     if (e != cudaSuccess) return record_cuda(h, e);
-    h->launches[batch <= 2 ? 0 : 1] += (uint64_t)kernels_per_step(h->d);
+    h->launches[variant] += (uint64_t)kernels_per_step(h->d);
     h->last_batch = batch;
     return MOEDEC_OK;
 }
@@ -397,9 +426,20 @@ MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t 
     return MOEDEC_OK;
 }
 
+MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream) {
+    if (!h || !out || !n_cta || !h->ws.trace || *n_cta < h->n_sm) return MOEDEC_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(out, h->ws.trace, (size_t)h->n_sm * kTraceStamps * sizeof(uint64_t),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return record_cuda(h, e);
+    *n_cta = h->n_sm;
+    return MOEDEC_OK;
+}
+
 MOEDEC_API int moedec_kernels_per_step(moedec_handle *h, int batch) {
     if (!h || batch <= 0) return 0;
-    return kernels_per_step(h->d);
+    return (h->cfg.flags & MOEDEC_FLAG_MULTI_KERNEL) ? kernels_per_step(h->d) : 1;
 }
 
 }  // extern "C"

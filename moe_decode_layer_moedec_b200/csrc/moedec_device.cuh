@@ -44,10 +44,24 @@ DEVI uint4 ldg_weights_l1(const void *p) {
     return r;
 }
 
+// 4 bytes of static weights (4-byte aligned).
+DEVI uint32_t ldg_weights_u32(const void *p) {
+    uint32_t r;
+    asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    return r;
+}
+
 DEVI uint32_t ldg_weight_byte(const uint8_t *p) {
     uint16_t r;
     asm("ld.global.nc.u8 %0, [%1];" : "=h"(r) : "l"(p));
     return r;
+}
+
+// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned start) into L2; no data returns to the
+// SM and nothing waits on it.  Issued for the weights of a CTA's or warp's next work item.
+DEVI void prefetch_l2(const void *p, uint32_t bytes) {
+    if (bytes == 0 || ((reinterpret_cast<uintptr_t>(p) | bytes) & 15u)) return;  // a hint: skip odd shapes
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // ---------------------------------------------------------------------------------------------

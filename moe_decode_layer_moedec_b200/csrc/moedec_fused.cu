@@ -1,0 +1,212 @@
+// moedec_fused.cu -- the whole decode layer step as one persistent kernel.
+//
+// One CTA per SM (cooperative launch, so every CTA is resident).  The step's work items sit in
+// eight queues that every CTA drains in the same order, claiming each next item one item ahead
+// and prefetching that item's weights into L2 while the current one runs:
+//
+//   0 router row blocks        (fp64 logits)                       CTA items
+//   1 top-k, one per token     waits: all router blocks            CTA items; last builds buckets
+//   2 W_dn row blocks          (h)                                 CTA items
+//   3 shared gate/up blocks    (sh_a)                              CTA items
+//   4 expert gate/up, 16 rows  waits: buckets, all of h            warp items
+//   5 shared down blocks       waits: all of sh_a                  CTA items
+//   6 expert down, 16 rows     waits: that expert's gate/up items  warp items; combine per token
+//   7 W_up row blocks          waits: their ylat rows, all of sh   CTA items; writes out
+//
+// An item only ever waits on items of earlier queues (all of which were claimed by resident CTAs
+// before any CTA moved on), so the waits always end; each one is still bounded (a.p.wait_limit_ns).  On a timeout the CTA records MOEDEC_ERR_TIMEOUT, sets the
+// abort word and leaves; the others see the abort word in their next wait and leave too.  The
+// last CTA to leave clears the control block, so the next step starts clean either way.
+//
+// Routing is known only after queue 1, but nothing waits for a kernel boundary: while one CTA
+// ranks the experts the others already stream W_dn and the shared expert, and an expert's down
+// rows start as soon as its own gate/up rows are done.
+#include "moedec_items.cuh"
+
+namespace moedec {
+
+enum Queue { Q_ROUTER = 0, Q_TOPK, Q_DN, Q_SGU, Q_EGU, Q_SD, Q_EDOWN, Q_UP, Q_COUNT };
+
+// Batch tiers: token-column tiles of the x consumers (NTX), the shared down (NTS, hi/lo split at
+// B <= 4) and the up-projection (NTU, always hi/lo).
+template <int TIER>
+struct Tier;
+template <> struct Tier<0> { static constexpr int NTX = 1, NTS = 1, NTU = 1; static constexpr bool SPLITS = true; };
+template <> struct Tier<1> { static constexpr int NTX = 1, NTS = 1, NTU = 2; static constexpr bool SPLITS = false; };
+template <> struct Tier<2> { static constexpr int NTX = 2, NTS = 2, NTU = 4; static constexpr bool SPLITS = false; };
+template <> struct Tier<3> { static constexpr int NTX = 4, NTS = 4, NTU = 8; static constexpr bool SPLITS = false; };
+template <> struct Tier<4> { static constexpr int NTX = 8, NTS = 8, NTU = 16; static constexpr bool SPLITS = false; };
+
+__host__ __device__ inline int tier_for_batch(int B) { return B <= 4 ? 0 : B <= 8 ? 1 : B <= 16 ? 2 : B <= 32 ? 3 : 4; }
+
+template <int TIER>
+__host__ __device__ inline size_t fused_smem(const StepArgs &a) {
+    using T = Tier<TIER>;
+    size_t m = (size_t)8 * (a.p.rt.krange + 4) * sizeof(double);
+    auto mx = [&](size_t v) { m = v > m ? v : m; };
+    mx((size_t)8 * T::NTX * bf16_pitch(a.p.dn.krange) * 2);
+    mx((size_t)8 * T::NTX * f16_pitch(a.p.sgu.krange) * 2);
+    mx((size_t)8 * T::NTS * f16_pitch(a.p.sd.krange) * 2);
+    mx((size_t)8 * T::NTU * bf16_pitch(up_chunk(T::NTU, a.p.up.krange)) * 2);
+    mx((size_t)8 * expert_warp_smem(a.B));
+    return m;
+}
+
+template <int TIER>
+__global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
+    using T = Tier<TIER>;
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ TopkSmem topk;
+    __shared__ unsigned s_flag;
+    __shared__ int s_ok;
+    __shared__ int s_ent[8][kExpertTokGroup];
+    __shared__ int s_shift[8][kExpertTokGroup];
+    __shared__ int s_next;
+    unsigned *ctl = a.ws.ctl;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    bool alive = true;
+    const int n_rt = a.p.rt.blocks * a.p.rt.splits, n_dn = a.p.dn.blocks * a.p.dn.splits;
+    const int n_sgu = a.d.n_shared ? a.p.sgu.blocks * a.p.sgu.splits : 0;
+    const int n_sd = a.d.n_shared ? a.p.sd.blocks * a.p.sd.splits : 0;
+    const int n_up = a.p.up.blocks * a.p.up.splits;
+    unsigned long long *trace = a.ws.trace ? a.ws.trace + (size_t)blockIdx.x * kTraceStamps : nullptr;
+    auto stamp = [&](int i) {
+        if (trace && threadIdx.x == 0) trace[i] = global_ns();
+    };
+    stamp(0);
+
+    // Items are taken dynamically (one atomic per item on the queue head) but one item ahead: the
+    // index of the next item is claimed when the current one starts, and that item's weights are
+    // prefetched into L2 while the current one runs.
+    auto cta_queue = [&](int q, int n, auto prefetch, auto body) {
+        __syncthreads();
+        if (threadIdx.x == 0) s_next = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
+        __syncthreads();
+        int it = s_next;
+        if (it < n) prefetch(it);
+        while (alive && it < n) {
+            __syncthreads();
+            if (threadIdx.x == 0) s_next = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
+            __syncthreads();
+            const int nxt = s_next;
+            if (nxt < n) prefetch(nxt);
+            alive = body(it);
+            it = nxt;
+        }
+    };
+    auto warp_queue = [&](int q, int n, bool down, auto body) {
+        int it = 0;
+        if (lane == 0) it = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
+        it = __shfl_sync(0xffffffffu, it, 0);
+        if (it < n) warp_prefetch_expert(a, it, down);
+        int ok = 1;
+        while (ok && it < n) {
+            int nxt = 0;
+            if (lane == 0) nxt = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
+            nxt = __shfl_sync(0xffffffffu, nxt, 0);
+            if (nxt < n) warp_prefetch_expert(a, nxt, down);
+            ok = body(it) ? 1 : 0;
+            it = nxt;
+        }
+        return ok;
+    };
+
+    // 0: router
+    cta_queue(Q_ROUTER, n_rt, [&](int it) { prefetch_router(a, it); },
+              [&](int it) { item_router<true>(a, it, smem, &s_flag); return true; });
+    stamp(1);
+    // 1: top-k
+    cta_queue(Q_TOPK, a.B, [](int) {}, [&](int it) { return item_topk<true>(a, it, topk); });
+    stamp(2);
+    // 2: W_dn
+    cta_queue(Q_DN, n_dn, [&](int it) { prefetch_dn(a, it); },
+              [&](int it) { item_dn<true, T::NTX>(a, it, smem, &s_flag); return true; });
+    stamp(3);
+    // 3: shared gate/up
+    cta_queue(Q_SGU, n_sgu, [&](int it) { prefetch_sgu(a, it); },
+              [&](int it) { item_sgu<true, T::NTX>(a, it, smem, &s_flag); return true; });
+    stamp(4);
+    // 4: expert gate/up (warp items): routing and all of h must be final
+    if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
+    if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)a.p.dn.blocks, &s_ok);
+    stamp(5);
+    if (alive) {
+        const int n = __ldcg(a.ws.n_active) * (a.d.I / 16);
+        uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)warp * expert_warp_smem(a.B));
+        warp_queue(Q_EGU, n, false, [&](int it) { return warp_expert_item<true, false>(a, xs, it, s_ent[warp], s_shift[warp]); });
+    }
+    stamp(6);
+    // 5: shared down
+    cta_queue(Q_SD, n_sd, [&](int it) { prefetch_sd(a, it); },
+              [&](int it) { return item_sd<true, T::NTS, T::SPLITS>(a, it, smem, &s_flag, &s_ok); });
+    stamp(7);
+    // 6: expert down (warp items), each waits on its expert's gate/up rows
+    if (alive) {
+        __syncthreads();
+        const int n = __ldcg(a.ws.n_active) * (a.d.L / 16);
+        uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)warp * expert_warp_smem(a.B));
+        const int ok = warp_queue(Q_EDOWN, n, true,
+                                  [&](int it) { return warp_expert_item<true, true>(a, xs, it, s_ent[warp], s_shift[warp]); });
+        alive = __syncthreads_and(ok) != 0;
+    }
+    stamp(8);
+    // 7: W_up and the output
+    cta_queue(Q_UP, n_up, [&](int it) { prefetch_up(a, it); },
+              [&](int it) { return item_up<true, T::NTU>(a, it, smem, &s_flag, &s_ok); });
+    stamp(9);
+    // leave; the last CTA out clears the control block for the next step
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        s_ok = (atomicAdd(ctl + CTL_EXIT, 1u) == gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    stamp(10);
+    if (s_ok) {
+        __threadfence();
+        const int nblk = a.d.L / 16;
+        for (int i = threadIdx.x; i < CTL_FIXED; i += blockDim.x) ctl[i] = 0u;
+        for (int i = threadIdx.x; i < a.d.E; i += blockDim.x) ctl[a.p.ctl_gu + i] = 0u;
+        for (int i = threadIdx.x; i < a.B * nblk; i += blockDim.x) ctl[a.p.ctl_comb + i] = 0u;
+        for (int i = threadIdx.x; i < nblk; i += blockDim.x) ctl[a.p.ctl_ylat + i] = 0u;
+        for (int i = threadIdx.x; i < a.B; i += blockDim.x) ctl[a.p.ctl_hamax + i] = 0u;
+    }
+}
+
+template <int TIER>
+static cudaError_t launch_fused_tier(const StepArgs &a, cudaStream_t s, int n_sm) {
+    const size_t sm = fused_smem<TIER>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(n_sm);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = sm;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_fused<TIER>, a);
+}
+
+cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm) {
+    switch (tier_for_batch(a.B)) {
+        case 0: return launch_fused_tier<0>(a, s, n_sm);
+        case 1: return launch_fused_tier<1>(a, s, n_sm);
+        case 2: return launch_fused_tier<2>(a, s, n_sm);
+        case 3: return launch_fused_tier<3>(a, s, n_sm);
+        default: return launch_fused_tier<4>(a, s, n_sm);
+    }
+}
+
+cudaError_t init_fused_attributes() {
+    const void *fns[] = {(const void *)k_fused<0>, (const void *)k_fused<1>, (const void *)k_fused<2>,
+                         (const void *)k_fused<3>, (const void *)k_fused<4>};
+    for (const void *f : fns) {
+        cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace moedec

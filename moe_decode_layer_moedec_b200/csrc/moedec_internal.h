@@ -15,6 +15,8 @@ constexpr int kRouterRows = 64;    // router CTA: 8 warps x 8 rows (fp64 m8n8k4)
 constexpr int kExpertWarps = 4;    // expert kernels: 4 warps x 16 rows per item
 constexpr int kExpertRows = 64;
 constexpr int kKChunk = 512;       // activation staging chunk along K
+constexpr int kExpertTokGroup = 16;  // tokens of one expert per pass (two 8-column n-tiles)
+constexpr int kTraceStamps = 16;     // MOEDEC_TRACE_STAMPS
 
 struct Dims {
     int H, L, E, k, I, Is, n_shared, max_batch;
@@ -35,6 +37,30 @@ struct Plan {
     SplitPlan rt, dn, up, sgu, sd;
     int ticket_rt, ticket_dn, ticket_up, ticket_sgu, ticket_sd, ticket_topk;  // offsets into tickets[]
     int n_tickets;
+    // control words of the fused step (zero at rest), offsets into ctl[]
+    int ctl_gu;     // [E]           gate/up warp items finished per active-expert slot
+    int ctl_comb;   // [maxB][L/16]  expert outputs finished per (token, 16-row latent block)
+    int ctl_ylat;   // [L/16]        tokens whose ylat rows of a 16-row block are final
+    int ctl_hamax;  // [maxB]        max |h| per token (float bits)
+    int ctl_shamax; // [maxB]        max |sh_a| per token (float bits), small-batch schedule
+    int ctl_tk;     // [E/8 + L/16 + I_s/16 + 2*H/16] per-tile tickets of the small-batch schedule
+    int ctl_tk_words;
+    int ctl_words;
+    long long wait_limit_ns;  // bound of every device-side wait of the fused step
+};
+
+// fixed control words of the fused step
+enum CtlWord {
+    CTL_QHEAD = 0,      // [8] next item of each work queue
+    CTL_RT_DONE = 8,    // router row blocks whose logits are final
+    CTL_DN_DONE,        // W_dn row blocks whose h rows are final
+    CTL_SGU_DONE,       // shared gate/up row blocks whose sh_a rows are final
+    CTL_SD_DONE,        // shared down row blocks whose sh rows are final
+    CTL_ROUTE_READY,    // 1 once idx / weights / expert buckets are final
+    CTL_TOPK_TICKET,    // tokens whose top-k is written
+    CTL_EXIT,           // CTAs that left the fused kernel
+    CTL_ABORT,          // set when a bounded wait gave up; every CTA then leaves
+    CTL_FIXED = 16
 };
 
 // Device workspace of one handle (all sized for max_batch).
@@ -62,6 +88,8 @@ struct Work {
     float *up_part;     // [up.splits][maxB][H]
     float *up_tap;      // [maxB][H] or nullptr
     unsigned *tickets;  // [n_tickets]
+    unsigned *ctl;      // [ctl_words] fused-step control block (zero at rest)
+    unsigned long long *trace;  // [n_sm][kTraceStamps] phase timestamps or nullptr
     unsigned *err;      // [1] sticky device error word
 };
 
@@ -73,6 +101,7 @@ struct StepArgs {
     const uint16_t *x;  // [B][H]
     uint16_t *out;      // [B][H]
     int B;
+    unsigned flags;     // MOEDEC_FLAG_* of the handle
 };
 
 // error word bits
@@ -89,6 +118,11 @@ cudaError_t launch_up(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_shared_gate_up(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_shared_down(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_scale_check(const uint8_t *s, size_t n, unsigned *bad, cudaStream_t st);
+cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t init_fused_attributes();
+bool fused_small_supports(const Dims &d, int B);
+cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t init_fused_small_attributes();
 int kernels_per_step(const Dims &d);
 cudaError_t init_kernel_attributes();
 

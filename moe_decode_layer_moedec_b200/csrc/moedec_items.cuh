@@ -1,0 +1,715 @@
+// moedec_items.cuh -- the work items of one decode layer step.
+//
+// Each item is one unit of the step: a router row block x K range, one token's top-k, a W_dn /
+// shared-expert / W_up row block x K range (whole CTA), or 16 rows of one routed expert (one
+// warp).  The same items run in two schedules:
+//   FUSED = false  one kernel per part, ordered by the stream (moedec_kernels.cu);
+//   FUSED = true   one persistent kernel whose CTAs pull items from in-order queues and wait on
+//                  completion counters (moedec_fused.cu).
+// The fused schedule is this library's form of the "megakernel" of the Kimi K3 decode work: the
+// parts of the step no longer wait for one another at kernel boundaries, and the weights of an
+// item are streamed before its inputs are ready ("NVIDIA uses a 12,000-line Megakernel to
+// optimize Kimi K3 inference…", section 一个工程师、1.2万行代码、AI辅助开发; "快是可以生成的，可信
+// 只能证明", section 他们换掉了什么, where every technique removes waiting).
+#pragma once
+
+#include "moedec_router.cuh"
+#include "moedec_tiles.cuh"
+
+namespace moedec {
+
+constexpr unsigned kFlagTestStall = 4u;  // MOEDEC_FLAG_TEST_STALL (see include/moedec.h)
+
+// ---------------------------------------------------------------------------------------------
+// device-side synchronisation of the fused step
+
+DEVI unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+DEVI unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Thread-level bounded wait for *p >= target.  Gives up when another CTA has aborted the step,
+// or after a.p.wait_limit_ns, in which case it records kErrTimeout and sets the abort word.
+DEVI bool wait_geq(const StepArgs &a, const unsigned *p, unsigned target) {
+    if (ld_acquire(p) >= target) return true;
+    unsigned *ctl = a.ws.ctl;
+    const unsigned long long t0 = global_ns();
+    unsigned ns = 32;
+    for (;;) {
+        __nanosleep(ns);
+        if (ns < 256) ns <<= 1;
+        if (ld_acquire(p) >= target) return true;
+        if (ld_acquire(ctl + CTL_ABORT)) return false;
+        if ((long long)(global_ns() - t0) > a.p.wait_limit_ns) {
+            atomicOr(a.ws.err, kErrTimeout);
+            atomicExch(ctl + CTL_ABORT, 1u);
+            return false;
+        }
+    }
+}
+
+// CTA-wide wait (thread 0 waits; every thread returns the outcome).
+DEVI bool cta_wait_geq(const StepArgs &a, const unsigned *p, unsigned target, int *s_ok) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        *s_ok = wait_geq(a, p, target) ? 1 : 0;
+        __threadfence();
+    }
+    __syncthreads();
+    return *s_ok != 0;
+}
+
+DEVI bool warp_wait_geq(const StepArgs &a, const unsigned *p, unsigned target) {
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) {
+        ok = wait_geq(a, p, target) ? 1 : 0;
+        __threadfence();
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Publish every prior write of the CTA, then add v to *counter (all threads call it).
+DEVI void cta_signal_add(unsigned *counter, unsigned v) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) atomicAdd(counter, v);
+}
+
+DEVI void warp_signal_add(unsigned *counter, unsigned v) {
+    __threadfence();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) atomicAdd(counter, v);
+}
+
+// ---------------------------------------------------------------------------------------------
+// router: one router row block x K range (fp64 MMAs); the block's last CTA publishes logits
+
+template <bool FUSED>
+DEVI void item_router(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
+    const bool last = router_block(a, bid, smem, s_flag);
+    if (FUSED && last && !(a.flags & kFlagTestStall)) cta_signal_add(a.ws.ctl + CTL_RT_DONE, 1u);
+}
+
+// ---------------------------------------------------------------------------------------------
+// h = W_dn x: one 128-row block x K range (bf16 MMAs); the block's last CTA publishes h rows and
+// folds their per-token max |h| into the token's staging exponent
+
+template <bool FUSED, int NT>
+DEVI void item_dn(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
+    __shared__ unsigned s_amax[kMaxBatch];
+    const int L = a.d.L, H = a.d.H, B = a.B, maxB = a.d.max_batch;
+    const int rb = bid / a.p.dn.splits, ks = bid % a.p.dn.splits;
+    const int KR = a.p.dn.krange, k0 = ks * KR;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    const int pitch = bf16_pitch(KR);
+    __syncthreads();
+    stage_bf16(xs, pitch, a.x, H, B, 8 * NT, k0, KR);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    const int row0 = rb * kDenseRows + warp * 16;
+    if (row0 < L) {
+        float acc[NT][4] = {};
+        tile_bf16<NT>(a.w.w_dn, H, row0, k0, KR / 32, xs, pitch, 0, B, acc);
+        float *part = a.ws.dn_part + (size_t)ks * maxB * L;
+        tile_foreach<NT, false>(acc, B, [&](int t, int r, float v) { part[(size_t)t * L + row0 + r] = v; });
+    }
+    if (cta_ticket_last(a.ws.tickets + a.p.ticket_dn + rb, a.p.dn.splits, s_flag)) {
+        for (int t = threadIdx.x; t < B; t += blockDim.x) s_amax[t] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
+            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+            if (r >= L) continue;
+            const float s = sum_splits(a.ws.dn_part + (size_t)b * L + r, (size_t)maxB * L, a.p.dn.splits);
+            a.ws.h[(size_t)b * L + r] = s;
+            atomicMax(s_amax + b, __float_as_uint(fabsf(s)));
+        }
+        __syncthreads();
+        for (int t = threadIdx.x; t < B; t += blockDim.x) atomicMax(a.ws.ctl + a.p.ctl_hamax + t, s_amax[t]);
+        if (FUSED) cta_signal_add(a.ws.ctl + CTL_DN_DONE, 1u);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// top-k of one token (any block size >= 256, up to 4 experts per thread), then, in the last
+// token's CTA, the per-expert token buckets
+
+struct TopkSmem {
+    unsigned hist[256];
+    int warp[32];
+    unsigned key[kMaxTopK];
+    int e[kMaxTopK];
+    int rank_e[kMaxTopK];
+    float rank_s[kMaxTopK];
+    unsigned digit, want;
+    int ok;
+    unsigned flag;
+    unsigned long long mask[kMaxExperts];
+    int off[kMaxExperts];
+};
+
+template <bool FUSED>
+DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t) {
+    const int E = a.d.E, K = a.d.k, B = a.B;
+    if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, (unsigned)a.p.rt.blocks, &t.ok)) return false;
+    const int tid = threadIdx.x;
+    // thread tid owns experts 4*tid .. 4*tid+3 (index order follows thread order)
+    unsigned key[4];
+    bool valid[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = 4 * tid + i;
+        valid[i] = e < E;
+        key[i] = 0u;
+        if (valid[i]) {
+            const float lg = __ldcg(a.ws.logits + (size_t)b * E + e);
+            const float sc = (float)(1.0 / (1.0 + exp(-(double)lg)));
+            key[i] = sc >= 0.0f ? __float_as_uint(sc) : 0u;  // non-negative fp32 orders like its bits
+        }
+    }
+    // radix select of the K-th largest key, 8 bits at a time from the top
+    unsigned prefix = 0u, mask = 0u, want = (unsigned)K;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        if (tid < 256) t.hist[tid] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (valid[i] && (key[i] & mask) == prefix) atomicAdd(&t.hist[(key[i] >> shift) & 255u], 1u);
+        __syncthreads();
+        if (tid < 32) {
+            // lane l holds bins 8l..8l+7; find the bin d holding the want-th largest key
+            unsigned c[8], tot = 0u;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                c[j] = t.hist[8 * tid + j];
+                tot += c[j];
+            }
+            unsigned sfx = tot;  // inclusive suffix sum over lanes tid..31
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned v = __shfl_down_sync(0xffffffffu, sfx, o);
+                if (tid + o < 32) sfx += v;
+            }
+            const unsigned above = sfx - tot;  // keys in the bins of higher lanes (higher digits)
+            if (above < want && want <= above + tot) {
+                unsigned acc = above;
+#pragma unroll
+                for (int j = 7; j >= 0; --j) {
+                    if (acc + c[j] >= want) {
+                        t.digit = 8u * tid + j;
+                        t.want = want - acc;
+                        break;
+                    }
+                    acc += c[j];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= t.digit << shift;
+        mask |= 255u << shift;
+        want = t.want;
+    }
+    const unsigned T = prefix;  // the K-th largest key; `want` keys equal to T are taken
+    int n_eq = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) n_eq += (valid[i] && key[i] == T) ? 1 : 0;
+    int tot;
+    int eq_rank = block_exclusive_scan(n_eq, t.warp, &tot);
+    bool sel[4];
+    int n_sel = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool eq = valid[i] && key[i] == T;
+        sel[i] = (valid[i] && key[i] > T) || (eq && eq_rank < (int)want);
+        eq_rank += eq ? 1 : 0;
+        n_sel += sel[i] ? 1 : 0;
+    }
+    int pos = block_exclusive_scan(n_sel, t.warp, &tot);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        if (sel[i]) {
+            t.key[pos] = key[i];
+            t.e[pos] = 4 * tid + i;
+            ++pos;
+        }
+    __syncthreads();
+    if (tid < K) {
+        const unsigned mk = t.key[tid];
+        const int me = t.e[tid];
+        int rank = 0;
+        for (int j = 0; j < K; ++j) rank += (t.key[j] > mk) || (t.key[j] == mk && t.e[j] < me);
+        t.rank_e[rank] = me;
+        t.rank_s[rank] = __uint_as_float(mk);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float S = 0.0f;
+        for (int r = 0; r < K; ++r) S += t.rank_s[r];
+        for (int r = 0; r < K; ++r) {
+            a.ws.idx[(size_t)b * K + r] = t.rank_e[r];
+            a.ws.wts[(size_t)b * K + r] = t.rank_s[r] / S;
+        }
+    }
+    // the last token's CTA groups the B*K selections by expert
+    if (!cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
+    for (int i = tid; i < E; i += blockDim.x) t.mask[i] = 0ull;
+    __syncthreads();
+    for (int i = tid; i < B * K; i += blockDim.x) {
+        const int ex = __ldcg(a.ws.idx + i);
+        if (ex >= 0 && ex < E) atomicOr(&t.mask[ex], 1ull << (i / K));
+        else atomicOr(a.ws.err, kErrBucket);
+        a.ws.a_amax[i] = 0u;
+    }
+    __syncthreads();
+    int cnt[4], n_act_t = 0, n_ent_t = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = 4 * tid + i;
+        cnt[i] = e < E ? __popcll(t.mask[e]) : 0;
+        n_act_t += cnt[i] > 0 ? 1 : 0;
+        n_ent_t += cnt[i];
+    }
+    int n_act, n_ent;
+    int j = block_exclusive_scan(n_act_t, t.warp, &n_act);
+    int off = block_exclusive_scan(n_ent_t, t.warp, &n_ent);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = 4 * tid + i;
+        if (e < E) t.off[e] = off;
+        if (cnt[i] > 0) {
+            a.ws.active_e[j] = e;
+            a.ws.active_cnt[j] = cnt[i];
+            a.ws.active_off[j] = off;
+            ++j;
+        }
+        off += cnt[i];
+    }
+    if (tid == 0) *a.ws.n_active = n_act;
+    __syncthreads();
+    for (int i = tid; i < B * K; i += blockDim.x) {
+        const int ex = __ldcg(a.ws.idx + i), tb = i / K;
+        if (ex < 0 || ex >= E) continue;
+        a.ws.entries[t.off[ex] + __popcll(t.mask[ex] & ((1ull << tb) - 1ull))] = i;
+    }
+    if (FUSED) cta_signal_add(a.ws.ctl + CTL_ROUTE_READY, 1u);
+    return true;
+}
+
+// ylat[b][l] = sum_r w[b][r] y[b*K + r][l] in slot order (all loads issued before the sum)
+DEVI float combine_value(const StepArgs &a, int b, int l) {
+    const int L = a.d.L, K = a.d.k;
+    float wv[kMaxTopK], yv[kMaxTopK];
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r)
+        if (r < K) {
+            wv[r] = __ldcg(a.ws.wts + (size_t)b * K + r);
+            yv[r] = __ldcg(a.ws.y + ((size_t)b * K + r) * L + l);
+        }
+    float s = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kMaxTopK; ++r)
+        if (r < K) s += wv[r] * yv[r];
+    return s;
+}
+
+// ---------------------------------------------------------------------------------------------
+// routed experts: one warp = 16 rows of one active expert for up to 16 of its tokens
+
+template <int NT, bool SPLIT>
+DEVI void warp_expert_gu(const StepArgs &a, uint16_t *xs, int e, int tile, const int *ent, const int *shift, int ntok) {
+    const int L = a.d.L, I = a.d.I, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int ncols = SPLIT ? 2 * ntok : ntok;
+    const int pitch = f16_pitch(kKChunk);
+    const int row0 = tile * 16;
+    const size_t eq = (size_t)e * I * (L / 2), es = (size_t)e * I * (L / 32);
+    float accg[NT][4] = {}, accu[NT][4] = {};
+    const int K = a.d.k;
+    for (int kc0 = 0; kc0 < L; kc0 += kKChunk) {
+        const int kc = min(kKChunk, L - kc0);
+        __syncwarp();
+        stage_f16_from_f32<SPLIT>(xs, pitch, a.ws.h, L, ntok, [&](int t) { return ent[t] / K; }, shift, kc0, kc, lane, 32);
+        __syncwarp();
+        // gate rows then up rows through one copy of the tile code (one weight stream live at a time)
+#pragma unroll 1
+        for (int m = 0; m < 2; ++m) {
+            float acc[NT][4];
+#pragma unroll
+            for (int i = 0; i < NT; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = m ? accu[i][j] : accg[i][j];
+            tile_fp4<NT, false>(m ? a.w.up_q + eq : a.w.gate_q + eq, m ? a.w.up_s + es : a.w.gate_s + es, nullptr, nullptr,
+                                L / 2, L / 32, row0, kc0, kc / 128, xs, pitch, 0, ncols, acc, acc);
+#pragma unroll
+            for (int i = 0; i < NT; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (m) accu[i][j] = acc[i][j];
+                    else accg[i][j] = acc[i][j];
+                }
+        }
+    }
+    // a = silu(g) * u; the per-token max |a| over these 16 rows feeds the down item's staging
+    constexpr int PER_NT = SPLIT ? 1 : 2;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int j = 0; j < PER_NT; ++j) {
+            const int tk = SPLIT ? nt * 4 + q : nt * 8 + 2 * q + j;
+            const bool ok = tk < ntok;
+            const float sc = ok ? exp2i(shift[tk]) : 0.0f;
+            float g0, g1, u0, u1;
+            if (SPLIT) {
+                g0 = accg[nt][0] + accg[nt][1];
+                g1 = accg[nt][2] + accg[nt][3];
+                u0 = accu[nt][0] + accu[nt][1];
+                u1 = accu[nt][2] + accu[nt][3];
+            } else {
+                g0 = accg[nt][j];
+                g1 = accg[nt][2 + j];
+                u0 = accu[nt][j];
+                u1 = accu[nt][2 + j];
+            }
+            g0 *= sc;
+            g1 *= sc;
+            u0 *= sc;
+            u1 *= sc;
+            const float a0 = g0 / (1.0f + expf(-g0)) * u0, a1 = g1 / (1.0f + expf(-g1)) * u1;
+            float m = ok ? fmaxf(fabsf(a0), fabsf(a1)) : 0.0f;
+            if (ok) {
+                float *dst = a.ws.a + (size_t)ent[tk] * I + row0;
+                dst[g] = a0;
+                dst[g + 8] = a1;
+            }
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+            if (ok && g == 0) atomicMax(a.ws.a_amax + ent[tk], __float_as_uint(m));
+        }
+    }
+}
+
+// y rows of 16-row block `tile` for the warp's tokens; FUSED also combines each token's latent
+// rows once all its top-k slots have written them (counter per token and 16-row block).
+template <bool FUSED, int NT, bool SPLIT>
+DEVI void warp_expert_down(const StepArgs &a, uint16_t *xs, int e, int tile, const int *ent, const int *shift, int ntok) {
+    const int L = a.d.L, I = a.d.I, K = a.d.k, lane = threadIdx.x & 31;
+    const int ncols = SPLIT ? 2 * ntok : ntok;
+    const int pitch = f16_pitch(kKChunk);
+    const int row0 = tile * 16;
+    const size_t eq = (size_t)e * L * (I / 2), es = (size_t)e * L * (I / 32);
+    float acc[NT][4] = {};
+    for (int kc0 = 0; kc0 < I; kc0 += kKChunk) {
+        const int kc = min(kKChunk, I - kc0);
+        __syncwarp();
+        stage_f16_from_f32<SPLIT>(xs, pitch, a.ws.a, I, ntok, [&](int t) { return ent[t]; }, shift, kc0, kc, lane, 32);
+        __syncwarp();
+        tile_fp4<NT, false>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I / 2, I / 32, row0, kc0, kc / 128, xs,
+                            pitch, 0, ncols, acc, acc);
+    }
+    tile_foreach<NT, SPLIT>(acc, ntok, [&](int t, int r, float v) {
+        a.ws.y[(size_t)ent[t] * L + row0 + r] = v * exp2i(shift[t]);
+    });
+    if (!FUSED) return;
+    __threadfence();
+    __syncwarp();
+    unsigned *comb = a.ws.ctl + a.p.ctl_comb;
+    const int nblk = L / 16;
+    bool mine = false;
+    if (lane < ntok) {
+        const int b = ent[lane] / K;
+        mine = atomicAdd(comb + (size_t)b * nblk + tile, 1u) == (unsigned)(K - 1);
+    }
+    unsigned todo = __ballot_sync(0xffffffffu, mine);
+    if (todo) __threadfence();  // acquire: the other slots' y rows are visible
+    while (todo) {
+        const int tl = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int b = ent[tl] / K;
+        if (lane < 16) a.ws.ylat[(size_t)b * L + row0 + lane] = combine_value(a, b, row0 + lane);
+        warp_signal_add(a.ws.ctl + a.p.ctl_ylat + tile, 1u);
+    }
+}
+
+// One warp item: 16 rows (`tile`) of active expert slot j, all its tokens in groups of 16.
+// Returns false if the fused step was aborted while waiting.
+template <bool FUSED, bool DOWN>
+DEVI bool warp_expert_item(const StepArgs &a, uint16_t *xs, int item, int *w_ent, int *w_shift) {
+    const int tiles = (DOWN ? a.d.L : a.d.I) / 16;
+    const int j = item / tiles, tile = item % tiles, lane = threadIdx.x & 31, K = a.d.k;
+    if (FUSED && DOWN && !warp_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(a.d.I / 16))) return false;
+    const int e = __ldcg(a.ws.active_e + j), cnt = __ldcg(a.ws.active_cnt + j), off = __ldcg(a.ws.active_off + j);
+    for (int t0 = 0; t0 < cnt; t0 += kExpertTokGroup) {
+        const int ntok = min(kExpertTokGroup, cnt - t0);
+        __syncwarp();
+        if (lane < ntok) {
+            const int ent = __ldcg(a.ws.entries + off + t0 + lane);
+            w_ent[lane] = ent;
+            const unsigned amax = DOWN ? __ldcg(a.ws.a_amax + ent) : __ldcg(a.ws.ctl + a.p.ctl_hamax + ent / K);
+            w_shift[lane] = prescale_shift(__uint_as_float(amax));
+        }
+        __syncwarp();
+        if (DOWN) {
+            if (ntok <= 4) warp_expert_down<FUSED, 1, true>(a, xs, e, tile, w_ent, w_shift, ntok);
+            else if (ntok <= 8) warp_expert_down<FUSED, 1, false>(a, xs, e, tile, w_ent, w_shift, ntok);
+            else warp_expert_down<FUSED, 2, false>(a, xs, e, tile, w_ent, w_shift, ntok);
+        } else {
+            if (ntok <= 4) warp_expert_gu<1, true>(a, xs, e, tile, w_ent, w_shift, ntok);
+            else if (ntok <= 8) warp_expert_gu<1, false>(a, xs, e, tile, w_ent, w_shift, ntok);
+            else warp_expert_gu<2, false>(a, xs, e, tile, w_ent, w_shift, ntok);
+        }
+    }
+    if (FUSED && !DOWN) warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, 1u);
+    return true;
+}
+
+// smem per warp of the expert items: staged columns x (kKChunk + pad) halfs
+__host__ __device__ __forceinline__ int expert_warp_cols(int B) { return B <= 8 ? 8 : 16; }
+__host__ __device__ __forceinline__ size_t expert_warp_smem(int B) {
+    return (size_t)expert_warp_cols(B) * f16_pitch(kKChunk) * 2;
+}
+
+// ---------------------------------------------------------------------------------------------
+// combine for the multi-kernel schedule: ylat[b][l] = sum_r w[b][r] y[b*K + r][l]
+
+DEVI void combine_rows(const StepArgs &a, int b, int l) { a.ws.ylat[(size_t)b * a.d.L + l] = combine_value(a, b, l); }
+
+// ---------------------------------------------------------------------------------------------
+// up-projection: one 128-row block of W_up x K range; the block's last CTA writes
+// out = bf16(W_up ylat + sh).  ylat enters as bf16 hi/lo column pairs.
+
+template <bool FUSED, int NT>
+DEVI bool item_up(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag, int *s_ok) {
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    const int H = a.d.H, L = a.d.L, B = a.B, maxB = a.d.max_batch;
+    const int rb = bid / a.p.up.splits, ks = bid % a.p.up.splits;
+    const int KR = a.p.up.krange, k0 = ks * KR;
+    const int kc = up_chunk(NT, KR);
+    const int pitch = bf16_pitch(kc);
+    const int warp = threadIdx.x >> 5;
+    const int row0 = rb * kDenseRows + warp * 16;
+    if (FUSED) {
+        // ylat rows k0 .. k0+KR of every token must be final: one thread per 16-row block waits
+        // (they all poll at once), then the CTA agrees on the outcome
+        const int nblk = KR / 16;
+        int ok = 1;
+        if (threadIdx.x < nblk) {
+            ok = wait_geq(a, a.ws.ctl + a.p.ctl_ylat + k0 / 16 + threadIdx.x, (unsigned)B) ? 1 : 0;
+            __threadfence();
+        }
+        if (!__syncthreads_and(ok)) return false;
+    }
+    float acc[NT][4] = {};
+    for (int c0 = k0; c0 < k0 + KR; c0 += kc) {
+        __syncthreads();
+        stage_bf16split_from_f32(xs, pitch, a.ws.ylat, L, B, c0, kc);
+        for (int i = threadIdx.x; i < (8 * NT - 2 * B) * (kc / 8); i += blockDim.x) {  // unused columns
+            const int col = 2 * B + i / (kc / 8), u = i % (kc / 8);
+            *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncthreads();
+        if (row0 < H) tile_bf16<NT>(a.w.w_up, L, row0, c0, kc / 32, xs, pitch, 0, 2 * B, acc);
+    }
+    if (row0 < H) {
+        float *part = a.ws.up_part + (size_t)ks * maxB * H;
+        tile_foreach<NT, true>(acc, B, [&](int t, int r, float v) { part[(size_t)t * H + row0 + r] = v; });
+    }
+    if (cta_ticket_last(a.ws.tickets + a.p.ticket_up + rb, a.p.up.splits, s_flag)) {
+        if (FUSED && a.d.n_shared && !cta_wait_geq(a, a.ws.ctl + CTL_SD_DONE, (unsigned)a.p.sd.blocks, s_ok)) return false;
+        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
+            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+            if (r >= H) continue;
+            const float s = sum_splits(a.ws.up_part + (size_t)b * H + r, (size_t)maxB * H, a.p.up.splits);
+            if (a.ws.up_tap) a.ws.up_tap[(size_t)b * H + r] = s;
+            const float shv = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)b * H + r) : 0.0f;
+            a.out[(size_t)b * H + r] = f32_to_bf16_rne(s + shv);
+        }
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------------------------
+// shared expert.  gate/up: 128 rows of I_s (gate, then up) x K range of H; down: 128 rows of H
+// x K range of I_s.  Tokens are staged as fp16 with a per-token exponent over the K range.
+
+template <bool FUSED, int NT>
+DEVI void item_sgu(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
+    __shared__ int s_shift[kMaxBatch];
+    __shared__ unsigned s_amax[kMaxBatch];
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    const int H = a.d.H, Is = a.d.Is, B = a.B, maxB = a.d.max_batch;
+    const int rb = bid / a.p.sgu.splits, ks = bid % a.p.sgu.splits;
+    const int KR = a.p.sgu.krange, k0 = ks * KR;
+    const int pitch = f16_pitch(KR);
+    __syncthreads();
+    for (int t = threadIdx.x; t < B; t += blockDim.x) s_amax[t] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < B * (KR / 8); i += blockDim.x) {
+        const int t = i / (KR / 8), u = i % (KR / 8);
+        const uint4 v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * H + k0 + 8 * u);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
+        atomicMax(s_amax + t, __float_as_uint(m));
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < B; t += blockDim.x) s_shift[t] = prescale_shift(__uint_as_float(s_amax[t]));
+    __syncthreads();
+    stage_f16_from_bf16(xs, pitch, a.x, H, B, s_shift, k0, KR);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    const int row0 = rb * kDenseRows + warp * 16;
+    if (row0 < Is) {
+        float *part = a.ws.sgu_part + (size_t)ks * maxB * 2 * Is;
+#pragma unroll 1
+        for (int m = 0; m < 2; ++m) {
+            float acc[NT][4] = {};
+            tile_fp4<NT, false>(m ? a.w.sh_up_q : a.w.sh_gate_q, m ? a.w.sh_up_s : a.w.sh_gate_s, nullptr, nullptr, H / 2,
+                                H / 32, row0, k0, KR / 128, xs, pitch, 0, B, acc, acc);
+            tile_foreach<NT, false>(acc, B, [&](int t, int r, float v) {
+                part[(size_t)t * 2 * Is + m * Is + row0 + r] = v * exp2i(s_shift[t]);
+            });
+        }
+    }
+    if (cta_ticket_last(a.ws.tickets + a.p.ticket_sgu + rb, a.p.sgu.splits, s_flag)) {
+        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
+            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+            if (r >= Is) continue;
+            const float *p = a.ws.sgu_part + (size_t)b * 2 * Is + r;
+            const float gs = sum_splits(p, (size_t)maxB * 2 * Is, a.p.sgu.splits);
+            const float us = sum_splits(p + Is, (size_t)maxB * 2 * Is, a.p.sgu.splits);
+            a.ws.sh_a[(size_t)b * Is + r] = gs / (1.0f + expf(-gs)) * us;
+        }
+        if (FUSED) cta_signal_add(a.ws.ctl + CTL_SGU_DONE, 1u);
+    }
+}
+
+template <bool FUSED, int NT, bool SPLIT>
+DEVI bool item_sd(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag, int *s_ok) {
+    __shared__ int s_shift[kMaxBatch];
+    __shared__ unsigned s_amax[kMaxBatch];
+    if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_SGU_DONE, (unsigned)a.p.sgu.blocks, s_ok)) return false;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    const int H = a.d.H, Is = a.d.Is, B = a.B, maxB = a.d.max_batch;
+    const int rb = bid / a.p.sd.splits, ks = bid % a.p.sd.splits;
+    const int KR = a.p.sd.krange, k0 = ks * KR;
+    const int pitch = f16_pitch(KR);
+    __syncthreads();
+    for (int t = threadIdx.x; t < B; t += blockDim.x) s_amax[t] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < B * (KR / 4); i += blockDim.x) {
+        const int t = i / (KR / 4), u = i % (KR / 4);
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.ws.sh_a + (size_t)t * Is + k0) + u);
+        atomicMax(s_amax + t, __float_as_uint(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)))));
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < B; t += blockDim.x) s_shift[t] = prescale_shift(__uint_as_float(s_amax[t]));
+    __syncthreads();
+    stage_f16_from_f32<SPLIT>(xs, pitch, a.ws.sh_a, Is, B, [](int t) { return t; }, s_shift, k0, KR);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    const int row0 = rb * kDenseRows + warp * 16;
+    const int ncols = SPLIT ? 2 * B : B;
+    if (row0 < H) {
+        float acc[NT][4] = {};
+        tile_fp4<NT, false>(a.w.sh_down_q, a.w.sh_down_s, nullptr, nullptr, Is / 2, Is / 32, row0, k0, KR / 128, xs,
+                            pitch, 0, ncols, acc, acc);
+        float *part = a.ws.sd_part + (size_t)ks * maxB * H;
+        tile_foreach<NT, SPLIT>(acc, B, [&](int t, int r, float v) {
+            part[(size_t)t * H + row0 + r] = v * exp2i(s_shift[t]);
+        });
+    }
+    if (cta_ticket_last(a.ws.tickets + a.p.ticket_sd + rb, a.p.sd.splits, s_flag)) {
+        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
+            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+            if (r >= H) continue;
+            const float s = sum_splits(a.ws.sd_part + (size_t)b * H + r, (size_t)maxB * H, a.p.sd.splits);
+            a.ws.sh[(size_t)b * H + r] = s;
+        }
+        if (FUSED) cta_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
+    }
+    return true;
+}
+
+// ---------------------------------------------------------------------------------------------
+// L2 prefetch of an item's weights (issued one item ahead by the fused schedule).  CTA items
+// spread their row segments over the CTA's threads; warp items issue a few whole-tile ranges.
+
+DEVI void prefetch_rows(const void *base, size_t row_bytes, int rows, size_t off, uint32_t seg) {
+    for (int r = threadIdx.x; r < rows; r += blockDim.x)
+        prefetch_l2(static_cast<const uint8_t *>(base) + (size_t)r * row_bytes + off, seg);
+}
+
+DEVI void prefetch_router(const StepArgs &a, int bid) {
+    const int rb = bid / a.p.rt.splits, ks = bid % a.p.rt.splits, H = a.d.H;
+    const int rows = min(kRouterRows, a.d.E - rb * kRouterRows);
+    prefetch_rows(a.w.router + (size_t)rb * kRouterRows * H, (size_t)H * 2, rows, (size_t)ks * a.p.rt.krange * 2,
+                  a.p.rt.krange * 2);
+}
+
+DEVI void prefetch_dn(const StepArgs &a, int bid) {
+    const int rb = bid / a.p.dn.splits, ks = bid % a.p.dn.splits, H = a.d.H;
+    const int rows = min(kDenseRows, a.d.L - rb * kDenseRows);
+    prefetch_rows(a.w.w_dn + (size_t)rb * kDenseRows * H, (size_t)H * 2, rows, (size_t)ks * a.p.dn.krange * 2,
+                  a.p.dn.krange * 2);
+}
+
+DEVI void prefetch_up(const StepArgs &a, int bid) {
+    const int rb = bid / a.p.up.splits, ks = bid % a.p.up.splits, L = a.d.L;
+    const int rows = min(kDenseRows, a.d.H - rb * kDenseRows);
+    prefetch_rows(a.w.w_up + (size_t)rb * kDenseRows * L, (size_t)L * 2, rows, (size_t)ks * a.p.up.krange * 2,
+                  a.p.up.krange * 2);
+}
+
+// MXFP4 row block: codes (K/2 bytes per row) and scales (K/32 bytes per row) of a K range
+DEVI void prefetch_fp4_rows(const uint8_t *q, const uint8_t *s, int K, int row0, int rows, int k0, int kr) {
+    prefetch_rows(q + (size_t)row0 * (K / 2), (size_t)K / 2, rows, (size_t)k0 / 2, kr / 2);
+    prefetch_rows(s + (size_t)row0 * (K / 32), (size_t)K / 32, rows, (size_t)k0 / 32, kr / 32);
+}
+
+DEVI void prefetch_sgu(const StepArgs &a, int bid) {
+    const int rb = bid / a.p.sgu.splits, ks = bid % a.p.sgu.splits, H = a.d.H;
+    const int rows = min(kDenseRows, a.d.Is - rb * kDenseRows), kr = a.p.sgu.krange;
+    prefetch_fp4_rows(a.w.sh_gate_q, a.w.sh_gate_s, H, rb * kDenseRows, rows, ks * kr, kr);
+    prefetch_fp4_rows(a.w.sh_up_q, a.w.sh_up_s, H, rb * kDenseRows, rows, ks * kr, kr);
+}
+
+DEVI void prefetch_sd(const StepArgs &a, int bid) {
+    const int rb = bid / a.p.sd.splits, ks = bid % a.p.sd.splits, Is = a.d.Is;
+    const int rows = min(kDenseRows, a.d.H - rb * kDenseRows), kr = a.p.sd.krange;
+    prefetch_fp4_rows(a.w.sh_down_q, a.w.sh_down_s, Is, rb * kDenseRows, rows, ks * kr, kr);
+}
+
+// 16 rows of an active expert, whole K: contiguous in the row-major layout (lane 0 issues them)
+DEVI void warp_prefetch_expert(const StepArgs &a, int item, bool down) {
+    if ((threadIdx.x & 31) != 0) return;
+    const int L = a.d.L, I = a.d.I;
+    const int tiles = (down ? L : I) / 16, j = item / tiles, tile = item % tiles;
+    const int e = __ldcg(a.ws.active_e + j);
+    if (down) {
+        const size_t q0 = (size_t)e * L * (I / 2) + (size_t)tile * 16 * (I / 2), s0 = (size_t)e * L * (I / 32) + (size_t)tile * 16 * (I / 32);
+        prefetch_l2(a.w.down_q + q0, 16 * (I / 2));
+        prefetch_l2(a.w.down_s + s0, 16 * (I / 32));
+    } else {
+        const size_t q0 = (size_t)e * I * (L / 2) + (size_t)tile * 16 * (L / 2), s0 = (size_t)e * I * (L / 32) + (size_t)tile * 16 * (L / 32);
+        prefetch_l2(a.w.gate_q + q0, 16 * (L / 2));
+        prefetch_l2(a.w.up_q + q0, 16 * (L / 2));
+        prefetch_l2(a.w.gate_s + s0, 16 * (L / 32));
+        prefetch_l2(a.w.up_s + s0, 16 * (L / 32));
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// token-column tiles of each dense part for batch B
+
+__host__ __device__ __forceinline__ int nt_for_cols(int cols) {
+    return cols <= 8 ? 1 : cols <= 16 ? 2 : cols <= 32 ? 4 : cols <= 64 ? 8 : 16;
+}
+
+}  // namespace moedec

@@ -6,7 +6,7 @@
 // router weights, the tokens and the output; nothing is allocated on any call.
 #include <mutex>
 
-#include "../../include/moedec.h"
+#include "moedec.h"
 #include "moedec_internal.h"
 #include "moedec_router.cuh"
 

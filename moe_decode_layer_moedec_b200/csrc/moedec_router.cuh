@@ -9,10 +9,12 @@
 
 #include "moedec_device.cuh"
 #include "moedec_internal.h"
+#include "moedec_tiles.cuh"
 
 namespace moedec {
 
-DEVI void router_block(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
+// Returns true in every thread of the CTA that reduced its row block (the last of its splits).
+DEVI bool router_block(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
     const int E = a.d.E, H = a.d.H, B = a.B, maxB = a.d.max_batch;
     const int rb = bid / a.p.rt.splits, ks = bid % a.p.rt.splits;
     const int KR = a.p.rt.krange, k0 = ks * KR;
@@ -23,8 +25,16 @@ DEVI void router_block(const StepArgs &a, int bid, unsigned char *smem, unsigned
     const bool row_ok = row < E;
     const uint16_t *rrow = a.w.router + (size_t)(row_ok ? row : 0) * H + k0 + 8 * q;
     const int half_units = KR / 2;  // units of two doubles
+    const int nchunks = KR / 32;    // <= 16
     for (int tg = 0; tg < B; tg += 8) {
         const int ntok = min(8, B - tg);
+        // the first 8 chunks of the router rows are in flight while the tokens are staged; each
+        // further chunk is requested 8 chunks ahead of its use (L1-allocating: token groups
+        // after the first re-read these rows)
+        uint4 A[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            A[c] = (row_ok && c < nchunks) ? ldg_weights_l1(rrow + 32 * c) : make_uint4(0u, 0u, 0u, 0u);
         __syncthreads();
         for (int i = threadIdx.x; i < 8 * half_units; i += blockDim.x) {
             const int t = i / half_units, u = i % half_units;
@@ -38,36 +48,46 @@ DEVI void router_block(const StepArgs &a, int bid, unsigned char *smem, unsigned
         }
         __syncthreads();
         // m8n8k4 fp64: lane (g,q) holds A[row g][slot q] and B[slot q][token g]; MMA step s of
-        // chunk c maps slot q to k = 32c + 8q + s.
-        double c0 = 0.0, c1 = 0.0;
+        // chunk c maps slot q to k = 32c + 8q + s.  Two accumulator pairs halve the MMA chain.
+        double c0 = 0.0, c1 = 0.0, d0 = 0.0, d1 = 0.0;
         const double *xr = xs + (size_t)g * pitch;
-        for (int c = 0; c < KR / 32; ++c) {
-            const uint4 A = row_ok ? ldg_weights_l1(rrow + 32 * c) : make_uint4(0u, 0u, 0u, 0u);
-            const double av[8] = {bf16_lo(A.x), bf16_hi(A.x), bf16_lo(A.y), bf16_hi(A.y),
-                                  bf16_lo(A.z), bf16_hi(A.z), bf16_lo(A.w), bf16_hi(A.w)};
-            double2 xv[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int u = (16 * c + 4 * q + i) ^ (q >> 1);
-                xv[i] = *reinterpret_cast<const double2 *>(xr + 2 * u);
+        for (int c = 0; c < 16; ++c) {
+            if (c < nchunks) {
+                const uint4 Ac = A[c & 7];
+                if (c + 8 < nchunks) A[c & 7] = row_ok ? ldg_weights_l1(rrow + 32 * (c + 8)) : make_uint4(0u, 0u, 0u, 0u);
+                const double av[8] = {bf16_lo(Ac.x), bf16_hi(Ac.x), bf16_lo(Ac.y), bf16_hi(Ac.y),
+                                      bf16_lo(Ac.z), bf16_hi(Ac.z), bf16_lo(Ac.w), bf16_hi(Ac.w)};
+                double2 xv[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int u = (16 * c + 4 * q + i) ^ (q >> 1);
+                    xv[i] = *reinterpret_cast<const double2 *>(xr + 2 * u);
+                }
+#pragma unroll
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    mma_f64(c0, c1, av[2 * s2], xv[s2].x);
+                    mma_f64(d0, d1, av[2 * s2 + 1], xv[s2].y);
+                }
             }
-#pragma unroll
-            for (int s = 0; s < 8; ++s) mma_f64(c0, c1, av[s], (s & 1) ? xv[s >> 1].y : xv[s >> 1].x);
         }
+        c0 += d0;
+        c1 += d1;
         if (row_ok) {
             if (2 * q < ntok) a.ws.rt_part[((size_t)ks * maxB + tg + 2 * q) * E + row] = c0;
             if (2 * q + 1 < ntok) a.ws.rt_part[((size_t)ks * maxB + tg + 2 * q + 1) * E + row] = c1;
         }
     }
-    if (cta_ticket_last(a.ws.tickets + a.p.ticket_rt + rb, a.p.rt.splits, s_flag)) {
+    const bool last = cta_ticket_last(a.ws.tickets + a.p.ticket_rt + rb, a.p.rt.splits, s_flag);
+    if (last) {
         for (int i = threadIdx.x; i < kRouterRows * B; i += blockDim.x) {
             const int r = rb * kRouterRows + (i % kRouterRows), b = i / kRouterRows;
             if (r >= E) continue;
-            double s = 0.0;
-            for (int k = 0; k < a.p.rt.splits; ++k) s += __ldcg(a.ws.rt_part + ((size_t)k * maxB + b) * E + r);
+            const double s = sum_splits(a.ws.rt_part + (size_t)b * E + r, (size_t)maxB * E, a.p.rt.splits);
             a.ws.logits[(size_t)b * E + r] = (float)s;
         }
     }
+    return last;
 }
 
 }  // namespace moedec

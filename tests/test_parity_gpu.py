@@ -24,9 +24,15 @@ def torch_cuda():
     return torch
 
 
-def _make_layer(w, W_dev, max_batch, flags=None):
-    from moe_decode_layer_moedec_b200 import FLAG_TAPS, MoeDecodeLayer
-    return MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=max_batch, flags=FLAG_TAPS if flags is None else flags)
+SCHEDULES = ["fused", "multi"]
+
+
+def _make_layer(w, W_dev, max_batch, flags=None, schedule="fused"):
+    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_TAPS, MoeDecodeLayer
+    f = FLAG_TAPS if flags is None else flags
+    if schedule == "multi":
+        f |= FLAG_MULTI_KERNEL
+    return MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=max_batch, flags=f)
 
 
 def _check_step(w, W, x, layer, tokens=None, check_all_routing=True):
@@ -58,17 +64,19 @@ def tiny(torch_cuda):
     return w, W, upload_weights(W)
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("B", [1, 2, 3, 5, 8, 9, 17, 33, 64])
-def test_tiny_parity(tiny, B):
+def test_tiny_parity(tiny, B, schedule):
     w, W, W_dev = tiny
-    layer = _make_layer(w, W_dev, max_batch=64)
+    layer = _make_layer(w, W_dev, max_batch=64, schedule=schedule)
     x = synth.tokens(w, step=B, batch=B)
     _check_step(w, W, x, layer)
 
 
-def test_tiny_launch_variant_counts(tiny):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_tiny_launch_variant_counts(tiny, schedule):
     w, W, W_dev = tiny
-    layer = _make_layer(w, W_dev, max_batch=16)
+    layer = _make_layer(w, W_dev, max_batch=16, schedule=schedule)
     run_layer(layer, synth.tokens(w, batch=1))
     run_layer(layer, synth.tokens(w, batch=2))
     c = layer.launch_counts()
@@ -77,9 +85,10 @@ def test_tiny_launch_variant_counts(tiny):
     assert layer.launch_counts()["splitk"] == layer.kernels_per_step(16)
 
 
-def test_tiny_deterministic(tiny):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_tiny_deterministic(tiny, schedule):
     w, W, W_dev = tiny
-    layer = _make_layer(w, W_dev, max_batch=8)
+    layer = _make_layer(w, W_dev, max_batch=8, schedule=schedule)
     x = synth.tokens(w, batch=8)
     a = run_layer(layer, x)
     b = run_layer(layer, x)
@@ -88,12 +97,13 @@ def test_tiny_deterministic(tiny):
         assert np.array_equal(a[3][k], b[3][k]), k
 
 
-def test_tiny_back_to_back_steps_see_their_own_tokens(tiny, torch_cuda):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_tiny_back_to_back_steps_see_their_own_tokens(tiny, torch_cuda, schedule):
     # Several steps queued on one stream with different tokens, then one graph replay of two
     # steps: every output must match its own token batch (no stale activations).
     torch = torch_cuda
     w, W, W_dev = tiny
-    layer = _make_layer(w, W_dev, max_batch=4, flags=0)
+    layer = _make_layer(w, W_dev, max_batch=4, flags=0, schedule=schedule)
     xs = [synth.tokens(w, step=100 + i, batch=4) for i in range(3)]
     xd = [to_device(x) for x in xs]
     outs = [layer.step(x) for x in xd]
@@ -140,6 +150,35 @@ def test_batch_zero_and_limits(tiny, torch_cuda):
     assert lib.moedec_step(None, x.data_ptr(), 1, out.data_ptr(), s) == -1
     with pytest.raises(MoedecError):
         layer.routing(3)  # not the last step's batch
+
+
+def test_fused_wait_timeout_is_reported_and_context_stays_usable(tiny):
+    # MOEDEC_FLAG_TEST_STALL: the router never publishes its logits, so the top-k item's bounded
+    # wait runs out (20 ms); every CTA leaves and the step reports MOEDEC_ERR_TIMEOUT.
+    from moe_decode_layer_moedec_b200 import FLAG_TEST_STALL, MoedecError
+    w, W, W_dev = tiny
+    stalled = _make_layer(w, W_dev, max_batch=2, flags=FLAG_TEST_STALL)
+    x = to_device(synth.tokens(w, batch=2))
+    stalled.step(x)
+    with pytest.raises(MoedecError, match="TIMEOUT"):
+        stalled.routing(2)
+    stalled.step(x)  # the control block was cleared on the way out: it stalls again, no hang
+    with pytest.raises(MoedecError, match="TIMEOUT"):
+        stalled.routing(2)
+    stalled.close()
+    layer = _make_layer(w, W_dev, max_batch=2)
+    _check_step(w, W, synth.tokens(w, batch=2), layer)
+
+
+def test_fused_and_multi_agree(tiny):
+    w, W, W_dev = tiny
+    x = synth.tokens(w, step=5, batch=9)
+    a = run_layer(_make_layer(w, W_dev, max_batch=16, schedule="fused"), x)
+    b = run_layer(_make_layer(w, W_dev, max_batch=16, schedule="multi"), x)
+    assert np.array_equal(a[1], b[1])
+    for k in ("h", "ylat", "sh", "up"):
+        r, m = rel_errors(a[3][k], b[3][k])
+        assert r < 1e-5, (k, r)
 
 
 def test_create_rejects_bad_config(tiny):
@@ -194,27 +233,30 @@ def full_layers(torch_cuda):
     return get
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("name", ["full_b1", "full_b2"])
-def test_full_small_batches_all_tokens(full_layers, name):
+def test_full_small_batches_all_tokens(full_layers, name, schedule):
     w, W, W_dev = full_layers(name)
-    layer = _make_layer(w, W_dev, max_batch=w.batch)
+    layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
     x = synth.tokens(w)
     out, idx = _check_step(w, W, x, layer)
     if name == "full_b2":
         assert 0 < len(set(idx[0]) & set(idx[1])) < w.dims.top_k
 
 
-def test_full_b16_sampled_tokens(full_layers):
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_full_b16_sampled_tokens(full_layers, schedule):
     w, W, W_dev = full_layers("full_b16")
-    layer = _make_layer(w, W_dev, max_batch=w.batch)
+    layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
     x = synth.tokens(w)
     _check_step(w, W, x, layer, tokens=[0, 7, 15])
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("layer_idx", [0, 31])
-def test_full_b64_skewed_sampled_tokens(full_layers, layer_idx):
+def test_full_b64_skewed_sampled_tokens(full_layers, layer_idx, schedule):
     w, W, W_dev = full_layers("full_b64_skewed", layer_idx)
-    layer = _make_layer(w, W_dev, max_batch=w.batch)
+    layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
     x = synth.tokens(w)
     _, ridx_all = oracle.route(W["router"], x, w.dims.top_k)[0], oracle.route(W["router"], x, w.dims.top_k)[1]
     # sample the token with the most hot selections, one with none, and the last token
