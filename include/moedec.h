@@ -213,7 +213,8 @@ MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, const uint16
  * Phase timeline of the last fused step (MOEDEC_FLAG_TRACE): host array out[n_cta][MOEDEC_TRACE_STAMPS]
  * of %globaltimer nanoseconds, stamp i taken by CTA c when it finished phase i (0 start, 1 router,
  * 2 top-k, 3 W_dn, 4 shared gate/up, 5 routing wait, 6 expert gate/up, 7 shared down, 8 expert down,
- * 9 W_up, 10 exit; 0 where a phase was skipped).  *n_cta in/out (capacity in rows, CTAs out).
+ * 9 W_up, 10 exit; 0 where a phase was skipped).  *n_cta in/out: capacity in rows (at least 2 per SM)
+ * in, rows written out (2 per SM; rows of CTAs that the last step did not launch stay 0).
  * Synchronises `stream`.  INVALID_ARG without MOEDEC_FLAG_TRACE.
  */
 MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream);

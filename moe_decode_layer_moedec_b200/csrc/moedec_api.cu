@@ -1,4 +1,5 @@
 // moedec_api.cu -- the C ABI: argument checks, workspace, side stream, launch order.
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -48,6 +49,13 @@ bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 int krange_for(int K) { return K % 512 == 0 ? 512 : K % 256 == 0 ? 256 : 128; }
 
+// largest n <= max_n with K a multiple of n * unit (1 if none)
+int small_split(int K, int unit, int max_n) {
+    for (int n = max_n; n > 1; --n)
+        if (K % (n * unit) == 0) return n;
+    return 1;
+}
+
 SplitPlan split(int rows, int rows_per_block, int K) {
     SplitPlan s;
     s.blocks = (rows + rows_per_block - 1) / rows_per_block;
@@ -75,9 +83,9 @@ void layout(moedec_handle *h, char *base) {
     const Plan &p = h->p;
     Carver c{base};
     Work &w = h->ws;
-    w.rt_part = c.take<double>((size_t)p.rt.splits * B * d.E);
+    w.rt_part = c.take<double>((size_t)std::max(p.rt.splits, kSmallSplitRt) * B * d.E);
     w.logits = c.take<float>(B * d.E);
-    w.dn_part = c.take<float>((size_t)p.dn.splits * B * d.L);
+    w.dn_part = c.take<float>((size_t)std::max(p.dn.splits, kSmallSplitDn) * B * d.L);
     w.h = c.take<float>(B * d.L);
     w.h_shift = c.take<int>(B);
     w.idx = c.take<int>(B * d.k);
@@ -87,19 +95,20 @@ void layout(moedec_handle *h, char *base) {
     w.active_cnt = c.take<int>(d.E);
     w.active_off = c.take<int>(d.E);
     w.entries = c.take<int>(B * d.k);
+    w.egu_part = c.take<float>((size_t)kSmallSplitEgu * std::min<size_t>(B, kSmallMaxBatch) * d.k * 2 * d.I);
     w.a = c.take<float>(B * d.k * d.I);
     w.a_amax = c.take<unsigned>(B * d.k);
     w.y = c.take<float>(B * d.k * d.L);
     w.ylat = c.take<float>(B * d.L);
-    w.sgu_part = c.take<float>((size_t)p.sgu.splits * B * 2 * d.Is);
+    w.sgu_part = c.take<float>((size_t)std::max(p.sgu.splits, kSmallSplitSgu) * B * 2 * d.Is);
     w.sh_a = c.take<float>(B * d.Is);
-    w.sd_part = c.take<float>((size_t)p.sd.splits * B * d.H);
+    w.sd_part = c.take<float>((size_t)std::max(p.sd.splits, kSmallSplitSd) * B * d.H);
     w.sh = c.take<float>(B * d.H);
-    w.up_part = c.take<float>((size_t)p.up.splits * B * d.H);
+    w.up_part = c.take<float>((size_t)std::max(p.up.splits, kSmallSplitUp) * B * d.H);
     w.up_tap = (h->cfg.flags & MOEDEC_FLAG_TAPS) ? c.take<float>(B * d.H) : nullptr;
     w.tickets = c.take<unsigned>((size_t)p.n_tickets);
     w.ctl = c.take<unsigned>((size_t)p.ctl_words);
-    w.trace = (h->cfg.flags & MOEDEC_FLAG_TRACE) ? c.take<unsigned long long>((size_t)h->n_sm * kTraceStamps) : nullptr;
+    w.trace = (h->cfg.flags & MOEDEC_FLAG_TRACE) ? c.take<unsigned long long>((size_t)h->n_sm * kMaxCtasPerSm * kTraceStamps) : nullptr;
     w.err = c.take<unsigned>(1);
     h->buf_bytes = c.off;
 }
@@ -241,7 +250,13 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     p.ctl_hamax = p.ctl_ylat + d.L / 16;
     p.ctl_shamax = p.ctl_hamax + d.max_batch;
     p.ctl_tk = p.ctl_shamax + d.max_batch;
-    p.ctl_tk_words = (d.E + 7) / 8 + d.L / 16 + d.Is / 16 + 2 * (d.H / 16);
+    p.ctl_tk_words = (d.E + 7) / 8 + d.L / 16 + d.Is / 16 + 2 * (d.H / 16) + d.E * (d.I / 16);
+    p.s_rt = small_split(d.H, 32, kSmallSplitRt);
+    p.s_dn = small_split(d.H, 32, kSmallSplitDn);
+    p.s_sgu = small_split(d.H, 128, kSmallSplitSgu);
+    p.s_egu = small_split(d.L, 128, kSmallSplitEgu);
+    p.s_sd = small_split(d.Is, 128, kSmallSplitSd);
+    p.s_up = small_split(d.L, 32, kSmallSplitUp);
     p.ctl_words = p.ctl_tk + p.ctl_tk_words;
     p.wait_limit_ns = (c.flags & MOEDEC_FLAG_TEST_STALL) ? 20000000LL : 1000000000LL;
 
@@ -427,13 +442,14 @@ MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t 
 }
 
 MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream) {
-    if (!h || !out || !n_cta || !h->ws.trace || *n_cta < h->n_sm) return MOEDEC_ERR_INVALID_ARG;
+    const int rows = h ? h->n_sm * kMaxCtasPerSm : 0;
+    if (!h || !out || !n_cta || !h->ws.trace || *n_cta < rows) return MOEDEC_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(out, h->ws.trace, (size_t)h->n_sm * kTraceStamps * sizeof(uint64_t),
+    cudaError_t e = cudaMemcpyAsync(out, h->ws.trace, (size_t)rows * kTraceStamps * sizeof(uint64_t),
                                     cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return record_cuda(h, e);
-    *n_cta = h->n_sm;
+    *n_cta = rows;
     return MOEDEC_OK;
 }
 

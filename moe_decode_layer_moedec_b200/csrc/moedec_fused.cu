@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
               [&](int it) { item_router<true>(a, it, smem, &s_flag); return true; });
     stamp(1);
     // 1: top-k
-    cta_queue(Q_TOPK, a.B, [](int) {}, [&](int it) { return item_topk<true>(a, it, topk); });
+    cta_queue(Q_TOPK, a.B, [](int) {}, [&](int it) { return item_topk<true>(a, it, topk, (unsigned)a.p.rt.blocks); });
     stamp(2);
     // 2: W_dn
     cta_queue(Q_DN, n_dn, [&](int it) { prefetch_dn(a, it); },

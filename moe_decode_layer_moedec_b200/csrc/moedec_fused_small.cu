@@ -1,66 +1,176 @@
 // moedec_fused_small.cu -- the decode layer step for batches of at most 4 tokens, one persistent
-// kernel.
+// kernel of independent warps.
 //
 // This is the small-matrix variant of the step: the Kimi K3 decode work picks a small-matrix
 // kernel shape at batch 1-2 and split-K above ("快是可以生成的，可信只能证明（vLLM 重写 Kimi K3
-// 解码路径…）", section 他们换掉了什么).  With at most 4 tokens the whole activation of a part fits
-// in shared memory, so every work item covers full K: the CTA's 8 warps split K (or rows x K)
-// between them and add their accumulators in shared memory in a fixed order.  There are no
-// split-K partials in global memory and no tickets; an item's result is final when the item ends.
+// 解码路径…）", section 他们换掉了什么).  Decode at this batch is pure weight streaming, and on
+// B200 a loaded HBM access takes on the order of 2 us, so an SM must keep ~64 KB of weights in
+// flight.  Every work item is therefore a warp item (16 weight rows x a K range) that a warp
+// streams on its own with a software-pipelined register ring; warps never wait for each other
+// inside a phase, so while one warp starts an item the others keep the SM's loads in flight.
+// A CTA only synchronises when it enters a phase, to stage that phase's activations (all tokens,
+// full K) in shared memory once.  K splits of a tile are added by the warp that finishes last
+// (per-tile ticket), in split order; routed experts read the staged columns of their own tokens.
 //
-// Queues, drained in this order by every CTA (one CTA per SM, cooperative launch), each item
-// claimed one ahead so that its weights are prefetched into L2 while the previous one runs:
-//   router       8 rows x K=H       fp64 MMAs, warps split K               -> logits rows
-//   top-k        one per token      waits: all router items                -> routing, buckets
-//   W_dn         16 rows x K=H      warps split K                          -> h rows, max |h|
-//   shared g/u   32 rows x K=H      2 row tiles x 4 K quarters, gate+up    -> sh_a rows
-//   expert g/u   128 rows of one    waits: buckets, all of h               -> a rows
-//                expert, K=L        one 16-row tile per warp
-//   shared down  64 rows x K=I_s    4 row tiles x 2 K halves               -> sh rows
-//   expert down  128 rows of one    waits: the expert's g/u items          -> y rows; the item that
-//                expert, K=I        one 16-row tile per warp                 completes a token's 128
-//                                                                            rows combines them to ylat
-//   W_up         64 rows x K=L      4 row tiles x 2 K halves; waits: ylat, sh -> out rows
+// Phases, in order (each CTA claims items from one queue at a time):
+//   router       8 rows x K/4            fp64 MMAs                    -> logits (per 8 rows)
+//   top-k        one CTA per token       waits: all logits            -> routing, buckets
+//   W_dn         16 rows x K/4           bf16 MMAs                    -> h rows, max |h|
+//   shared g/u   16 rows x K/4, g and u  MXFP4, x staged as fp16      -> sh_a rows, max |sh_a|
+//   expert g/u   16 rows of one expert   waits: buckets, all of h     -> a rows, max |a|
+//   shared down  16 rows x K/2           waits: all of sh_a           -> sh rows
+//   expert down  16 rows of one expert   waits: its g/u rows          -> y rows; completing a token's
+//                                                                        16 rows combines them (ylat)
+//   W_up         16 rows x K/2           waits: ylat, sh              -> out rows
+#include <algorithm>
+
 #include "moedec_items.cuh"
 
 namespace moedec {
 
-constexpr int kFsRouterRows = 8, kFsDnRows = 16, kFsSguRows = 32, kFsExpRows = 128, kFsSdRows = 64, kFsUpRows = 64;
-enum SmallQueue { Q_ROUTER_S = 0, Q_TOPK_S, Q_DN_S, Q_SGU_S, Q_EGU_S, Q_SD_S, Q_EDOWN_S, Q_UP_S };
+enum SmallQueue { QS_ROUTER = 0, QS_TOPK, QS_DN, QS_SGU, QS_EGU, QS_SD, QS_EDOWN, QS_UP };
+constexpr int kWarps = 8;
+constexpr size_t kSmallSmemLimit = 100 * 1024;  // dynamic shared memory of one CTA (two CTAs per SM)
 
-struct FsSmem {
-    double rd[8][32][2];  // router partials of the 8 warps
-    float rf[8][32][8];   // tile accumulators of the 8 warps (gate and up)
-    int ent[8];
-    int shift[8];
-    int xshift[8];
-    int flag[8];
-    int ok;
-    int item;
-};
+// ---------------------------------------------------------------------------------------------
+// one 16-row tile x one 8-column token tile; `col` is the staged column that this lane's MMA
+// column (g) reads, or -1 for a zero operand
 
-// prefetch `bytes` (multiple of 16) starting at p into L2, 32 KB per thread
-DEVI void fs_prefetch(const void *p, size_t bytes) {
-    const size_t piece = 32768;
-    const size_t n = (bytes + piece - 1) / piece;
-    for (size_t i = threadIdx.x; i < n; i += blockDim.x) {
-        const size_t off = i * piece;
-        const size_t len = bytes - off < piece ? bytes - off : piece;
-        prefetch_l2(static_cast<const uint8_t *>(p) + off, (uint32_t)len);
+template <int D>
+DEVI void s_bf16(const uint16_t *__restrict__ W, size_t ldw, int row0, int kg, int nrounds, const uint16_t *xs,
+                 int pitch, int kofs, int col, float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const uint16_t *wa = W + (size_t)(row0 + g) * ldw + kg + 8 * q;
+    const uint16_t *wb = wa + 8 * ldw;
+    const uint16_t *xr = xs + (size_t)(col >= 0 ? col : 0) * pitch + kofs + 8 * q;
+    float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+    uint4 A[D], Bm[D];
+#pragma unroll
+    for (int s = 0; s < D; ++s)
+        if (s < nrounds) {
+            A[s] = ldg_weights(wa + 32 * s);
+            Bm[s] = ldg_weights(wb + 32 * s);
+        }
+    for (int r0 = 0; r0 < nrounds; r0 += D) {
+#pragma unroll
+        for (int s = 0; s < D; ++s) {
+            const int r = r0 + s;
+            if (r < nrounds) {
+                const uint4 a = A[s], b = Bm[s];
+                if (r + D < nrounds) {
+                    A[s] = ldg_weights(wa + 32 * (r + D));
+                    Bm[s] = ldg_weights(wb + 32 * (r + D));
+                }
+                uint4 xb = make_uint4(0u, 0u, 0u, 0u);
+                if (col >= 0) xb = *reinterpret_cast<const uint4 *>(xr + 32 * r);
+                mma_bf16(acc, a.x, b.x, a.y, b.y, xb.x, xb.y);
+                mma_bf16(acc2, a.z, b.z, a.w, b.w, xb.z, xb.w);
+            }
+        }
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] += acc2[j];
 }
 
-// ---- router: 8 rows, full K; warp w sums k in [w*H/8, (w+1)*H/8) ---------------------------------
+template <int D, bool PAIR>
+DEVI void s_fp4(const uint8_t *__restrict__ Qa, const uint8_t *__restrict__ Sa, const uint8_t *__restrict__ Qb,
+                const uint8_t *__restrict__ Sb, size_t ldq, size_t lds, int row0, int kg, int nrounds, const uint16_t *xs,
+                int pitch, int kofs, int col, float (&acc)[4], float (&acc2)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const size_t ra = (size_t)(row0 + g), rb = ra + 8;
+    const uint8_t *qa0 = Qa + ra * ldq + kg / 2 + 16 * q, *qa1 = Qa + rb * ldq + kg / 2 + 16 * q;
+    const uint8_t *sa0 = Sa + ra * lds + kg / 32, *sa1 = Sa + rb * lds + kg / 32;
+    const uint8_t *qb0 = qa0, *qb1 = qa1, *sb0 = sa0, *sb1 = sa1;
+    if (PAIR) {
+        qb0 = Qb + ra * ldq + kg / 2 + 16 * q;
+        qb1 = Qb + rb * ldq + kg / 2 + 16 * q;
+        sb0 = Sb + ra * lds + kg / 32;
+        sb1 = Sb + rb * lds + kg / 32;
+    }
+    const uint16_t *xc = xs + (size_t)(col >= 0 ? col : 0) * pitch;
+    const int ubase = kofs / 8 + 4 * q, flip = q >> 1, sh = 8 * q;
+    float odd[4] = {0.f, 0.f, 0.f, 0.f};  // second MMA of each step pair: an independent chain
+    Fp4Round fa[D], fb[PAIR ? D : 1];
+#pragma unroll
+    for (int s = 0; s < D; ++s)
+        if (s < nrounds) {
+            fp4_load(fa[s], qa0, qa1, sa0, sa1, s);
+            if (PAIR) fp4_load(fb[PAIR ? s : 0], qb0, qb1, sb0, sb1, s);
+        }
+    for (int r0 = 0; r0 < nrounds; r0 += D) {
+#pragma unroll
+        for (int s = 0; s < D; ++s) {
+            const int r = r0 + s;
+            if (r < nrounds) {
+                const Fp4Round a = fa[s];
+                Fp4Round b = a;
+                if (PAIR) b = fb[PAIR ? s : 0];
+                if (r + D < nrounds) {
+                    fp4_load(fa[s], qa0, qa1, sa0, sa1, r + D);
+                    if (PAIR) fp4_load(fb[PAIR ? s : 0], qb0, qb1, sb0, sb1, r + D);
+                }
+                const uint32_t fa0 = e8m0_to_f16x2((a.s0 >> sh) & 0xffu), fa1 = e8m0_to_f16x2((a.s1 >> sh) & 0xffu);
+                const uint32_t fb0 = e8m0_to_f16x2((b.s0 >> sh) & 0xffu), fb1 = e8m0_to_f16x2((b.s1 >> sh) & 0xffu);
+                const uint32_t wa0[4] = {a.c0.x, a.c0.y, a.c0.z, a.c0.w}, wa1[4] = {a.c1.x, a.c1.y, a.c1.z, a.c1.w};
+                const uint32_t wb0[4] = {b.c0.x, b.c0.y, b.c0.z, b.c0.w}, wb1[4] = {b.c1.x, b.c1.y, b.c1.z, b.c1.w};
+                const int u = ubase + 16 * r;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (col >= 0) v = *reinterpret_cast<const uint4 *>(xc + 8 * ((u + w) ^ flip));
+                    uint32_t d0[4], d1[4];
+                    fp4_decode_word(wa0[w], fa0, d0);
+                    fp4_decode_word(wa1[w], fa1, d1);
+                    mma_f16(acc, d0[0], d1[0], d0[1], d1[1], v.x, v.y);
+                    if (PAIR) {
+                        mma_f16(acc, d0[2], d1[2], d0[3], d1[3], v.z, v.w);
+                        uint32_t e0[4], e1[4];
+                        fp4_decode_word(wb0[w], fb0, e0);
+                        fp4_decode_word(wb1[w], fb1, e1);
+                        mma_f16(acc2, e0[0], e1[0], e0[1], e1[1], v.x, v.y);
+                        mma_f16(acc2, e0[2], e1[2], e0[3], e1[3], v.z, v.w);
+                    } else {
+                        mma_f16(odd, d0[2], d1[2], d0[3], d1[3], v.z, v.w);
+                    }
+                }
+            }
+        }
+    }
+    if (!PAIR)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] += odd[j];
+}
 
-DEVI void fs_router(const StepArgs &a, int item, const uint16_t *xs, FsSmem &f) {
-    const int E = a.d.E, H = a.d.H, B = a.B;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int row = item * kFsRouterRows + g;
+// ---------------------------------------------------------------------------------------------
+// warp-level ticket: publish this warp's partial, count it; true (in every lane) for the warp
+// that completes the tile, which then owns every partial of it
+
+DEVI bool warp_ticket_last(unsigned *counter, unsigned expected) {
+    __threadfence();
+    __syncwarp();
+    unsigned last = 0;
+    if ((threadIdx.x & 31) == 0) {
+        last = (atomicAdd(counter, 1u) == expected - 1u) ? 1u : 0u;
+        if (last) *counter = 0u;  // every other split has counted already
+    }
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (last) __threadfence();  // acquire the other splits' partials
+    return last != 0;
+}
+
+// ---------------------------------------------------------------------------------------------
+// warp items
+
+// router: 8 rows x K/s_rt (fp64 m8n8k4; slot q of step s of chunk c holds k = 32c + 8q + s)
+DEVI void w_router(const StepArgs &a, int item, const uint16_t *xs) {
+    const int E = a.d.E, H = a.d.H, B = a.B, maxB = a.d.max_batch;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int rg = item / a.p.s_rt, ks = item % a.p.s_rt;
+    const int row = rg * 8 + g;
     const bool row_ok = row < E;
-    const int KW = H / 8, k0 = warp * KW, nch = KW / 32;
-    const int pitch = bf16_pitch(H);
+    const int KW = H / a.p.s_rt, k0 = ks * KW, nch = KW / 32;
     const uint16_t *rrow = a.w.router + (size_t)(row_ok ? row : 0) * H + k0 + 8 * q;
-    const uint16_t *xr = xs + (size_t)g * pitch + k0 + 8 * q;
+    const uint16_t *xr = xs + (size_t)(g < B ? g : 0) * bf16_pitch(H) + k0 + 8 * q;
     double c0 = 0.0, c1 = 0.0, d0 = 0.0, d1 = 0.0;
     constexpr int D = 8;
     uint4 A[D];
@@ -73,12 +183,12 @@ DEVI void fs_router(const StepArgs &a, int item, const uint16_t *xs, FsSmem &f) 
             if (c < nch) {
                 const uint4 Ac = A[s];
                 if (c + D < nch) A[s] = row_ok ? ldg_weights(rrow + 32 * (c + D)) : make_uint4(0u, 0u, 0u, 0u);
-                const uint4 xb = *reinterpret_cast<const uint4 *>(xr + 32 * c);
+                uint4 xb = make_uint4(0u, 0u, 0u, 0u);
+                if (g < B) xb = *reinterpret_cast<const uint4 *>(xr + 32 * c);
                 const double av[8] = {bf16_lo(Ac.x), bf16_hi(Ac.x), bf16_lo(Ac.y), bf16_hi(Ac.y),
                                       bf16_lo(Ac.z), bf16_hi(Ac.z), bf16_lo(Ac.w), bf16_hi(Ac.w)};
                 const double xv[8] = {bf16_lo(xb.x), bf16_hi(xb.x), bf16_lo(xb.y), bf16_hi(xb.y),
                                       bf16_lo(xb.z), bf16_hi(xb.z), bf16_lo(xb.w), bf16_hi(xb.w)};
-                // m8n8k4 step s of chunk c: slot q holds k = 32c + 8q + s
 #pragma unroll
                 for (int s2 = 0; s2 < 4; ++s2) {
                     mma_f64(c0, c1, av[2 * s2], xv[2 * s2]);
@@ -87,409 +197,414 @@ DEVI void fs_router(const StepArgs &a, int item, const uint16_t *xs, FsSmem &f) 
             }
         }
     }
-    f.rd[warp][lane][0] = c0 + d0;
-    f.rd[warp][lane][1] = c1 + d1;
-    __syncthreads();
-    if (warp == 0 && row_ok) {
-        double s0 = 0.0, s1 = 0.0;
-        for (int w = 0; w < 8; ++w) {
-            s0 += f.rd[w][lane][0];
-            s1 += f.rd[w][lane][1];
-        }
-        if (2 * q < B) a.ws.logits[(size_t)(2 * q) * E + row] = (float)s0;
-        if (2 * q + 1 < B) a.ws.logits[(size_t)(2 * q + 1) * E + row] = (float)s1;
+    c0 += d0;
+    c1 += d1;
+    if (row_ok) {
+        if (2 * q < B) a.ws.rt_part[((size_t)ks * maxB + 2 * q) * E + row] = c0;
+        if (2 * q + 1 < B) a.ws.rt_part[((size_t)ks * maxB + 2 * q + 1) * E + row] = c1;
     }
-    if (!(a.flags & kFlagTestStall)) cta_signal_add(a.ws.ctl + CTL_RT_DONE, 1u);
-    else __syncthreads();
+    if (!warp_ticket_last(a.ws.ctl + a.p.ctl_tk + rg, a.p.s_rt)) return;
+    if (row_ok)
+        for (int j = 0; j < 2; ++j) {
+            const int b = 2 * q + j;
+            if (b < B) a.ws.logits[(size_t)b * E + row] = (float)sum_splits(a.ws.rt_part + (size_t)b * E + row, (size_t)maxB * E, a.p.s_rt);
+        }
+    if (!(a.flags & kFlagTestStall)) warp_signal_add(a.ws.ctl + CTL_RT_DONE, 1u);
 }
 
-// ---- reduction of per-warp accumulators in shared memory -----------------------------------------
+// W_dn: 16 rows x K/s_dn
+DEVI void w_dn(const StepArgs &a, int item, const uint16_t *xs) {
+    const int L = a.d.L, H = a.d.H, B = a.B, maxB = a.d.max_batch;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int tile = item / a.p.s_dn, ks = item % a.p.s_dn, row0 = tile * 16;
+    const int KW = H / a.p.s_dn, k0 = ks * KW;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    s_bf16<6>(a.w.w_dn, H, row0, k0, KW / 32, xs, bf16_pitch(H), k0, g < B ? g : -1, acc);
+    float *part = a.ws.dn_part + (size_t)ks * maxB * L;
+    for (int j = 0; j < 2; ++j)
+        if (2 * q + j < B) {
+            part[(size_t)(2 * q + j) * L + row0 + g] = acc[j];
+            part[(size_t)(2 * q + j) * L + row0 + g + 8] = acc[2 + j];
+        }
+    if (!warp_ticket_last(a.ws.ctl + a.p.ctl_tk + (a.d.E + 7) / 8 + tile, a.p.s_dn)) return;
+    for (int j = 0; j < 2; ++j) {
+        const int b = 2 * q + j;
+        float m = 0.0f;
+        if (b < B)
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int r = row0 + g + 8 * h2;
+                const float v = sum_splits(a.ws.dn_part + (size_t)b * L + r, (size_t)maxB * L, a.p.s_dn);
+                a.ws.h[(size_t)b * L + r] = v;
+                m = fmaxf(m, fabsf(v));
+            }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        if (b < B && g == 0) atomicMax(a.ws.ctl + a.p.ctl_hamax + b, __float_as_uint(m));
+    }
+    warp_signal_add(a.ws.ctl + CTL_DN_DONE, 1u);
+}
 
-// Sum the accumulators (n floats per lane) of warps w0, w0+ws, ..., (cnt warps) in that order.
-DEVI void fs_sum(const FsSmem &f, int w0, int wstride, int cnt, int n, float *out) {
+// shared gate/up: 16 rows of gate and up x K/s_sgu; x staged as fp16 * 2^-xshift[token]
+DEVI void w_sgu(const StepArgs &a, int item, const uint16_t *xs16, const int *xshift) {
+    const int H = a.d.H, Is = a.d.Is, B = a.B, maxB = a.d.max_batch;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int tile = item / a.p.s_sgu, ks = item % a.p.s_sgu, row0 = tile * 16;
+    const int KW = H / a.p.s_sgu, k0 = ks * KW;
+    float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
+    s_fp4<3, true>(a.w.sh_gate_q, a.w.sh_gate_s, a.w.sh_up_q, a.w.sh_up_s, H / 2, H / 32, row0, k0, KW / 128, xs16,
+                   f16_pitch(H), k0, g < B ? g : -1, accg, accu);
+    float *part = a.ws.sgu_part + (size_t)ks * maxB * 2 * Is;
+    for (int j = 0; j < 2; ++j)
+        if (2 * q + j < B) {
+            float *p = part + (size_t)(2 * q + j) * 2 * Is + row0;
+            p[g] = accg[j];
+            p[g + 8] = accg[2 + j];
+            p[Is + g] = accu[j];
+            p[Is + g + 8] = accu[2 + j];
+        }
+    const int tk = a.p.ctl_tk + (a.d.E + 7) / 8 + a.d.L / 16 + tile;
+    if (!warp_ticket_last(a.ws.ctl + tk, a.p.s_sgu)) return;
+    for (int j = 0; j < 2; ++j) {
+        const int b = 2 * q + j;
+        float m = 0.0f;
+        if (b < B) {
+            const float sc = exp2i(xshift[b]);
+            const float *p = a.ws.sgu_part + (size_t)b * 2 * Is;
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int r = row0 + g + 8 * h2;
+                const float gs = sum_splits(p + r, (size_t)maxB * 2 * Is, a.p.s_sgu) * sc;
+                const float us = sum_splits(p + Is + r, (size_t)maxB * 2 * Is, a.p.s_sgu) * sc;
+                const float v = gs / (1.0f + expf(-gs)) * us;
+                a.ws.sh_a[(size_t)b * Is + r] = v;
+                m = fmaxf(m, fabsf(v));
+            }
+        }
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        if (b < B && g == 0) atomicMax(a.ws.ctl + a.p.ctl_shamax + b, __float_as_uint(m));
+    }
+    warp_signal_add(a.ws.ctl + CTL_SGU_DONE, 1u);
+}
+
+// this warp's entries of active expert slot j: ent[i] for i < cnt (lane i holds entry i)
+struct Entries {
+    int e, cnt, my_ent;
+};
+
+DEVI Entries warp_entries(const StepArgs &a, int j) {
     const int lane = threadIdx.x & 31;
-    for (int i = 0; i < n; ++i) out[i] = 0.0f;
-    for (int k = 0; k < cnt; ++k)
-        for (int i = 0; i < n; ++i) out[i] += f.rf[w0 + k * wstride][lane][i];
+    Entries r;
+    r.e = __ldcg(a.ws.active_e + j);
+    r.cnt = __ldcg(a.ws.active_cnt + j);
+    const int off = __ldcg(a.ws.active_off + j);
+    r.my_ent = lane < r.cnt ? __ldcg(a.ws.entries + off + lane) : 0;
+    return r;
 }
 
-// ---- W_dn: 16 rows, full K; warp w sums k in [w*H/8, (w+1)*H/8) ----------------------------------
-
-DEVI void fs_dn(const StepArgs &a, int item, const uint16_t *xs, FsSmem &f) {
-    const int L = a.d.L, H = a.d.H, B = a.B;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int row0 = item * kFsDnRows, KW = H / 8, k0 = warp * KW;
-    float acc[1][4] = {};
-    tile_bf16<1>(a.w.w_dn, H, row0, k0, KW / 32, xs, bf16_pitch(H), k0, B, acc);
-    for (int j = 0; j < 4; ++j) f.rf[warp][lane][j] = acc[0][j];
-    __syncthreads();
-    if (warp == 0) {
-        float v[4];
-        fs_sum(f, 0, 1, 8, 4, v);
-        // lane holds rows g, g+8 for tokens 2q, 2q+1
-        for (int j = 0; j < 2; ++j) {
-            const int t = 2 * q + j;
-            float m = 0.0f;
-            if (t < B) {
-                a.ws.h[(size_t)t * L + row0 + g] = v[j];
-                a.ws.h[(size_t)t * L + row0 + g + 8] = v[2 + j];
-                m = fmaxf(fabsf(v[j]), fabsf(v[2 + j]));
-            }
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-            if (t < B && g == 0) atomicMax(a.ws.ctl + a.p.ctl_hamax + t, __float_as_uint(m));
-        }
-    }
-    cta_signal_add(a.ws.ctl + CTL_DN_DONE, 1u);
-}
-
-// ---- shared gate/up: 32 rows (2 tiles) x full K (4 quarters), gate and up together ----------------
-
-DEVI void fs_sgu(const StepArgs &a, int item, const uint16_t *xs16, FsSmem &f) {
-    const int H = a.d.H, Is = a.d.Is, B = a.B;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int tile = warp >> 2, kq = warp & 3;
-    const int row0 = item * kFsSguRows + tile * 16, KW = H / 4, k0 = kq * KW;
-    float accg[1][4] = {}, accu[1][4] = {};
-    tile_fp4<1, true>(a.w.sh_gate_q, a.w.sh_gate_s, a.w.sh_up_q, a.w.sh_up_s, H / 2, H / 32, row0, k0, KW / 128, xs16,
-                      f16_pitch(H), k0, B, accg, accu);
-    for (int j = 0; j < 4; ++j) {
-        f.rf[warp][lane][j] = accg[0][j];
-        f.rf[warp][lane][4 + j] = accu[0][j];
-    }
-    __syncthreads();
-    if (kq == 0) {
-        float v[8];
-        fs_sum(f, warp, 1, 4, 8, v);
-        for (int j = 0; j < 2; ++j) {
-            const int t = 2 * q + j;
-            float m = 0.0f;
-            if (t < B) {
-                const float sc = exp2i(f.xshift[t]);
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const float gg = v[j + 2 * h2] * sc, uu = v[4 + j + 2 * h2] * sc;
-                    const float av = gg / (1.0f + expf(-gg)) * uu;
-                    a.ws.sh_a[(size_t)t * Is + row0 + g + 8 * h2] = av;
-                    m = fmaxf(m, fabsf(av));
-                }
-            }
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-            if (t < B && g == 0) atomicMax(a.ws.ctl + a.p.ctl_shamax + t, __float_as_uint(m));
-        }
-    }
-    cta_signal_add(a.ws.ctl + CTL_SGU_DONE, 1u);
-}
-
-// ---- expert gate/up: 128 rows of one active expert, full K, one 16-row tile per warp --------------
-
-DEVI void fs_egu(const StepArgs &a, int item, uint16_t *xs, FsSmem &f) {
-    const int L = a.d.L, I = a.d.I, K = a.d.k;
-    const int blocks = I / kFsExpRows, j = item / blocks, blk = item % blocks;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int e = __ldcg(a.ws.active_e + j), cnt = __ldcg(a.ws.active_cnt + j), off = __ldcg(a.ws.active_off + j);
-    __syncthreads();  // the previous item is done with xs and f.ent
-    if (threadIdx.x < cnt) {
-        const int en = __ldcg(a.ws.entries + off + threadIdx.x);
-        f.ent[threadIdx.x] = en;
-        f.shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(a.ws.ctl + a.p.ctl_hamax + en / K)));
-    }
-    __syncthreads();
-    stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, cnt, [&](int t) { return f.ent[t] / K; }, f.shift, 0, L);
-    __syncthreads();
-    const int row0 = blk * kFsExpRows + warp * 16;
-    const size_t eq = (size_t)e * I * (L / 2), es = (size_t)e * I * (L / 32);
-    float accg[1][4] = {}, accu[1][4] = {};
-    tile_fp4<1, true>(a.w.gate_q + eq, a.w.gate_s + es, a.w.up_q + eq, a.w.up_s + es, L / 2, L / 32, row0, 0, L / 128, xs,
-                      f16_pitch(L), 0, 2 * cnt, accg, accu);
-    // hi/lo columns: token q's values are (acc[0]+acc[1]) for row g and (acc[2]+acc[3]) for row g+8
-    const int t = q;
-    const bool ok = t < cnt;
-    const float sc = ok ? exp2i(f.shift[t]) : 0.0f;
-    const float g0 = (accg[0][0] + accg[0][1]) * sc, g1 = (accg[0][2] + accg[0][3]) * sc;
-    const float u0 = (accu[0][0] + accu[0][1]) * sc, u1 = (accu[0][2] + accu[0][3]) * sc;
-    const float a0 = g0 / (1.0f + expf(-g0)) * u0, a1 = g1 / (1.0f + expf(-g1)) * u1;
-    float m = ok ? fmaxf(fabsf(a0), fabsf(a1)) : 0.0f;
+// expert gate/up: 16 rows of active expert slot j x K/s_egu; h of all tokens staged as fp16
+// hi/lo columns (2b, 2b+1) with a per-token exponent; the last split applies silu(gate) * up
+DEVI void w_egu(const StepArgs &a, int item, const uint16_t *hs, const int *hshift) {
+    const int L = a.d.L, I = a.d.I, K = a.d.k, S = a.p.s_egu;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int tiles = I / 16, ks = item % S, jt = item / S, j = jt / tiles, row0 = (jt % tiles) * 16;
+    const int KW = L / S, k0 = ks * KW;
+    const Entries en = warp_entries(a, j);
+    // MMA column g: entry g/2, hi (g even) or lo (g odd) part of its token's staged h
+    const int ent_g = __shfl_sync(0xffffffffu, en.my_ent, (g >> 1) & 31);
+    const int col = (g >> 1) < en.cnt ? 2 * (ent_g / K) + (g & 1) : -1;
+    const size_t eq = (size_t)en.e * I * (L / 2), es = (size_t)en.e * I * (L / 32);
+    float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
+    s_fp4<2, true>(a.w.gate_q + eq, a.w.gate_s + es, a.w.up_q + eq, a.w.up_s + es, L / 2, L / 32, row0, k0, KW / 128, hs,
+                   f16_pitch(L), k0, col, accg, accu);
+    // accumulator columns 2q, 2q+1 are entry q's hi and lo parts
+    const int ent_q = __shfl_sync(0xffffffffu, en.my_ent, q);
+    const bool ok = q < en.cnt;
+    const size_t nent = (size_t)(a.B < kSmallMaxBatch ? a.B : kSmallMaxBatch) * K;  // entries per split
     if (ok) {
-        float *dst = a.ws.a + (size_t)f.ent[t] * I + row0;
-        dst[g] = a0;
-        dst[g + 8] = a1;
+        float *p = a.ws.egu_part + ((size_t)ks * nent + ent_q) * 2 * I + row0;
+        p[g] = accg[0] + accg[1];
+        p[g + 8] = accg[2] + accg[3];
+        p[I + g] = accu[0] + accu[1];
+        p[I + g + 8] = accu[2] + accu[3];
+    }
+    const int tk = a.p.ctl_tk + (a.d.E + 7) / 8 + a.d.L / 16 + a.d.Is / 16 + 2 * (a.d.H / 16) + jt;
+    if (S > 1 && !warp_ticket_last(a.ws.ctl + tk, (unsigned)S)) return;
+    float m = 0.0f;
+    if (ok) {
+        const float sc = exp2i(hshift[ent_q / K]);
+        const float *p = a.ws.egu_part + (size_t)ent_q * 2 * I + row0;
+        const size_t st = nent * 2 * I;
+        float *dst = a.ws.a + (size_t)ent_q * I + row0;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = g + 8 * h2;
+            const float gs = (S > 1 ? sum_splits(p + r, st, S) : __ldcg(p + r)) * sc;
+            const float us = (S > 1 ? sum_splits(p + I + r, st, S) : __ldcg(p + I + r)) * sc;
+            const float v = gs / (1.0f + expf(-gs)) * us;
+            dst[r] = v;
+            m = fmaxf(m, fabsf(v));
+        }
     }
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-    if (ok && g == 0) atomicMax(a.ws.a_amax + f.ent[t], __float_as_uint(m));
-    cta_signal_add(a.ws.ctl + a.p.ctl_gu + j, 1u);
+    if (ok && g == 0) atomicMax(a.ws.a_amax + ent_q, __float_as_uint(m));
+    warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, 1u);
 }
 
-// ---- shared down: 64 rows x full K (2 halves); sh_a staged once per CTA ----------------------------
-
-DEVI void fs_sd(const StepArgs &a, int item, const uint16_t *xs, FsSmem &f) {
-    const int H = a.d.H, Is = a.d.Is, B = a.B;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int tile = warp & 3, kh = warp >> 2;
-    const int row0 = item * kFsSdRows + tile * 16, KW = Is / 2, k0 = kh * KW;
-    float acc[1][4] = {};
-    tile_fp4<1, false>(a.w.sh_down_q, a.w.sh_down_s, nullptr, nullptr, Is / 2, Is / 32, row0, k0, KW / 128, xs,
-                       f16_pitch(Is), k0, 2 * B, acc, acc);
-    for (int j = 0; j < 4; ++j) f.rf[warp][lane][j] = acc[0][j];
-    __syncthreads();
-    if (kh == 0) {
-        float v[4];
-        fs_sum(f, warp, 4, 2, 4, v);
-        const int t = q;
-        if (t < B) {
-            const float sc = exp2i(f.shift[t]);
-            a.ws.sh[(size_t)t * H + row0 + g] = (v[0] + v[1]) * sc;
-            a.ws.sh[(size_t)t * H + row0 + g + 8] = (v[2] + v[3]) * sc;
+// shared down: 16 rows x K/s_sd; sh_a staged as fp16 hi/lo columns (2b, 2b+1)
+DEVI void w_sd(const StepArgs &a, int item, const uint16_t *ss, const int *sshift) {
+    const int H = a.d.H, Is = a.d.Is, B = a.B, maxB = a.d.max_batch;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int tile = item / a.p.s_sd, ks = item % a.p.s_sd, row0 = tile * 16;
+    const int KW = Is / a.p.s_sd, k0 = ks * KW;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, dummy[4];
+    s_fp4<5, false>(a.w.sh_down_q, a.w.sh_down_s, nullptr, nullptr, Is / 2, Is / 32, row0, k0, KW / 128, ss,
+                    f16_pitch(Is), k0, g < 2 * B ? g : -1, acc, dummy);
+    float *part = a.ws.sd_part + (size_t)ks * maxB * H;
+    if (q < B) {
+        part[(size_t)q * H + row0 + g] = acc[0] + acc[1];
+        part[(size_t)q * H + row0 + g + 8] = acc[2] + acc[3];
+    }
+    const int tk = a.p.ctl_tk + (a.d.E + 7) / 8 + a.d.L / 16 + a.d.Is / 16 + tile;
+    if (!warp_ticket_last(a.ws.ctl + tk, a.p.s_sd)) return;
+    if (q < B) {
+        const float sc = exp2i(sshift[q]);
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = row0 + g + 8 * h2;
+            a.ws.sh[(size_t)q * H + r] = sum_splits(a.ws.sd_part + (size_t)q * H + r, (size_t)maxB * H, a.p.s_sd) * sc;
         }
     }
-    cta_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
+    warp_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
 }
 
-// ---- expert down: 128 rows of L for one active expert, full K; combine completed tokens ------------
+// ylat[b][row0 + i], i < 16, combined by one warp: lane (i, half) adds the weighted slots of its
+// parity in slot order, then the two halves are added
+DEVI void warp_combine_rows(const StepArgs &a, int b, int row0) {
+    const int L = a.d.L, K = a.d.k, lane = threadIdx.x & 31, l = row0 + (lane & 15), h = lane >> 4;
+    float s = 0.0f;
+    for (int r0 = h; r0 < K; r0 += 16) {
+        float wv[8], yv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int r = r0 + 2 * j;
+            wv[j] = r < K ? __ldcg(a.ws.wts + (size_t)b * K + r) : 0.0f;
+            yv[j] = r < K ? __ldcg(a.ws.y + ((size_t)b * K + r) * L + l) : 0.0f;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s += wv[j] * yv[j];
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 16);
+    if (lane < 16) a.ws.ylat[(size_t)b * L + l] = s;
+}
 
-DEVI bool fs_edown(const StepArgs &a, int item, uint16_t *xs, FsSmem &f) {
+// expert down: 16 rows of L of active expert slot j, full K; a staged per warp (fp16 hi/lo of
+// the expert's entries, 512 k at a time); the warp that completes a token's 16 rows combines them
+DEVI bool w_edown(const StepArgs &a, int item, uint16_t *ws) {
     const int L = a.d.L, I = a.d.I, K = a.d.k;
-    const int blocks = L / kFsExpRows, j = item / blocks, blk = item % blocks;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    if (!cta_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(I / kFsExpRows), &f.ok)) return false;
-    const int e = __ldcg(a.ws.active_e + j), cnt = __ldcg(a.ws.active_cnt + j), off = __ldcg(a.ws.active_off + j);
-    if (threadIdx.x < cnt) {
-        const int en = __ldcg(a.ws.entries + off + threadIdx.x);
-        f.ent[threadIdx.x] = en;
-        f.shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(a.ws.a_amax + en)));
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int tiles = L / 16, j = item / tiles, tile = item % tiles, row0 = tile * 16;
+    if (!warp_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(I / 16))) return false;
+    const Entries en = warp_entries(a, j);
+    __shared__ int s_ent[kWarps][kMaxTopK], s_shift[kWarps][kMaxTopK];  // cnt <= B <= 4
+    const int warp = threadIdx.x >> 5;
+    __syncwarp();
+    if (lane < en.cnt) {
+        s_ent[warp][lane] = en.my_ent;
+        s_shift[warp][lane] = prescale_shift(__uint_as_float(__ldcg(a.ws.a_amax + en.my_ent)));
     }
-    __syncthreads();
-    stage_f16_from_f32<true>(xs, f16_pitch(I), a.ws.a, I, cnt, [&](int t) { return f.ent[t]; }, f.shift, 0, I);
-    __syncthreads();
-    const int row0 = blk * kFsExpRows + warp * 16;
-    const size_t eq = (size_t)e * L * (I / 2), es = (size_t)e * L * (I / 32);
-    float acc[1][4] = {};
-    tile_fp4<1, false>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I / 2, I / 32, row0, 0, I / 128, xs,
-                       f16_pitch(I), 0, 2 * cnt, acc, acc);
-    if (q < cnt) {
-        const float sc = exp2i(f.shift[q]);
-        float *dst = a.ws.y + (size_t)f.ent[q] * L + row0;
-        dst[g] = (acc[0][0] + acc[0][1]) * sc;
-        dst[g + 8] = (acc[0][2] + acc[0][3]) * sc;
+    __syncwarp();
+    const size_t eq = (size_t)en.e * L * (I / 2), es = (size_t)en.e * L * (I / 32);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, dummy[4];
+    const int kc = kKChunk < I ? kKChunk : I;
+    for (int c0 = 0; c0 < I; c0 += kc) {
+        __syncwarp();
+        stage_f16_from_f32<true>(ws, f16_pitch(kc), a.ws.a, I, en.cnt, [&](int t) { return s_ent[warp][t]; },
+                                 s_shift[warp], c0, kc, lane, 32);
+        __syncwarp();
+        s_fp4<5, false>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I / 2, I / 32, row0, c0, kc / 128, ws,
+                        f16_pitch(kc), 0, g < 2 * en.cnt ? g : -1, acc, dummy);
     }
-    // count this block's rows for every token; the item that completes a token's K slots combines
+    if (q < en.cnt) {
+        const float sc = exp2i(s_shift[warp][q]);
+        float *dst = a.ws.y + (size_t)s_ent[warp][q] * L + row0;
+        dst[g] = (acc[0] + acc[1]) * sc;
+        dst[g + 8] = (acc[2] + acc[3]) * sc;
+    }
     __threadfence();
-    __syncthreads();
-    const int nb = L / kFsExpRows;
-    if (threadIdx.x < cnt) {
-        const int b = f.ent[threadIdx.x] / K;
-        f.flag[threadIdx.x] = (atomicAdd(a.ws.ctl + a.p.ctl_comb + b * nb + blk, 1u) == (unsigned)(K - 1)) ? 1 : 0;
+    __syncwarp();
+    bool mine = false;
+    if (lane < en.cnt)
+        mine = atomicAdd(a.ws.ctl + a.p.ctl_comb + (size_t)(en.my_ent / K) * (L / 16) + tile, 1u) == (unsigned)(K - 1);
+    unsigned todo = __ballot_sync(0xffffffffu, mine);
+    if (todo) __threadfence();  // acquire: the other slots' y rows of this block are visible
+    while (todo) {
+        const int tl = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int b = s_ent[warp][tl] / K;
+        warp_combine_rows(a, b, row0);
+        warp_signal_add(a.ws.ctl + a.p.ctl_ylat + tile, 1u);
     }
-    __syncthreads();
-    int done = 0;
-    for (int t = 0; t < cnt; ++t) {
-        if (!f.flag[t]) continue;
-        ++done;
-        __threadfence();  // acquire: every slot's y rows of this block are visible
-        const int b = f.ent[t] / K;
-        for (int r = threadIdx.x; r < kFsExpRows; r += blockDim.x)
-            a.ws.ylat[(size_t)b * L + blk * kFsExpRows + r] = combine_value(a, b, blk * kFsExpRows + r);
-    }
-    if (done) cta_signal_add(a.ws.ctl + a.p.ctl_ylat + blk, (unsigned)done);
     return true;
 }
 
-// ---- W_up: 64 rows x full K (2 halves); ylat staged once per CTA; out = bf16(W_up ylat + sh) ------
-
-DEVI void fs_up(const StepArgs &a, int item, const uint16_t *xs, FsSmem &f) {
-    const int H = a.d.H, L = a.d.L, B = a.B;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int tile = warp & 3, kh = warp >> 2;
-    const int row0 = item * kFsUpRows + tile * 16, KW = L / 2, k0 = kh * KW;
-    float acc[1][4] = {};
-    tile_bf16<1>(a.w.w_up, L, row0, k0, KW / 32, xs, bf16_pitch(L), k0, 2 * B, acc);
-    for (int j = 0; j < 4; ++j) f.rf[warp][lane][j] = acc[0][j];
-    __syncthreads();
-    if (kh == 0) {
-        float v[4];
-        fs_sum(f, warp, 4, 2, 4, v);
-        const int t = q;
-        if (t < B) {
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int r = row0 + g + 8 * h2;
-                const float s = v[2 * h2] + v[2 * h2 + 1];
-                if (a.ws.up_tap) a.ws.up_tap[(size_t)t * H + r] = s;
-                const float shv = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)t * H + r) : 0.0f;
-                a.out[(size_t)t * H + r] = f32_to_bf16_rne(s + shv);
-            }
-        }
+// W_up: 16 rows x K/s_up; ylat staged as bf16 hi/lo columns (2b, 2b+1); out = bf16(. + sh)
+DEVI void w_up(const StepArgs &a, int item, const uint16_t *ys) {
+    const int H = a.d.H, L = a.d.L, B = a.B, maxB = a.d.max_batch;
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int tile = item / a.p.s_up, ks = item % a.p.s_up, row0 = tile * 16;
+    const int KW = L / a.p.s_up, k0 = ks * KW;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    s_bf16<6>(a.w.w_up, L, row0, k0, KW / 32, ys, bf16_pitch(L), k0, g < 2 * B ? g : -1, acc);
+    float *part = a.ws.up_part + (size_t)ks * maxB * H;
+    if (q < B) {
+        part[(size_t)q * H + row0 + g] = acc[0] + acc[1];
+        part[(size_t)q * H + row0 + g + 8] = acc[2] + acc[3];
     }
-    __syncthreads();
+    const int tk = a.p.ctl_tk + (a.d.E + 7) / 8 + a.d.L / 16 + a.d.Is / 16 + a.d.H / 16 + tile;
+    if (!warp_ticket_last(a.ws.ctl + tk, a.p.s_up)) return;
+    if (q < B)
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = row0 + g + 8 * h2;
+            const float s = sum_splits(a.ws.up_part + (size_t)q * H + r, (size_t)maxB * H, a.p.s_up);
+            if (a.ws.up_tap) a.ws.up_tap[(size_t)q * H + r] = s;
+            const float shv = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)q * H + r) : 0.0f;
+            a.out[(size_t)q * H + r] = f32_to_bf16_rne(s + shv);
+        }
 }
 
-// ---- the kernel ---------------------------------------------------------------------------------------
+// ---------------------------------------------------------------------------------------------
+// the kernel
 
 __host__ __device__ inline size_t fused_small_smem(const StepArgs &a) {
-    size_t m = (size_t)8 * bf16_pitch(a.d.H) * 2;                    // x, bf16
+    const int B = a.B;
+    size_t m = (size_t)B * bf16_pitch(a.d.H) * 2;                        // x, bf16
     auto mx = [&](size_t v) { m = v > m ? v : m; };
-    mx((size_t)8 * f16_pitch(a.d.H) * 2);                              // x, fp16 (shared gate/up)
-    mx((size_t)8 * f16_pitch(a.d.L) * 2);                              // h (expert gate/up)
-    mx((size_t)8 * f16_pitch(a.d.I) * 2);                              // a (expert down)
-    mx((size_t)8 * f16_pitch(a.d.Is) * 2);                             // sh_a (shared down)
-    mx((size_t)8 * bf16_pitch(a.d.L) * 2);                             // ylat (W_up)
+    mx((size_t)B * f16_pitch(a.d.H) * 2);                                 // x, fp16
+    mx((size_t)2 * B * f16_pitch(a.d.L) * 2);                             // h, fp16 hi/lo
+    mx((size_t)2 * B * f16_pitch(a.d.Is) * 2);                            // sh_a, fp16 hi/lo
+    mx((size_t)kWarps * 2 * B * f16_pitch(kKChunk < a.d.I ? kKChunk : a.d.I) * 2);  // a, per warp
+    mx((size_t)2 * B * bf16_pitch(a.d.L) * 2);                            // ylat, bf16 hi/lo
     return m;
 }
 
-__global__ void __launch_bounds__(256, 1) k_fused_small(StepArgs a) {
+__global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ TopkSmem topk;
-    __shared__ FsSmem f;
+    __shared__ int s_shift[kMaxBatch], s_ok;
+    __shared__ unsigned s_amax[kMaxBatch];
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     unsigned *ctl = a.ws.ctl;
     const int H = a.d.H, L = a.d.L, I = a.d.I, Is = a.d.Is, B = a.B, E = a.d.E;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     bool alive = true;
     unsigned long long *trace = a.ws.trace ? a.ws.trace + (size_t)blockIdx.x * kTraceStamps : nullptr;
     auto stamp = [&](int i) {
         if (trace && threadIdx.x == 0) trace[i] = global_ns();
     };
     stamp(0);
-    const int n_rt = (E + kFsRouterRows - 1) / kFsRouterRows, n_dn = L / kFsDnRows;
-    const int n_sgu = a.d.n_shared ? Is / kFsSguRows : 0, n_sd = a.d.n_shared ? H / kFsSdRows : 0;
-    const int n_up = H / kFsUpRows;
+    const int n_rt = (E + 7) / 8 * a.p.s_rt, n_dn = L / 16 * a.p.s_dn;
+    const int n_sgu = a.d.n_shared ? Is / 16 * a.p.s_sgu : 0, n_sd = a.d.n_shared ? H / 16 * a.p.s_sd : 0;
+    const int n_up = H / 16 * a.p.s_up;
 
-    // one item ahead: claim the next index when the current item starts, prefetch its weights
-    auto queue = [&](int qi, int n, auto prefetch, auto body) {
-        if (threadIdx.x == 0) f.item = (int)atomicAdd(ctl + CTL_QHEAD + qi, 1u);
-        __syncthreads();
-        int it = f.item;
-        __syncthreads();
-        if (it < n) prefetch(it);
-        while (alive && it < n) {
-            if (threadIdx.x == 0) f.item = (int)atomicAdd(ctl + CTL_QHEAD + qi, 1u);
-            __syncthreads();
-            const int nxt = f.item;
-            __syncthreads();
-            if (nxt < n) prefetch(nxt);
-            alive = body(it);
-            it = nxt;
+    // warps take items of queue qi until it runs dry; the next index is claimed when an item starts
+    auto warp_queue = [&](int qi, int n, auto body) {
+        int it = 0;
+        if (lane == 0) it = (int)atomicAdd(ctl + CTL_QHEAD + qi, 1u);
+        it = __shfl_sync(0xffffffffu, it, 0);
+        int ok = 1;
+        while (ok && it < n) {
+            int nxt = 0;
+            if (lane == 0) nxt = (int)atomicAdd(ctl + CTL_QHEAD + qi, 1u);
+            ok = body(it) ? 1 : 0;
+            it = __shfl_sync(0xffffffffu, nxt, 0);
         }
+        return ok;
+    };
+    auto stage_x_bf16 = [&]() {
+        stage_bf16(xs, bf16_pitch(H), a.x, H, B, B, 0, H);
+        __syncthreads();
     };
 
-    // x as bf16, 8 columns (zeros beyond B), for the router and W_dn
-    stage_bf16(xs, bf16_pitch(H), a.x, H, B, 8, 0, H);
-    __syncthreads();
-    queue(Q_ROUTER_S, n_rt,
-          [&](int it) {
-              const int rows = min(kFsRouterRows, E - it * kFsRouterRows);
-              if (rows > 0) fs_prefetch(a.w.router + (size_t)it * kFsRouterRows * H, (size_t)rows * H * 2);
-          },
-          [&](int it) { fs_router(a, it, xs, f); return true; });
+    // router and W_dn read x as bf16
+    stage_x_bf16();
+    warp_queue(QS_ROUTER, n_rt, [&](int it) { w_router(a, it, xs); return true; });
     stamp(1);
-    queue(Q_TOPK_S, B, [](int) {}, [&](int it) { return item_topk<true>(a, it, topk); });
+    __syncthreads();
+    for (int it = blockIdx.x; alive && it < B; it += gridDim.x) alive = item_topk<true>(a, it, topk, (unsigned)((E + 7) / 8));
     stamp(2);
-    queue(Q_DN_S, n_dn, [&](int it) { fs_prefetch(a.w.w_dn + (size_t)it * kFsDnRows * H, (size_t)kFsDnRows * H * 2); },
-          [&](int it) { fs_dn(a, it, xs, f); return true; });
+    if (alive) warp_queue(QS_DN, n_dn, [&](int it) { w_dn(a, it, xs); return true; });
     stamp(3);
+    __syncthreads();
+    // shared gate/up read x as fp16 with a per-token exponent over all of H
     if (alive && n_sgu) {
-        // x as fp16 with a per-token exponent (over all of H), no hi/lo split: bf16 fits in fp16
-        __syncthreads();
-        if (threadIdx.x < 8) f.flag[threadIdx.x] = 0;
+        if (threadIdx.x < B) s_amax[threadIdx.x] = 0u;
         __syncthreads();
         for (int i = threadIdx.x; i < B * (H / 8); i += blockDim.x) {
             const int t = i / (H / 8), u = i % (H / 8);
             const uint4 v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * H + 8 * u);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
             float m = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w[j])), fabsf(bf16_hi(w[j]))));
-            atomicMax(reinterpret_cast<unsigned *>(&f.flag[t]), __float_as_uint(m));
+            for (int k = 0; k < 4; ++k) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w4[k])), fabsf(bf16_hi(w4[k]))));
+            atomicMax(s_amax + t, __float_as_uint(m));
         }
         __syncthreads();
-        if (threadIdx.x < 8) f.xshift[threadIdx.x] = prescale_shift(__uint_as_float((unsigned)f.flag[threadIdx.x]));
+        if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(s_amax[threadIdx.x]));
         __syncthreads();
-        stage_f16_from_bf16(xs, f16_pitch(H), a.x, H, B, f.xshift, 0, H);
-        for (int i = threadIdx.x; i < (8 - B) * (H / 8); i += blockDim.x) {  // unused columns
-            const int col = B + i / (H / 8), u = i % (H / 8);
-            *reinterpret_cast<uint4 *>(xs + (size_t)col * f16_pitch(H) + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
-        }
+        stage_f16_from_bf16(xs, f16_pitch(H), a.x, H, B, s_shift, 0, H);
         __syncthreads();
-        queue(Q_SGU_S, n_sgu,
-              [&](int it) {
-                  const size_t r0 = (size_t)it * kFsSguRows;
-                  fs_prefetch(a.w.sh_gate_q + r0 * (H / 2), (size_t)kFsSguRows * (H / 2));
-                  fs_prefetch(a.w.sh_up_q + r0 * (H / 2), (size_t)kFsSguRows * (H / 2));
-                  fs_prefetch(a.w.sh_gate_s + r0 * (H / 32), (size_t)kFsSguRows * (H / 32));
-                  fs_prefetch(a.w.sh_up_s + r0 * (H / 32), (size_t)kFsSguRows * (H / 32));
-              },
-              [&](int it) { fs_sgu(a, it, xs, f); return true; });
+        warp_queue(QS_SGU, n_sgu, [&](int it) { w_sgu(a, it, xs, s_shift); return true; });
     }
     stamp(4);
-    if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &f.ok);
-    if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)n_dn, &f.ok);
+    // expert gate/up: routing and all of h final; stage h of every token (fp16 hi/lo)
+    if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
+    if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)(L / 16), &s_ok);
     stamp(5);
     if (alive) {
-        const int blocks = I / kFsExpRows;
-        const int n = __ldcg(a.ws.n_active) * blocks;
-        queue(Q_EGU_S, n,
-              [&](int it) {
-                  const int e = __ldcg(a.ws.active_e + it / blocks);
-                  const size_t r0 = (size_t)e * I + (size_t)(it % blocks) * kFsExpRows;
-                  fs_prefetch(a.w.gate_q + r0 * (L / 2), (size_t)kFsExpRows * (L / 2));
-                  fs_prefetch(a.w.up_q + r0 * (L / 2), (size_t)kFsExpRows * (L / 2));
-                  fs_prefetch(a.w.gate_s + r0 * (L / 32), (size_t)kFsExpRows * (L / 32));
-                  fs_prefetch(a.w.up_s + r0 * (L / 32), (size_t)kFsExpRows * (L / 32));
-              },
-              [&](int it) { fs_egu(a, it, xs, f); return true; });
+        if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
+        __syncthreads();
+        stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, B, [](int t) { return t; }, s_shift, 0, L);
+        __syncthreads();
+        const int n = __ldcg(a.ws.n_active) * (I / 16) * a.p.s_egu;
+        warp_queue(QS_EGU, n, [&](int it) { w_egu(a, it, xs, s_shift); return true; });
     }
     stamp(6);
+    // shared down: all of sh_a final; stage it (fp16 hi/lo)
     if (alive && n_sd) {
-        alive = cta_wait_geq(a, ctl + CTL_SGU_DONE, (unsigned)n_sgu, &f.ok);
+        alive = cta_wait_geq(a, ctl + CTL_SGU_DONE, (unsigned)(Is / 16), &s_ok);
         if (alive) {
-            if (threadIdx.x < B) f.shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_shamax + threadIdx.x)));
+            if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_shamax + threadIdx.x)));
             __syncthreads();
-            stage_f16_from_f32<true>(xs, f16_pitch(Is), a.ws.sh_a, Is, B, [](int t) { return t; }, f.shift, 0, Is);
+            stage_f16_from_f32<true>(xs, f16_pitch(Is), a.ws.sh_a, Is, B, [](int t) { return t; }, s_shift, 0, Is);
             __syncthreads();
-            queue(Q_SD_S, n_sd,
-                  [&](int it) {
-                      const size_t r0 = (size_t)it * kFsSdRows;
-                      fs_prefetch(a.w.sh_down_q + r0 * (Is / 2), (size_t)kFsSdRows * (Is / 2));
-                      fs_prefetch(a.w.sh_down_s + r0 * (Is / 32), (size_t)kFsSdRows * (Is / 32));
-                  },
-                  [&](int it) { fs_sd(a, it, xs, f); return true; });
+            warp_queue(QS_SD, n_sd, [&](int it) { w_sd(a, it, xs, s_shift); return true; });
         }
     }
     stamp(7);
+    // expert down (per-warp staging of the expert's entries)
     if (alive) {
-        const int blocks = L / kFsExpRows;
-        const int n = __ldcg(a.ws.n_active) * blocks;
-        queue(Q_EDOWN_S, n,
-              [&](int it) {
-                  const int e = __ldcg(a.ws.active_e + it / blocks);
-                  const size_t r0 = (size_t)e * L + (size_t)(it % blocks) * kFsExpRows;
-                  fs_prefetch(a.w.down_q + r0 * (I / 2), (size_t)kFsExpRows * (I / 2));
-                  fs_prefetch(a.w.down_s + r0 * (I / 32), (size_t)kFsExpRows * (I / 32));
-              },
-              [&](int it) { return fs_edown(a, it, xs, f); });
+        __syncthreads();
+        const int n = __ldcg(a.ws.n_active) * (L / 16);
+        const int kc = kKChunk < I ? kKChunk : I;
+        uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(kc);
+        const int ok = warp_queue(QS_EDOWN, n, [&](int it) { return w_edown(a, it, ws); });
+        alive = __syncthreads_and(ok) != 0;
     }
     stamp(8);
+    // W_up: every ylat block final for every token, and all of sh; stage ylat (bf16 hi/lo)
     if (alive) {
-        // ylat (every token, every row) and sh must be final; each thread polls one ylat block
-        __syncthreads();
         int ok = 1;
-        for (int blk = threadIdx.x; blk < L / kFsExpRows; blk += blockDim.x)
+        for (int blk = threadIdx.x; blk < L / 16; blk += blockDim.x)
             ok &= wait_geq(a, ctl + a.p.ctl_ylat + blk, (unsigned)B) ? 1 : 0;
-        if (threadIdx.x == 0 && a.d.n_shared) ok &= wait_geq(a, ctl + CTL_SD_DONE, (unsigned)n_sd) ? 1 : 0;
+        if (threadIdx.x == 0 && a.d.n_shared) ok &= wait_geq(a, ctl + CTL_SD_DONE, (unsigned)(H / 16)) ? 1 : 0;
         __threadfence();
         alive = __syncthreads_and(ok) != 0;
         if (alive) {
             stage_bf16split_from_f32(xs, bf16_pitch(L), a.ws.ylat, L, B, 0, L);
-            for (int i = threadIdx.x; i < (8 - 2 * B) * (L / 8); i += blockDim.x) {  // unused columns
-                const int col = 2 * B + i / (L / 8), u = i % (L / 8);
-                *reinterpret_cast<uint4 *>(xs + (size_t)col * bf16_pitch(L) + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
-            }
             __syncthreads();
-            queue(Q_UP_S, n_up,
-                  [&](int it) { fs_prefetch(a.w.w_up + (size_t)it * kFsUpRows * L, (size_t)kFsUpRows * L * 2); },
-                  [&](int it) { fs_up(a, it, xs, f); return true; });
+            warp_queue(QS_UP, n_up, [&](int it) { w_up(a, it, xs); return true; });
         }
     }
     stamp(9);
@@ -497,34 +612,49 @@ __global__ void __launch_bounds__(256, 1) k_fused_small(StepArgs a) {
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        f.ok = (atomicAdd(ctl + CTL_EXIT, 1u) == gridDim.x - 1) ? 1 : 0;
+        s_ok = (atomicAdd(ctl + CTL_EXIT, 1u) == gridDim.x - 1) ? 1 : 0;
     }
     __syncthreads();
     stamp(10);
-    if (f.ok) {
+    if (s_ok) {
         __threadfence();
         for (int i = threadIdx.x; i < CTL_FIXED; i += blockDim.x) ctl[i] = 0u;
         for (int i = threadIdx.x; i < E; i += blockDim.x) ctl[a.p.ctl_gu + i] = 0u;
-        for (int i = threadIdx.x; i < B * (L / kFsExpRows); i += blockDim.x) ctl[a.p.ctl_comb + i] = 0u;
-        for (int i = threadIdx.x; i < L / kFsExpRows; i += blockDim.x) ctl[a.p.ctl_ylat + i] = 0u;
+        for (int i = threadIdx.x; i < B * (L / 16); i += blockDim.x) ctl[a.p.ctl_comb + i] = 0u;
+        for (int i = threadIdx.x; i < L / 16; i += blockDim.x) ctl[a.p.ctl_ylat + i] = 0u;
         for (int i = threadIdx.x; i < B; i += blockDim.x) {
             ctl[a.p.ctl_hamax + i] = 0u;
             ctl[a.p.ctl_shamax + i] = 0u;
         }
+        // tickets: all but the expert gate/up ones, then those of the active slots
+        const int n_fixed_tk = (E + 7) / 8 + L / 16 + Is / 16 + 2 * (H / 16);
+        const int n_egu_tk = __ldcg(a.ws.n_active) * (I / 16);
+        for (int i = threadIdx.x; i < n_fixed_tk + n_egu_tk; i += blockDim.x) ctl[a.p.ctl_tk + i] = 0u;
     }
 }
 
 bool fused_small_supports(const Dims &d, int B) {
-    // full-K items: H/8 and H/4 split evenly into bf16 (32) and MXFP4 (128) rounds, I_s/2 into
-    // MXFP4 rounds; at most 4 tokens so that hi/lo columns of every part fit one 8-column tile
-    return B <= 4 && d.H % 512 == 0 && d.L % 128 == 0 && d.I % 128 == 0 && (d.n_shared == 0 || d.Is % 256 == 0);
+    // K splits of whole bf16 (32) and MXFP4 (128) rounds; at most 4 tokens so that the hi/lo
+    // columns of every part fit one 8-column MMA tile
+    const int kc = kKChunk < d.I ? kKChunk : d.I;
+    const size_t x16 = (size_t)B * (d.H + 32) * 2, hl = (size_t)2 * B * (d.L + 32) * 2;
+    const size_t smem = std::max(std::max(x16, hl), std::max((size_t)2 * B * (d.Is + 16) * 2,
+                                                             (size_t)kWarps * 2 * B * (kc + 16) * 2));
+    return B <= kSmallMaxBatch && d.H % 128 == 0 && d.L % 128 == 0 && d.I % 128 == 0 && d.I % kc == 0 &&
+           (d.n_shared == 0 || d.Is % 128 == 0) && d.k <= kMaxTopK && smem <= kSmallSmemLimit;
 }
 
 cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm) {
+    int per_sm = 0;
+    const size_t sm = fused_small_smem(a);
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_fused_small, 256, sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(n_sm);
+    cfg.gridDim = dim3(n_sm * per_sm);
     cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = fused_small_smem(a);
+    cfg.dynamicSmemBytes = sm;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
@@ -535,7 +665,7 @@ cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm) {
 }
 
 cudaError_t init_fused_small_attributes() {
-    return cudaFuncSetAttribute(k_fused_small, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    return cudaFuncSetAttribute(k_fused_small, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmallSmemLimit);
 }
 
 }  // namespace moedec

@@ -16,6 +16,12 @@ constexpr int kExpertWarps = 4;    // expert kernels: 4 warps x 16 rows per item
 constexpr int kExpertRows = 64;
 constexpr int kKChunk = 512;       // activation staging chunk along K
 constexpr int kExpertTokGroup = 16;  // tokens of one expert per pass (two 8-column n-tiles)
+constexpr int kMaxCtasPerSm = 2;  // persistent kernels: CTAs per SM at most (trace rows per SM)
+// Largest K splits of the small-batch step's warp items (router, W_dn, shared gate/up, expert
+// gate/up, shared down, W_up); the plan takes the largest count <= these that divides K evenly.
+constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmallSplitEgu = 2, kSmallSplitSd = 4,
+              kSmallSplitUp = 8;
+constexpr int kSmallMaxBatch = 4;  // tokens of the small-batch step
 constexpr int kTraceStamps = 16;     // MOEDEC_TRACE_STAMPS
 
 struct Dims {
@@ -43,8 +49,9 @@ struct Plan {
     int ctl_ylat;   // [L/16]        tokens whose ylat rows of a 16-row block are final
     int ctl_hamax;  // [maxB]        max |h| per token (float bits)
     int ctl_shamax; // [maxB]        max |sh_a| per token (float bits), small-batch schedule
-    int ctl_tk;     // [E/8 + L/16 + I_s/16 + 2*H/16] per-tile tickets of the small-batch schedule
+    int ctl_tk;     // [E/8 + L/16 + I_s/16 + 2*H/16 + E*I/16] per-tile tickets of the small-batch schedule
     int ctl_tk_words;
+    int s_rt, s_dn, s_sgu, s_egu, s_sd, s_up;  // K splits of the small-batch schedule
     int ctl_words;
     long long wait_limit_ns;  // bound of every device-side wait of the fused step
 };
@@ -77,6 +84,7 @@ struct Work {
     int *active_cnt;    // [E]  tokens per active expert
     int *active_off;    // [E]  offset of the expert's entries
     int *entries;       // [maxB*k] entry = b*k + r, grouped by expert, token-ascending inside a group
+    float *egu_part;    // [s_egu][min(maxB,4)*k][2][I] expert gate then up partials (small-batch step)
     float *a;           // [maxB*k][I]  silu(gate) * up per entry
     unsigned *a_amax;   // [maxB*k]     max |a| per entry (float bits)
     float *y;           // [maxB*k][L]  expert output per entry

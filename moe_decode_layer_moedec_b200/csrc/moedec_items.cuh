@@ -154,10 +154,11 @@ struct TopkSmem {
     int off[kMaxExperts];
 };
 
+// FUSED: first wait until CTL_RT_DONE reaches rt_done (the schedule's count of router signals).
 template <bool FUSED>
-DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t) {
+DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u) {
     const int E = a.d.E, K = a.d.k, B = a.B;
-    if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, (unsigned)a.p.rt.blocks, &t.ok)) return false;
+    if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, rt_done, &t.ok)) return false;
     const int tid = threadIdx.x;
     // thread tid owns experts 4*tid .. 4*tid+3 (index order follows thread order)
     unsigned key[4];

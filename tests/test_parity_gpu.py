@@ -170,9 +170,11 @@ def test_fused_wait_timeout_is_reported_and_context_stays_usable(tiny):
     _check_step(w, W, synth.tokens(w, batch=2), layer)
 
 
-def test_fused_and_multi_agree(tiny):
+@pytest.mark.parametrize("batch", [3, 9])
+def test_fused_and_multi_agree(tiny, batch):
+    # batch 3 runs the small-batch fused kernel, batch 9 the split-K one
     w, W, W_dev = tiny
-    x = synth.tokens(w, step=5, batch=9)
+    x = synth.tokens(w, step=5, batch=batch)
     a = run_layer(_make_layer(w, W_dev, max_batch=16, schedule="fused"), x)
     b = run_layer(_make_layer(w, W_dev, max_batch=16, schedule="multi"), x)
     assert np.array_equal(a[1], b[1])
