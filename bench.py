@@ -44,7 +44,7 @@ def parse():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="full_b1", choices=sorted(synth.WORKLOADS))
     p.add_argument("--layers", type=int, default=0, help="distinct layers cycled through (default 32)")
-    p.add_argument("--schedule", choices=["fused", "multi"], default="fused",
+    p.add_argument("--schedule", choices=["fused", "multi", "stream"], default="fused",
                    help="one persistent kernel per step (default) or eight stream-ordered kernels")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
@@ -76,6 +76,7 @@ def kernel_bytes(d: synth.Dims, unique_experts: float, B: int) -> dict:
         "shared_down": fp4(H, Is),
         "fused_step_splitk": step_bytes(d, unique_experts, B),
         "fused_step_small": step_bytes(d, unique_experts, B),
+        "fused_step_stream": step_bytes(d, unique_experts, B),
     }
 
 
@@ -146,6 +147,8 @@ class ClockSampler:
 
 
 KERNEL_SOURCES = {
+    "fused_step_stream": ["moedec_stream.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
+                          "moedec_router.cuh", "moedec_internal.h"],
     "fused_step_small": ["moedec_fused_small.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
                          "moedec_router.cuh", "moedec_internal.h"],
 }
@@ -256,7 +259,8 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
-    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_SKIP_SCALE_CHECK, LayerDims, MoeDecodeLayer
+    from moe_decode_layer_moedec_b200 import (FLAG_MULTI_KERNEL, FLAG_SKIP_SCALE_CHECK, FLAG_STREAM, LayerDims,
+                                              MoeDecodeLayer)
 
     w = synth.WORKLOADS[args.workload]
     d = w.dims
@@ -277,6 +281,8 @@ def main():
         flags = 0 if l == 0 else FLAG_SKIP_SCALE_CHECK  # layer 0 runs the create-time scale scan
         if args.schedule == "multi":
             flags |= FLAG_MULTI_KERNEL
+        if args.schedule == "stream":
+            flags |= FLAG_STREAM
         layers.append(MoeDecodeLayer(dims, Wd, max_batch=B, flags=flags))
         dev_weights.append(Wd)
         if rank == 0 and (l % 8 == 7 or l == n_layers - 1):

@@ -70,6 +70,10 @@ typedef enum moedec_status {
                                           on the side stream) instead of one fused persistent kernel */
 #define MOEDEC_FLAG_TRACE 16u          /* fused step: every CTA stamps %globaltimer at its phase
                                           boundaries (read with moedec_get_trace) */
+#define MOEDEC_FLAG_STREAM 32u         /* batches of 1-2 tokens: run the step as four launches of the
+                                          streaming kernel (each warp streams its work items through
+                                          a shared-memory ring of cp.async stages) instead of the
+                                          small-batch persistent kernel */
 #define MOEDEC_TRACE_STAMPS 16         /* stamps per CTA */
 
 typedef struct moedec_config {
@@ -159,12 +163,14 @@ MOEDEC_API int moedec_get_taps(moedec_handle *h, float *logits, float *hlat, flo
 
 /*
  * Launch counters (host values): launches[i] counts the kernels of variant i issued by this
- * handle since creation; i = 0 the small-batch schedule (batch <= 4: full-K work items, no split-K
- * partials), 1 the split-K schedule (batch >= 5).  n_variants in/out.
+ * handle since creation; i = 0 the small-batch schedules (batch <= 4), 1 the split-K schedule
+ * (batch >= 5).  n_variants in/out.
  */
 MOEDEC_API int moedec_get_launch_counts(moedec_handle *h, uint64_t *launches, int *n_variants);
 
-/* Kernels issued per step by the current build (so a timed loop can count its launches). */
+/* Kernels issued per step of `batch` tokens by this handle (so a timed loop can count its launches):
+ * 4 for the streaming schedule (MOEDEC_FLAG_STREAM, batch <= 2), 1 for the other fused schedules, 8 with
+ * MOEDEC_FLAG_MULTI_KERNEL (7 without a shared expert). */
 MOEDEC_API int moedec_kernels_per_step(moedec_handle *h, int batch);
 
 /* Last CUDA error string recorded by the handle ("" if none); static storage of the handle. */
@@ -210,12 +216,18 @@ MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, const uint16
                                             int batch, float *logits, void *stream);
 
 /*
- * Phase timeline of the last fused step (MOEDEC_FLAG_TRACE): host array out[n_cta][MOEDEC_TRACE_STAMPS]
- * of %globaltimer nanoseconds, stamp i taken by CTA c when it finished phase i (0 start, 1 router,
- * 2 top-k, 3 W_dn, 4 shared gate/up, 5 routing wait, 6 expert gate/up, 7 shared down, 8 expert down,
- * 9 W_up, 10 exit; 0 where a phase was skipped).  *n_cta in/out: capacity in rows (at least 2 per SM)
- * in, rows written out (2 per SM; rows of CTAs that the last step did not launch stay 0).
- * Synchronises `stream`.  INVALID_ARG without MOEDEC_FLAG_TRACE.
+ * Phase timeline of the last fused step (MOEDEC_FLAG_TRACE): host array out[rows][MOEDEC_TRACE_STAMPS]
+ * of %globaltimer nanoseconds, 0 where nothing was stamped; rows = 16 per SM.  *n_cta in/out:
+ * capacity in rows in, rows written out.  Synchronises `stream`.  INVALID_ARG without
+ * MOEDEC_FLAG_TRACE.
+ *   split-K and small-batch kernels, row = CTA: 0 start, 1 router, 2 top-k, 3 W_dn, 4 shared
+ *     gate/up, 5 routing wait, 6 expert gate/up, 7 shared down, 8 expert down, 9 W_up, 10 exit.
+ *   streaming kernel (batch <= 2), row = 16 * CTA + warp: 0 start, 1 fp16 copy of x done,
+ *     2..6 SM clock cycles spent issuing copies and claiming work, waiting for a stage's data,
+ *     waiting for activation blocks, in MMAs, in item epilogues; 7 stages consumed; 9 last stage
+ *     done, 10 exit, 11 expert buckets published (the ranking warp), 12 routing tables loaded
+ *     (the loading warp), 14 last router group done and 15 top-k done (the ranking warp);
+ *     row 16 * CTA + 12: start and end of the CTA in each of the step's 4 launches (stamps 0..7).
  */
 MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream);
 

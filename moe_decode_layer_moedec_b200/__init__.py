@@ -22,6 +22,7 @@ FLAG_SKIP_SCALE_CHECK = 2
 FLAG_TEST_STALL = 4
 FLAG_MULTI_KERNEL = 8
 FLAG_TRACE = 16
+FLAG_STREAM = 32
 TRACE_STAMPS = 16
 STATUS = {0: "MOEDEC_OK", -1: "MOEDEC_ERR_INVALID_ARG", -2: "MOEDEC_ERR_UNSUPPORTED", -3: "MOEDEC_ERR_CUDA",
           -4: "MOEDEC_ERR_OOM", -5: "MOEDEC_ERR_TIMEOUT", -6: "MOEDEC_ERR_DEVICE"}
@@ -197,7 +198,7 @@ class MoeDecodeLayer:
 
     def trace(self, stream=None):
         """Per-CTA phase timestamps (ns) of the last fused step: list of rows (FLAG_TRACE only)."""
-        cap = 1024
+        cap = 16 * 256  # 16 rows per SM
         buf = (ctypes.c_uint64 * (cap * TRACE_STAMPS))()
         n = ctypes.c_int(cap)
         self._check("moedec_get_trace", lib.moedec_get_trace(self._h, buf, ctypes.byref(n), _stream_ptr(stream)))

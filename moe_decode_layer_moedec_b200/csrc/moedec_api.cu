@@ -11,6 +11,8 @@
 
 using namespace moedec;
 
+extern "C" MOEDEC_API int moedec_kernels_per_step(moedec_handle *h, int batch);
+
 struct moedec_handle {
     moedec_config cfg;
     Dims d;
@@ -106,9 +108,29 @@ void layout(moedec_handle *h, char *base) {
     w.sh = c.take<float>(B * d.H);
     w.up_part = c.take<float>((size_t)std::max(p.up.splits, kSmallSplitUp) * B * d.H);
     w.up_tap = (h->cfg.flags & MOEDEC_FLAG_TAPS) ? c.take<float>(B * d.H) : nullptr;
+    {  // streaming small-batch step: at most 2 tokens
+        const StreamPlan &sp = p.st;
+        const size_t Is = d.n_shared ? d.Is : 128, nent = (size_t)2 * d.k;
+        w.st_rt_part = c.take<double>((size_t)sp.s_rt * 2 * d.E);
+        w.st_key = c.take<unsigned>((size_t)2 * d.E);
+        w.st_dn_part = c.take<float>((size_t)sp.s_dn * 2 * d.L);
+        w.st_sgu_part = c.take<float>((size_t)sp.s_sgu * 2 * 2 * Is);
+        w.st_egu_part = c.take<float>((size_t)sp.s_egu * nent * 2 * d.I);
+        w.st_sd_part = c.take<float>((size_t)sp.s_sd * 2 * d.H);
+        w.st_up_part = c.take<float>((size_t)sp.s_up * 2 * d.H);
+        w.x16 = c.take<uint16_t>((size_t)2 * d.H);
+        w.x16e = c.take<int>((size_t)sp.s_sgu * 4);
+        w.h16 = c.take<uint16_t>((size_t)4 * d.L);
+        w.h16e = c.take<int>((size_t)sp.s_egu * 4);
+        w.sh16 = c.take<uint16_t>((size_t)4 * Is);
+        w.sh16e = c.take<int>((size_t)sp.s_sd * 4);
+        w.a16 = c.take<uint16_t>(nent * 2 * d.I);
+        w.a16e = c.take<int>((size_t)d.E * 4);
+        w.ylat16 = c.take<uint16_t>((size_t)4 * d.L);
+    }
     w.tickets = c.take<unsigned>((size_t)p.n_tickets);
     w.ctl = c.take<unsigned>((size_t)p.ctl_words);
-    w.trace = (h->cfg.flags & MOEDEC_FLAG_TRACE) ? c.take<unsigned long long>((size_t)h->n_sm * kMaxCtasPerSm * kTraceStamps) : nullptr;
+    w.trace = (h->cfg.flags & MOEDEC_FLAG_TRACE) ? c.take<unsigned long long>((size_t)h->n_sm * kTraceRowsPerSm * kTraceStamps) : nullptr;
     w.err = c.take<unsigned>(1);
     h->buf_bytes = c.off;
 }
@@ -139,11 +161,11 @@ int check_scales(moedec_handle *h) {
 
 enum KernelKind {
     K_ROUTER_DN, K_TOPK, K_EXPERT_GU, K_EXPERT_DOWN, K_COMBINE, K_UP, K_SHARED_GU, K_SHARED_DOWN, K_FUSED,
-    K_FUSED_SMALL, K_COUNT
+    K_FUSED_SMALL, K_FUSED_STREAM, K_COUNT
 };
 const char *const kKernelNames[K_COUNT] = {"router_dn", "topk",        "expert_gate_up", "expert_down",
                                            "combine",   "up",          "shared_gate_up", "shared_down",
-                                           "fused_step_splitk", "fused_step_small"};
+                                           "fused_step_splitk", "fused_step_small", "fused_step_stream"};
 
 cudaEvent_t pool_get(moedec_handle *h) {
     if (!h->pool.empty()) {
@@ -257,7 +279,8 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     p.s_egu = small_split(d.L, 128, kSmallSplitEgu);
     p.s_sd = small_split(d.Is, 128, kSmallSplitSd);
     p.s_up = small_split(d.L, 32, kSmallSplitUp);
-    p.ctl_words = p.ctl_tk + p.ctl_tk_words;
+    stream_plan(d, p.st, p.ctl_tk + p.ctl_tk_words);
+    p.ctl_words = p.st.words;
     p.wait_limit_ns = (c.flags & MOEDEC_FLAG_TEST_STALL) ? 20000000LL : 1000000000LL;
 
     int rc = MOEDEC_OK;
@@ -266,6 +289,7 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     if (e == cudaSuccess) e = init_kernel_attributes();
     if (e == cudaSuccess) e = init_fused_attributes();
     if (e == cudaSuccess) e = init_fused_small_attributes();
+    if (e == cudaSuccess) e = init_stream_attributes();
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming);
@@ -326,12 +350,14 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     cudaError_t e = cudaSuccess;
     const int variant = batch <= 4 ? 0 : 1;
     if (!(h->cfg.flags & MOEDEC_FLAG_MULTI_KERNEL)) {
-        if (fused_small_supports(h->d, batch))
+        if ((h->cfg.flags & MOEDEC_FLAG_STREAM) && stream_supports(h->d, batch))
+            e = timed(h, K_FUSED_STREAM, s, [&] { return launch_stream(a, s, h->n_sm); });
+        else if (fused_small_supports(h->d, batch))
             e = timed(h, K_FUSED_SMALL, s, [&] { return launch_fused_small(a, s, h->n_sm); });
         else
             e = timed(h, K_FUSED, s, [&] { return launch_fused(a, s, h->n_sm); });
         if (e != cudaSuccess) return record_cuda(h, e);
-        h->launches[variant] += 1;
+        h->launches[variant] += (uint64_t)moedec_kernels_per_step(h, batch);
         h->last_batch = batch;
         return MOEDEC_OK;
     }
@@ -442,7 +468,7 @@ MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t 
 }
 
 MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream) {
-    const int rows = h ? h->n_sm * kMaxCtasPerSm : 0;
+    const int rows = h ? h->n_sm * kTraceRowsPerSm : 0;
     if (!h || !out || !n_cta || !h->ws.trace || *n_cta < rows) return MOEDEC_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync(out, h->ws.trace, (size_t)rows * kTraceStamps * sizeof(uint64_t),
@@ -455,7 +481,8 @@ MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, voi
 
 MOEDEC_API int moedec_kernels_per_step(moedec_handle *h, int batch) {
     if (!h || batch <= 0) return 0;
-    return (h->cfg.flags & MOEDEC_FLAG_MULTI_KERNEL) ? kernels_per_step(h->d) : 1;
+    if (h->cfg.flags & MOEDEC_FLAG_MULTI_KERNEL) return kernels_per_step(h->d);
+    return ((h->cfg.flags & MOEDEC_FLAG_STREAM) && stream_supports(h->d, batch)) ? kStreamLaunches : 1;
 }
 
 }  // extern "C"

@@ -494,6 +494,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     __shared__ TopkSmem topk;
     __shared__ int s_shift[kMaxBatch], s_ok;
     __shared__ unsigned s_amax[kMaxBatch];
+    __shared__ CtaTake claim;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     unsigned *ctl = a.ws.ctl;
     const int H = a.d.H, L = a.d.L, I = a.d.I, Is = a.d.Is, B = a.B, E = a.d.E;
@@ -508,17 +509,18 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     const int n_sgu = a.d.n_shared ? Is / 16 * a.p.s_sgu : 0, n_sd = a.d.n_shared ? H / 16 * a.p.s_sd : 0;
     const int n_up = H / 16 * a.p.s_up;
 
-    // warps take items of queue qi until it runs dry; the next index is claimed when an item starts
+    // warps take items of queue qi until this CTA's range of it runs dry
     auto warp_queue = [&](int qi, int n, auto body) {
-        int it = 0;
-        if (lane == 0) it = (int)atomicAdd(ctl + CTL_QHEAD + qi, 1u);
-        it = __shfl_sync(0xffffffffu, it, 0);
         int ok = 1;
-        while (ok && it < n) {
-            int nxt = 0;
-            if (lane == 0) nxt = (int)atomicAdd(ctl + CTL_QHEAD + qi, 1u);
-            ok = body(it) ? 1 : 0;
-            it = __shfl_sync(0xffffffffu, nxt, 0);
+        for (;;) {
+            int it = -1;
+            if (lane == 0) it = cta_take(claim, qi, n);
+            it = __shfl_sync(0xffffffffu, it, 0);
+            if (it < 0) break;
+            if (!body(it)) {
+                ok = 0;
+                break;
+            }
         }
         return ok;
     };
@@ -527,6 +529,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         __syncthreads();
     };
 
+    cta_take_init(claim);
     // router and W_dn read x as bf16
     stage_x_bf16();
     warp_queue(QS_ROUTER, n_rt, [&](int it) { w_router(a, it, xs); return true; });

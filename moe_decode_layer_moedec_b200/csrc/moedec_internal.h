@@ -16,7 +16,8 @@ constexpr int kExpertWarps = 4;    // expert kernels: 4 warps x 16 rows per item
 constexpr int kExpertRows = 64;
 constexpr int kKChunk = 512;       // activation staging chunk along K
 constexpr int kExpertTokGroup = 16;  // tokens of one expert per pass (two 8-column n-tiles)
-constexpr int kMaxCtasPerSm = 2;  // persistent kernels: CTAs per SM at most (trace rows per SM)
+constexpr int kMaxCtasPerSm = 2;  // persistent kernels: CTAs per SM at most
+constexpr int kTraceRowsPerSm = 16;  // trace rows per SM (one per CTA, or one per warp)
 // Largest K splits of the small-batch step's warp items (router, W_dn, shared gate/up, expert
 // gate/up, shared down, W_up); the plan takes the largest count <= these that divides K evenly.
 constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmallSplitEgu = 2, kSmallSplitSd = 4,
@@ -39,8 +40,32 @@ struct SplitPlan {
     int blocks, splits, krange;
 };
 
+// Streaming small-batch step (moedec_stream.cu): K range of one work item per matrix (a multiple of
+// 128 dividing K; the splits are K / range), and its control words (offsets into ctl[]).
+struct StreamPlan {
+    int kr_rt, kr_dn, kr_sgu, kr_egu, kr_sd, kr_up;
+    int s_rt, s_dn, s_sgu, s_egu, s_sd, s_up;
+    int c_rt_tk;   // [ceil(E/16)]   router 16-row groups: K splits done
+    int c_dn_tk;   // [L/16]         W_dn tiles: K splits done
+    int c_dnb;     // [s_egu]        W_dn tiles done per h block (block = the expert gate/up K range)
+    int c_h16;     // [s_egu]        1 once the block's fp16 copy of h is written
+    int c_x16;     // [s_sgu]        tokens whose fp16 copy of x is written, per block
+    int c_sgu_tk;  // [I_s/64]       shared gate/up tiles: K splits done
+    int c_sgb;     // [s_sd]         shared gate/up tiles done per sh_a block
+    int c_sh16;    // [s_sd]         1 once the block's fp16 copy of sh_a is written
+    int c_egu_tk;  // [E*(I/64)]     expert gate/up tiles (per active slot): K splits done
+    int c_gu;      // [E]            expert gate/up tiles done per active slot
+    int c_a16;     // [E]            1 once the slot's fp16 copy of a is written
+    int c_sd_tk;   // [H/64]         shared down tiles: K splits done
+    int c_comb;    // [2*(L/64)]     expert down tiles done per (token, 64-row latent tile)
+    int c_yl;      // [s_up]         (token, 64-row tile) pairs of ylat written per block
+    int c_up_tk;   // [H/16]         W_up tiles: K splits done
+    int words;     // end of the region
+};
+
 struct Plan {
     SplitPlan rt, dn, up, sgu, sd;
+    StreamPlan st;
     int ticket_rt, ticket_dn, ticket_up, ticket_sgu, ticket_sd, ticket_topk;  // offsets into tickets[]
     int n_tickets;
     // control words of the fused step (zero at rest), offsets into ctl[]
@@ -95,9 +120,26 @@ struct Work {
     float *sh;          // [maxB][H]
     float *up_part;     // [up.splits][maxB][H]
     float *up_tap;      // [maxB][H] or nullptr
+    // streaming small-batch step (at most 2 tokens): partials and MMA-ready activation copies
+    double *st_rt_part;   // [s_rt][2][E]
+    unsigned *st_key;     // [2][E]       top-k key per (token, expert): fp32 score bits + 1
+    float *st_dn_part;    // [s_dn][2][L]
+    float *st_sgu_part;   // [s_sgu][2][2][I_s]
+    float *st_egu_part;   // [s_egu][2k][2][I]
+    float *st_sd_part;    // [s_sd][2][H]
+    float *st_up_part;    // [s_up][2][H]
+    uint16_t *x16;        // [2][H]       fp16 x * 2^-e, e per (block, token)
+    int *x16e;            // [s_sgu][4]
+    uint16_t *h16;        // [4][L]       fp16 hi/lo of h * 2^-e (row 2t + part)
+    int *h16e;            // [s_egu][4]
+    uint16_t *sh16;       // [4][I_s]
+    int *sh16e;           // [s_sd][4]
+    uint16_t *a16;        // [2k][2][I]   fp16 hi/lo of a * 2^-e per entry
+    int *a16e;            // [E][4]       exponents of the slot's entries, in entry order
+    uint16_t *ylat16;     // [4][L]       bf16 hi/lo of ylat (row 2t + part)
     unsigned *tickets;  // [n_tickets]
     unsigned *ctl;      // [ctl_words] fused-step control block (zero at rest)
-    unsigned long long *trace;  // [n_sm][kTraceStamps] phase timestamps or nullptr
+    unsigned long long *trace;  // [n_sm * 16][kTraceStamps] phase timestamps or nullptr
     unsigned *err;      // [1] sticky device error word
 };
 
@@ -128,6 +170,11 @@ cudaError_t launch_shared_down(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_scale_check(const uint8_t *s, size_t n, unsigned *bad, cudaStream_t st);
 cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm);
 cudaError_t init_fused_attributes();
+constexpr int kStreamLaunches = 4;  // launches of the streaming small-batch step
+bool stream_supports(const Dims &d, int B);
+void stream_plan(const Dims &d, StreamPlan &sp, int ctl_base);
+cudaError_t launch_stream(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t init_stream_attributes();
 bool fused_small_supports(const Dims &d, int B);
 cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm);
 cudaError_t init_fused_small_attributes();

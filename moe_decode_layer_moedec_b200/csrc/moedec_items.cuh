@@ -89,6 +89,30 @@ DEVI void warp_signal_add(unsigned *counter, unsigned v) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Work claiming.  Items of a queue are uniform, and every queue's length is known when a CTA
+// reaches it, so CTA c owns the contiguous range [n*c/G, n*(c+1)/G) of each queue and its warps
+// take items from it with a shared-memory counter: no global atomic (a queue head is one L2
+// address that thousands of warps would otherwise serialise on) and no lock.
+
+struct CtaTake {
+    int next[8];
+};
+
+// by every thread of the CTA before the first take (a __syncthreads must follow)
+DEVI void cta_take_init(CtaTake &t) {
+    for (int i = threadIdx.x; i < 8; i += blockDim.x) t.next[i] = 0;
+}
+
+// next item of queue q (n items) of this CTA's range for the calling thread (one lane per
+// warp), or -1 once the range is used up
+DEVI int cta_take(CtaTake &t, int q, int n) {
+    const long long G = gridDim.x, c = blockIdx.x;
+    const int lo = (int)((long long)n * c / G), hi = (int)((long long)n * (c + 1) / G);
+    const int k = atomicAdd(t.next + q, 1);
+    return lo + k < hi ? lo + k : -1;
+}
+
+// ---------------------------------------------------------------------------------------------
 // router: one router row block x K range (fp64 MMAs); the block's last CTA publishes logits
 
 template <bool FUSED>

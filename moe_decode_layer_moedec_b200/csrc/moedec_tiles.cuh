@@ -23,15 +23,15 @@ __host__ __device__ constexpr int up_chunk(int nt, int krange) {
 
 // Sum of n (<= 16) split-K partials p[0], p[stride], ... in split order.  All loads are issued
 // before the first add (one L2 round trip instead of n); L1-bypassing, since other CTAs wrote them.
-template <class T>
+template <class T, int W = 8>
 DEVI T sum_splits(const T *p, size_t stride, int n) {
     T s = T(0);
-    for (int k0 = 0; k0 < n; k0 += 8) {  // eight loads in flight, then eight adds in split order
-        T v[8];
+    for (int k0 = 0; k0 < n; k0 += W) {  // W loads in flight, then W adds in split order
+        T v[W];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = k0 + k < n ? __ldcg(p + (size_t)(k0 + k) * stride) : T(0);
+        for (int k = 0; k < W; ++k) v[k] = k0 + k < n ? __ldcg(p + (size_t)(k0 + k) * stride) : T(0);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < W; ++k)
             if (k0 + k < n) s += v[k];
     }
     return s;

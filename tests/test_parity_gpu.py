@@ -24,14 +24,16 @@ def torch_cuda():
     return torch
 
 
-SCHEDULES = ["fused", "multi"]
+SCHEDULES = ["fused", "multi", "stream"]
 
 
 def _make_layer(w, W_dev, max_batch, flags=None, schedule="fused"):
-    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_TAPS, MoeDecodeLayer
+    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_STREAM, FLAG_TAPS, MoeDecodeLayer
     f = FLAG_TAPS if flags is None else flags
     if schedule == "multi":
         f |= FLAG_MULTI_KERNEL
+    if schedule == "stream":
+        f |= FLAG_STREAM
     return MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=max_batch, flags=f)
 
 
@@ -152,12 +154,13 @@ def test_batch_zero_and_limits(tiny, torch_cuda):
         layer.routing(3)  # not the last step's batch
 
 
-def test_fused_wait_timeout_is_reported_and_context_stays_usable(tiny):
+@pytest.mark.parametrize("schedule", ["fused", "stream"])
+def test_fused_wait_timeout_is_reported_and_context_stays_usable(tiny, schedule):
     # MOEDEC_FLAG_TEST_STALL: the router never publishes its logits, so the top-k item's bounded
     # wait runs out (20 ms); every CTA leaves and the step reports MOEDEC_ERR_TIMEOUT.
     from moe_decode_layer_moedec_b200 import FLAG_TEST_STALL, MoedecError
     w, W, W_dev = tiny
-    stalled = _make_layer(w, W_dev, max_batch=2, flags=FLAG_TEST_STALL)
+    stalled = _make_layer(w, W_dev, max_batch=2, flags=FLAG_TEST_STALL, schedule=schedule)
     x = to_device(synth.tokens(w, batch=2))
     stalled.step(x)
     with pytest.raises(MoedecError, match="TIMEOUT"):
@@ -166,16 +169,16 @@ def test_fused_wait_timeout_is_reported_and_context_stays_usable(tiny):
     with pytest.raises(MoedecError, match="TIMEOUT"):
         stalled.routing(2)
     stalled.close()
-    layer = _make_layer(w, W_dev, max_batch=2)
+    layer = _make_layer(w, W_dev, max_batch=2, schedule=schedule)
     _check_step(w, W, synth.tokens(w, batch=2), layer)
 
 
-@pytest.mark.parametrize("batch", [3, 9])
-def test_fused_and_multi_agree(tiny, batch):
-    # batch 3 runs the small-batch fused kernel, batch 9 the split-K one
+@pytest.mark.parametrize("batch,schedule", [(2, "stream"), (3, "fused"), (9, "fused")])
+def test_fused_and_multi_agree(tiny, batch, schedule):
+    # batch 2 runs the streaming kernel, batch 3 the small-batch fused kernel, batch 9 the split-K one
     w, W, W_dev = tiny
     x = synth.tokens(w, step=5, batch=batch)
-    a = run_layer(_make_layer(w, W_dev, max_batch=16, schedule="fused"), x)
+    a = run_layer(_make_layer(w, W_dev, max_batch=16, schedule=schedule), x)
     b = run_layer(_make_layer(w, W_dev, max_batch=16, schedule="multi"), x)
     assert np.array_equal(a[1], b[1])
     for k in ("h", "ylat", "sh", "up"):
