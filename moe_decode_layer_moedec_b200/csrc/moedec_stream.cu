@@ -154,34 +154,6 @@ DEVI int item_stages(const StepArgs &a, const Geo &g, int q) {
 // ---------------------------------------------------------------------------------------------
 // stage issue: weights (always) and the activation columns (when their block is final)
 
-// 16 bf16 rows x 128 k; row r's 16-byte unit u is stored at unit u ^ 4*(r & 1)
-DEVI void issue_bf16_rows(uint32_t slot, const uint16_t *W, size_t ld, int row0, int nrows, int k0) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int p = lane + 32 * i, r = p >> 4, u = p & 15;
-        const bool ok = row0 + r < nrows;
-        const uint16_t *src = W + (size_t)(ok ? row0 + r : 0) * ld + k0 + 8 * u;
-        cp16_zfill(slot + r * 256 + 16 * (u ^ ((r & 1) << 2)), src, ok);
-    }
-}
-
-// 64 MXFP4 rows x 128 k: codes (64 B per row) and the row's four E8M0 scale bytes
-DEVI void issue_fp4_rows(uint32_t slot, const uint8_t *Q, const uint8_t *S, size_t ldq, size_t lds, size_t row0,
-                         int k0) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int p = lane + 32 * i, r = p >> 2, u = p & 3;
-        cp16(slot + r * 64 + 16 * u, Q + (row0 + r) * ldq + k0 / 2 + 16 * u);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const int r = lane + 32 * i;
-        cp4(slot + kSlotSc + 4 * r, S + (row0 + r) * lds + k0 / 32);
-    }
-}
-
 // Activation part of a stage: column c of the slot is 128 k of global row src(c) starting at k0.
 // ASYNC: cp.async into the stage's copy group; else synchronous L2 loads and shared stores.
 template <bool ASYNC, class Src>
@@ -317,42 +289,143 @@ DEVI void copy_act(const StepArgs &a, const Geo &g, const StSmem &sm, unsigned c
     }
 }
 
-// weights of stage c of item t of queue q
-DEVI void issue_weights(const StepArgs &a, const Geo &g, const StSmem &sm, uint32_t slot, int q, const Item &t,
-                        int c) {
+// Per-lane copy plan of the item being issued, computed once per item: every stage's copies are
+// then the plan's pointers plus a per-stage offset (a few instructions per 16-byte copy).
+struct IssuePlan {
+    const unsigned char *w;       // lane's weight piece 0, stage 0, matrix 0
+    const unsigned char *s;       // MXFP4: lane's scale row, stage 0, matrix 0; bf16: a valid address
+    long long dw, ds;             // MXFP4 pairs: byte offset of the up matrix from the gate matrix
+    int wpi, spi;                 // bytes between the lane's weight pieces / its two scale rows
+    unsigned valid;               // bf16: bit i set when piece i's row exists
+    uint32_t dst;                 // lane's piece-0 offset in a slot
+    const unsigned char *a0, *a1; // lane's activation pieces at stage 0 (null: none)
+    uint32_t adst0, adst1;
+    const int *ex;                // lane's exponent source (null: none)
+    bool fp4, pair;
+};
+
+// activation column c of item t (its source row at the item's first k), for c < ncols
+DEVI const uint16_t *act_col(const StepArgs &a, const Geo &g, const StSmem &sm, int q, const Item &t, int c) {
     const StreamPlan &p = a.p.st;
     switch (q) {
-        case SQ_RT:
-            issue_bf16_rows(slot, a.w.router, g.H, 16 * t.a, g.E, t.ks * p.kr_rt + 128 * c);
-            break;
-        case SQ_DN:
-            issue_bf16_rows(slot, a.w.w_dn, g.H, 16 * t.a, g.L, t.ks * p.kr_dn + 128 * c);
-            break;
-        case SQ_UP:
-            issue_bf16_rows(slot, a.w.w_up, g.L, 16 * t.a, g.H, t.ks * p.kr_up + 128 * c);
-            break;
-        case SQ_SGU: {
-            const bool up = c & 1;
-            issue_fp4_rows(slot, up ? a.w.sh_up_q : a.w.sh_gate_q, up ? a.w.sh_up_s : a.w.sh_gate_s, g.H / 2, g.H / 32,
-                           (size_t)64 * t.a, t.ks * p.kr_sgu + 128 * (c >> 1));
-            break;
+        case SQ_RT: return a.x + (size_t)c * g.H + t.ks * p.kr_rt;
+        case SQ_DN: return a.x + (size_t)c * g.H + t.ks * p.kr_dn;
+        case SQ_UP: return a.ws.ylat16 + (size_t)c * g.L + t.ks * p.kr_up;
+        case SQ_SGU: return a.ws.x16 + (size_t)c * g.H + t.ks * p.kr_sgu;
+        case SQ_EGU:
+            return a.ws.h16 + (size_t)(2 * (sm.ent[sm.act_off[t.a] + (c >> 1)] / g.K) + (c & 1)) * g.L + t.ks * p.kr_egu;
+        case SQ_SD: return a.ws.sh16 + (size_t)c * g.Is + t.ks * p.kr_sd;
+        default: return a.ws.a16 + (size_t)(2 * sm.ent[sm.act_off[t.a] + (c >> 1)] + (c & 1)) * g.I;  // SQ_EDOWN
+    }
+}
+
+DEVI IssuePlan make_plan(const StepArgs &a, const Geo &g, const StSmem &sm, int q, const Item &t) {
+    const StreamPlan &p = a.p.st;
+    const int lane = threadIdx.x & 31;
+    IssuePlan P;
+    P.dw = P.ds = 0;
+    P.ex = nullptr;
+    P.fp4 = !(q == SQ_RT || q == SQ_DN || q == SQ_UP);
+    P.pair = (q == SQ_SGU || q == SQ_EGU);
+    if (!P.fp4) {
+        const uint16_t *W = q == SQ_RT ? a.w.router : q == SQ_DN ? a.w.w_dn : a.w.w_up;
+        const int ld = q == SQ_UP ? g.L : g.H;
+        const int nrows = q == SQ_RT ? g.E : q == SQ_DN ? g.L : g.H;
+        const int k0 = t.ks * (q == SQ_RT ? p.kr_rt : q == SQ_DN ? p.kr_dn : p.kr_up);
+        const int r0 = lane >> 4, u = lane & 15, row = 16 * t.a + r0;
+        P.w = reinterpret_cast<const unsigned char *>(W + (size_t)(row < nrows ? row : 0) * ld + k0 + 8 * u);
+        P.s = reinterpret_cast<const unsigned char *>(W);
+        P.wpi = 2 * ld * 2;
+        P.spi = 0;
+        P.valid = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) P.valid |= (row + 2 * i < nrows ? 1u : 0u) << i;
+        P.dst = r0 * 256 + 16 * (u ^ ((r0 & 1) << 2));
+    } else {
+        const uint8_t *Q, *S;
+        size_t ldq, lds, row0;
+        int k0;
+        if (q == SQ_SGU) {
+            Q = a.w.sh_gate_q; S = a.w.sh_gate_s; ldq = g.H / 2; lds = g.H / 32; row0 = (size_t)64 * t.a;
+            k0 = t.ks * p.kr_sgu;
+            P.dw = a.w.sh_up_q - a.w.sh_gate_q;
+            P.ds = a.w.sh_up_s - a.w.sh_gate_s;
+        } else if (q == SQ_EGU) {
+            Q = a.w.gate_q; S = a.w.gate_s; ldq = g.L / 2; lds = g.L / 32;
+            row0 = (size_t)sm.act_e[t.a] * g.I + 64 * t.b;
+            k0 = t.ks * p.kr_egu;
+            P.dw = a.w.up_q - a.w.gate_q;
+            P.ds = a.w.up_s - a.w.gate_s;
+        } else if (q == SQ_SD) {
+            Q = a.w.sh_down_q; S = a.w.sh_down_s; ldq = g.Is / 2; lds = g.Is / 32; row0 = (size_t)64 * t.a;
+            k0 = t.ks * p.kr_sd;
+        } else {  // SQ_EDOWN
+            Q = a.w.down_q; S = a.w.down_s; ldq = g.I / 2; lds = g.I / 32;
+            row0 = (size_t)sm.act_e[t.a] * g.L + 64 * t.b;
+            k0 = 0;
         }
-        case SQ_EGU: {
-            const bool up = c & 1;
-            const size_t row0 = (size_t)sm.act_e[t.a] * g.I + 64 * t.b;
-            issue_fp4_rows(slot, up ? a.w.up_q : a.w.gate_q, up ? a.w.up_s : a.w.gate_s, g.L / 2, g.L / 32, row0,
-                           t.ks * p.kr_egu + 128 * (c >> 1));
-            break;
+        P.w = Q + (row0 + (lane >> 2)) * ldq + k0 / 2 + 16 * (lane & 3);
+        P.s = S + (row0 + lane) * lds + k0 / 32;
+        P.wpi = (int)(8 * ldq);
+        P.spi = (int)(32 * lds);
+        P.valid = 0xffu;
+        P.dst = (lane >> 2) * 64 + 16 * (lane & 3);
+    }
+    // activation pieces of this lane (lane + 32j for j < 2) and its exponent
+    int ncols, pitch = kPitchF16;
+    bool swz = true;
+    switch (q) {
+        case SQ_RT: case SQ_DN: ncols = g.B; pitch = kPitchB16; swz = false; break;
+        case SQ_UP: ncols = 2 * g.B; pitch = kPitchB16; swz = false; break;
+        case SQ_SGU: ncols = g.B; break;
+        case SQ_SD: ncols = 2 * g.B; break;
+        default: ncols = 2 * sm.act_cnt[t.a]; break;  // SQ_EGU, SQ_EDOWN
+    }
+    if (q == SQ_SGU && lane < g.B) P.ex = a.ws.x16e + t.ks * 4 + lane;
+    if (q == SQ_SD && lane < g.B) P.ex = a.ws.sh16e + t.ks * 4 + lane;
+    if (q == SQ_EGU && lane < sm.act_cnt[t.a]) P.ex = a.ws.h16e + t.ks * 4 + sm.ent[sm.act_off[t.a] + lane] / g.K;
+    if (q == SQ_EDOWN && lane < sm.act_cnt[t.a]) P.ex = a.ws.a16e + t.a * 4 + lane;
+    P.a0 = P.a1 = nullptr;
+    P.adst0 = P.adst1 = 0;
+    {
+        const int c = lane >> 4, u = lane & 15;
+        if (c < ncols) {
+            P.a0 = reinterpret_cast<const unsigned char *>(act_col(a, g, sm, q, t, c) + 8 * u);
+            P.adst0 = kSlotAct + c * pitch + 16 * (swz ? swz2(u) : u);
         }
-        case SQ_SD:
-            issue_fp4_rows(slot, a.w.sh_down_q, a.w.sh_down_s, g.Is / 2, g.Is / 32, (size_t)64 * t.a,
-                           t.ks * p.kr_sd + 128 * c);
-            break;
-        case SQ_EDOWN: {
-            const size_t row0 = (size_t)sm.act_e[t.a] * g.L + 64 * t.b;
-            issue_fp4_rows(slot, a.w.down_q, a.w.down_s, g.I / 2, g.I / 32, row0, 128 * c);
-            break;
+        if (c + 2 < ncols) {
+            P.a1 = reinterpret_cast<const unsigned char *>(act_col(a, g, sm, q, t, c + 2) + 8 * u);
+            P.adst1 = kSlotAct + (c + 2) * pitch + 16 * (swz ? swz2(u) : u);
         }
+    }
+    return P;
+}
+
+// stage c of the planned item: weights always, the activation part when `act`
+DEVI void issue_planned(const IssuePlan &P, uint32_t slot, int c, bool act) {
+    const int lane = threadIdx.x & 31;
+    const int kk = P.pair ? (c >> 1) : c;
+    const bool up = P.pair && (c & 1);
+    if (P.fp4) {
+        const unsigned char *b = P.w + (up ? P.dw : 0) + 64 * kk;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cp16(slot + P.dst + 512 * i, b + i * P.wpi);
+        const unsigned char *sb = P.s + (up ? P.ds : 0) + 4 * kk;
+        cp4(slot + kSlotSc + 4 * lane, sb);
+        cp4(slot + kSlotSc + 4 * (lane + 32), sb + P.spi);
+    } else {
+        const unsigned char *b = P.w + 256 * kk;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool ok = (P.valid >> i) & 1u;
+            cp16_zfill(slot + P.dst + 512 * i, ok ? b + i * P.wpi : P.s, ok);
+        }
+    }
+    if (act) {
+        const int ka = 256 * kk;
+        if (P.a0) cp16(slot + P.adst0, P.a0 + ka);
+        if (P.a1) cp16(slot + P.adst1, P.a1 + ka);
+        if (P.ex) cp4(slot + kSlotExp + 4 * lane, P.ex);
     }
 }
 
@@ -998,8 +1071,9 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
     __syncthreads();
 
     // producer state (warp-uniform)
-    int pq = q_lo, pit = -1, pc = 0, pn = 0;
+    int pq = q_lo, pit = -1, pc = 0, pn = 0, pdep = kDepNone;
     Item pitem = {0, 0, 0};
+    IssuePlan pplan;
     int n_iss = 0, n_con = 0;
     bool alive = true;
     int n_active = -1;  // known once the CTA's routing copy is loaded
@@ -1036,6 +1110,8 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
                 pitem = decode_item(a, g, pq, it);
                 pc = 0;
                 pn = item_stages(a, g, pq);
+                pplan = make_plan(a, g, sm, pq, pitem);
+                pdep = item_dep(pq, pitem);
                 return true;
             }
             ++pq;
@@ -1051,10 +1127,8 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
             }
             const int s = n_iss % kStStages;
             unsigned char *slot = ring + (size_t)s * kSlotBytes;
-            const int dep = item_dep(pq, pitem);
-            const bool act = dep_known(sm, dep);
-            issue_weights(a, g, sm, smem_addr(slot), pq, pitem, pc);
-            if (act) copy_act<true>(a, g, sm, slot, pq, pitem, pc);
+            const bool act = dep_known(sm, pdep);
+            issue_planned(pplan, smem_addr(slot), pc, act);
             cp_commit();
             if (lane == 0) {
                 sm.meta[warp][s].q = pq;
@@ -1078,6 +1152,7 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
 
     Acc acc;
     acc_zero(acc);
+    Item cit = {0, 0, 0};  // the item being consumed
     long long cyc_issue = 0, cyc_data = 0, cyc_dep = 0, cyc_compute = 0, cyc_epi = 0;
     for (;;) {
         const long long ti0 = trace ? clock64() : 0;
@@ -1092,7 +1167,8 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
         const long long td0 = trace ? clock64() : 0;
         cyc_data += td0 - ti1;
         const SlotMeta m = sm.meta[warp][s];
-        const Item it = decode_item(a, g, m.q, m.item);
+        if (m.c == 0) cit = decode_item(a, g, m.q, m.item);
+        const Item it = cit;
         if (!m.act) {
             // the activation block was not final when the weights were issued: wait for it, then
             // copy the activation part of every issued stage that waits on the same block (those
