@@ -227,7 +227,11 @@ MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, const uint16
  *     waiting for activation blocks, in MMAs, in item epilogues; 7 stages consumed; 9 last stage
  *     done, 10 exit, 11 expert buckets published (the ranking warp), 12 routing tables loaded
  *     (the loading warp), 14 last router group done and 15 top-k done (the ranking warp);
- *     row 16 * CTA + 12: start and end of the CTA in each of the step's 4 launches (stamps 0..7).
+ *     row 16 * CTA + 12: start and end of the CTA in each of the step's 4 launches (stamps 0..7);
+ *     row 16 * CTA + 13: per launch, cycles summed over the CTA's warps in issue, data waits,
+ *     MMAs and epilogues (stamps 4 * launch + 0..3); row 16 * CTA + 14: per launch, ns from the
+ *     launch's start to its activations staged, and the latest and earliest warp finish after that
+ *     (stamps 4 * launch + 0..2).
  */
 MOEDEC_API int moedec_get_trace(moedec_handle *h, uint64_t *out, int *n_cta, void *stream);
 

@@ -110,7 +110,7 @@ void layout(moedec_handle *h, char *base) {
     w.up_tap = (h->cfg.flags & MOEDEC_FLAG_TAPS) ? c.take<float>(B * d.H) : nullptr;
     {  // streaming small-batch step: at most 2 tokens
         const StreamPlan &sp = p.st;
-        const size_t Is = d.n_shared ? d.Is : 128, nent = (size_t)2 * d.k;
+        const size_t Is = d.n_shared ? d.Is : 512, nent = (size_t)2 * d.k;
         w.st_rt_part = c.take<double>((size_t)sp.s_rt * 2 * d.E);
         w.st_key = c.take<unsigned>((size_t)2 * d.E);
         w.st_dn_part = c.take<float>((size_t)sp.s_dn * 2 * d.L);
@@ -118,15 +118,6 @@ void layout(moedec_handle *h, char *base) {
         w.st_egu_part = c.take<float>((size_t)sp.s_egu * nent * 2 * d.I);
         w.st_sd_part = c.take<float>((size_t)sp.s_sd * 2 * d.H);
         w.st_up_part = c.take<float>((size_t)sp.s_up * 2 * d.H);
-        w.x16 = c.take<uint16_t>((size_t)2 * d.H);
-        w.x16e = c.take<int>((size_t)sp.s_sgu * 4);
-        w.h16 = c.take<uint16_t>((size_t)4 * d.L);
-        w.h16e = c.take<int>((size_t)sp.s_egu * 4);
-        w.sh16 = c.take<uint16_t>((size_t)4 * Is);
-        w.sh16e = c.take<int>((size_t)sp.s_sd * 4);
-        w.a16 = c.take<uint16_t>(nent * 2 * d.I);
-        w.a16e = c.take<int>((size_t)d.E * 4);
-        w.ylat16 = c.take<uint16_t>((size_t)4 * d.L);
     }
     w.tickets = c.take<unsigned>((size_t)p.n_tickets);
     w.ctl = c.take<unsigned>((size_t)p.ctl_words);

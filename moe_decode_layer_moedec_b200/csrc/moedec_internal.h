@@ -40,25 +40,18 @@ struct SplitPlan {
     int blocks, splits, krange;
 };
 
-// Streaming small-batch step (moedec_stream.cu): K range of one work item per matrix (a multiple of
-// 128 dividing K; the splits are K / range), and its control words (offsets into ctl[]).
+// Streaming small-batch step (moedec_stream.cu): K range of one work item per matrix (a multiple
+// of the stage width dividing K; the splits are K / range), and its control words (offsets into
+// ctl[]).
 struct StreamPlan {
     int kr_rt, kr_dn, kr_sgu, kr_egu, kr_sd, kr_up;
     int s_rt, s_dn, s_sgu, s_egu, s_sd, s_up;
-    int c_rt_tk;   // [ceil(E/16)]   router 16-row groups: K splits done
+    int c_rt_tk;   // [E/16]         router 16-row groups: K splits done
     int c_dn_tk;   // [L/16]         W_dn tiles: K splits done
-    int c_dnb;     // [s_egu]        W_dn tiles done per h block (block = the expert gate/up K range)
-    int c_h16;     // [s_egu]        1 once the block's fp16 copy of h is written
-    int c_x16;     // [s_sgu]        tokens whose fp16 copy of x is written, per block
-    int c_sgu_tk;  // [I_s/64]       shared gate/up tiles: K splits done
-    int c_sgb;     // [s_sd]         shared gate/up tiles done per sh_a block
-    int c_sh16;    // [s_sd]         1 once the block's fp16 copy of sh_a is written
-    int c_egu_tk;  // [E*(I/64)]     expert gate/up tiles (per active slot): K splits done
-    int c_gu;      // [E]            expert gate/up tiles done per active slot
-    int c_a16;     // [E]            1 once the slot's fp16 copy of a is written
-    int c_sd_tk;   // [H/64]         shared down tiles: K splits done
-    int c_comb;    // [2*(L/64)]     expert down tiles done per (token, 64-row latent tile)
-    int c_yl;      // [s_up]         (token, 64-row tile) pairs of ylat written per block
+    int c_sgu_tk;  // [I_s/16]       shared gate/up tiles: K splits done
+    int c_egu_tk;  // [E*(I/16)]     expert gate/up tiles (per active slot): K splits done
+    int c_sd_tk;   // [H/16]         shared down tiles: K splits done
+    int c_comb;    // [2*(L/16)]     expert down tiles done per (token, 16-row latent tile)
     int c_up_tk;   // [H/16]         W_up tiles: K splits done
     int words;     // end of the region
 };
@@ -120,7 +113,7 @@ struct Work {
     float *sh;          // [maxB][H]
     float *up_part;     // [up.splits][maxB][H]
     float *up_tap;      // [maxB][H] or nullptr
-    // streaming small-batch step (at most 2 tokens): partials and MMA-ready activation copies
+    // streaming small-batch step (at most 2 tokens): split-K partials and top-k keys
     double *st_rt_part;   // [s_rt][2][E]
     unsigned *st_key;     // [2][E]       top-k key per (token, expert): fp32 score bits + 1
     float *st_dn_part;    // [s_dn][2][L]
@@ -128,15 +121,6 @@ struct Work {
     float *st_egu_part;   // [s_egu][2k][2][I]
     float *st_sd_part;    // [s_sd][2][H]
     float *st_up_part;    // [s_up][2][H]
-    uint16_t *x16;        // [2][H]       fp16 x * 2^-e, e per (block, token)
-    int *x16e;            // [s_sgu][4]
-    uint16_t *h16;        // [4][L]       fp16 hi/lo of h * 2^-e (row 2t + part)
-    int *h16e;            // [s_egu][4]
-    uint16_t *sh16;       // [4][I_s]
-    int *sh16e;           // [s_sd][4]
-    uint16_t *a16;        // [2k][2][I]   fp16 hi/lo of a * 2^-e per entry
-    int *a16e;            // [E][4]       exponents of the slot's entries, in entry order
-    uint16_t *ylat16;     // [4][L]       bf16 hi/lo of ylat (row 2t + part)
     unsigned *tickets;  // [n_tickets]
     unsigned *ctl;      // [ctl_words] fused-step control block (zero at rest)
     unsigned long long *trace;  // [n_sm * 16][kTraceStamps] phase timestamps or nullptr

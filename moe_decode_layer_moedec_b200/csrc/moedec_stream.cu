@@ -1,34 +1,27 @@
-// moedec_stream.cu -- the decode layer step for 1-2 tokens as one persistent kernel of streaming
-// warps.
+// moedec_stream.cu -- the decode layer step for 1-2 tokens as four launches of a kernel of
+// streaming warps.
 //
 // Batch 1-2 is the pages' small-matrix range of the Kimi K3 decode path ("快是可以生成的，可信
 // 只能证明（vLLM 重写 Kimi K3 解码路径…）", section 他们换掉了什么), and there the step is pure
 // weight streaming: 148 MB per full-size layer step at batch 1.  A loaded HBM access on B200 takes
-// about 2 us, so each SM must keep ~100 KB of weights in flight at all times, across work items
-// and across the step's dependency points (routing, h, a, ylat).  The same page lists the
-// techniques as ways of removing waiting; this kernel is built around exactly that.
+// about 2 us, so each SM must keep ~100 KB of weights in flight at all times.
 //
-// Each warp owns a ring of 3 shared-memory slots and streams its own sequence of work items
-// through it with cp.async: a slot holds one stage of one item, 4 KB of weights (16 bf16 rows or
-// 64 MXFP4 rows, 128 k each) plus the matching 128 k of activation columns.  The warp issues the
-// next stages (of the next items, claimed one ahead) before it computes the current one, so its
-// loads never drain between items.  Weights never depend on anything but routing; when a stage's
-// activation block is not final yet, its weights are loaded anyway and the activation part is
-// copied when the stage is consumed.
+// Each warp owns a ring of 3 shared-memory slots and streams its work items through it with bulk
+// copies (cp.async.bulk, the tensor memory accelerator's 1-D form): a slot holds one stage of one
+// item, 16 weight rows of 256 bytes (128 bf16 or 512 MXFP4 elements) plus, for MXFP4, the rows'
+// 16 E8M0 scale bytes, and completes on its own mbarrier.  One lane per row issues the copy, so a
+// stage costs the warp a handful of instructions; the warp issues the next stages (of its next
+// items) before it computes the current one, so its copies never drain between items.
 //
-// Work queues, in order (every warp drains them in this order; an item only waits on items of
-// earlier queues, so every wait ends):
-//   x16     fp16 copy of x per 512-k block and token (for the shared gate/up MMAs)
-//   router  16 rows x K range, fp64 MMAs; the warp that completes the last row group ranks the
-//           experts (top-k per token) and builds the expert buckets
-//   W_dn    16 rows x K range; a completed block of h is converted to fp16 hi/lo once
-//   shared  gate/up, 64 rows x K range; a completed block of sh_a is converted once
-//   expert  gate/up, 64 rows of one active expert x K range; a completed expert's a is converted
-//   shared  down, 64 rows x K range
-//   expert  down, 64 rows of one active expert; completing a token's 64 latent rows combines them
-//   W_up    16 rows x K range (K-range major, so it starts on the first final block of ylat)
-// Activations crossing CTAs live in global memory in MMA-ready form: fp16 hi/lo columns scaled by
-// a power of two per (token, block) for the MXFP4 products, bf16 hi/lo columns for W_up.
+// The step is four launches; each runs only work whose inputs earlier launches finished, so no
+// warp ever waits on another's results:
+//   1  router (16 rows x K range, fp64 MMAs; the warp that completes the last row group ranks the
+//      experts and builds the expert buckets), W_dn, shared gate/up        (x)
+//   2  shared down, expert gate/up of the active experts                  (sh_a, h)
+//   3  expert down; completing a token's 16 latent rows combines them      (a)
+//   4  W_up and the output                                                 (ylat, sh)
+// A launch stages the activation it reads in every CTA once, as MMA operands (bf16, or fp16 hi/lo
+// columns scaled by a power of two per token or expert entry), while its first copies fly.
 #include <algorithm>
 
 #include "moedec_items.cuh"
@@ -40,410 +33,221 @@ namespace {
 constexpr int kStWarps = 12;
 constexpr int kStStages = 3;
 constexpr int kStMaxBatch = 2;
-// slot layout: weights | scales | activation columns | exponents
-constexpr int kSlotSc = 4096, kSlotAct = 4352, kSlotExp = 5632, kSlotBytes = 5648;
-constexpr int kPitchF16 = 272;  // fp16 activation column (128 k, 16-unit swizzle) in a slot
-constexpr int kPitchB16 = 320;  // bf16 activation column in a slot
-constexpr int kStDynSmem = kStWarps * kStStages * kSlotBytes;
-constexpr int kMaxActive = 64;  // active experts at <= 2 tokens x <= 32 slots
+constexpr int kSlotSc = 4096, kSlotBytes = 4352;  // 16 rows x 256 B, then 16 rows x 16 scale bytes
+constexpr int kRingBytes = kStWarps * kStStages * kSlotBytes;
+constexpr int kMaxActive = 64;       // active experts at <= 2 tokens x <= 32 slots
+constexpr int kMaxEdownExperts = 2;  // experts of one CTA's expert-down range (see stream_supports)
 
-enum StQueue { SQ_X16 = 0, SQ_RT, SQ_DN, SQ_SGU, SQ_EGU, SQ_SD, SQ_EDOWN, SQ_UP, SQ_N };
-
-// dependency ids of a stage's activation block (bit index in the CTA's ready bitmap)
-constexpr int kDepNone = -1, kDepX16 = 0, kDepH16 = 64, kDepSh16 = 80, kDepYl = 96, kDepA16 = 128;
-constexpr int kDepBits = 192;
+enum StQueue { SQ_RT = 0, SQ_DN, SQ_SGU, SQ_SD, SQ_EGU, SQ_EDOWN, SQ_UP, SQ_N };
 
 struct SlotMeta {
     int q, item, c, n;  // queue, item, stage within the item, stages of the item
-    int act;            // 1 once the activation part of the slot is copied
 };
 
 struct StSmem {
+    unsigned long long bar[kStWarps][kStStages];  // one mbarrier per slot
     SlotMeta meta[kStWarps][kStStages];
-    unsigned dep_ready[kDepBits / 32];
-    int route_state;  // 0 not loaded, 1 loading, 2 loaded
+    int route_state;  // 0 not loaded, 1 loading, 2 loaded, 3 aborted
     int n_active;
     int act_e[kMaxActive], act_cnt[kMaxActive], act_off[kMaxActive], ent[kMaxActive];
-    // top-k scratch of the warp that ranks the experts
     int tk_idx[kMaxActive], srt_e[kMaxActive], srt_i[kMaxActive], first_pos[kMaxActive + 1];
+    int shift[2 * kMaxEdownExperts * kStMaxBatch];  // staging exponents of the launch's columns
+    unsigned amax[2 * kMaxEdownExperts * kStMaxBatch];
+    int ed_j0;  // expert-down launch: first active slot staged by this CTA
     int exit_last;
     CtaTake claim;
 };
 
 // ---------------------------------------------------------------------------------------------
-// async copies
+// bulk copies and their barriers
 
 DEVI uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-DEVI void cp16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+DEVI void mbar_init(unsigned long long *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }
-DEVI void cp16_zfill(uint32_t dst, const void *src, bool valid) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+// one arrival that also announces `bytes` of copies completing on the barrier
+DEVI void mbar_arrive_expect_tx(unsigned long long *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
                  : "memory");
 }
-DEVI void cp4(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+DEVI bool mbar_test(unsigned long long *bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
 }
-DEVI void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// wait until at most n of this thread's copy groups are pending
-DEVI void cp_wait(int n) {
-    if (n <= 0)
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-    else if (n == 1)
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-    else
-        asm volatile("cp.async.wait_group 2;" ::: "memory");
+// global -> shared bulk copy (16-byte aligned, size a multiple of 16) completing on `bar`
+DEVI void bulk_copy(uint32_t dst, const void *src, unsigned bytes, unsigned long long *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
 }
 
-// unit u (16 bytes) of an fp16 activation column: within each 16-unit column, units of lane
-// quads 2 and 3 are shifted by two, so that a phase's four lane quads hit distinct bank groups
-DEVI int swz2(int u) { return u ^ (((u >> 3) & 1) << 1); }
+// Bounded wait for phase `parity` of a slot's barrier (all lanes).  The copies always complete;
+// the limit only bounds a broken run.
+DEVI bool slot_wait(const StepArgs &a, unsigned long long *bar, unsigned parity) {
+    if (mbar_test(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (;;) {
+        if (mbar_test(bar, parity)) return true;
+        if ((long long)(global_ns() - t0) > a.p.wait_limit_ns) {
+            if ((threadIdx.x & 31) == 0) {
+                atomicOr(a.ws.err, kErrTimeout);
+                atomicExch(a.ws.ctl + CTL_ABORT, 1u);
+            }
+            return false;
+        }
+    }
+}
 
 // ---------------------------------------------------------------------------------------------
 // the step's geometry
 
 struct Geo {
     int H, L, E, K, I, Is, B, ns;  // ns: 1 with a shared expert
-    int rt_groups, dn_tiles, sgu_tiles, egu_tiles, sd_tiles, ed_tiles, up_tiles;
 };
 
 DEVI Geo geo(const StepArgs &a) {
     Geo g;
     g.H = a.d.H; g.L = a.d.L; g.E = a.d.E; g.K = a.d.k; g.I = a.d.I; g.Is = a.d.Is; g.B = a.B;
     g.ns = a.d.n_shared ? 1 : 0;
-    g.rt_groups = (g.E + 15) / 16;
-    g.dn_tiles = g.L / 16;
-    g.sgu_tiles = g.Is / 64;
-    g.egu_tiles = g.I / 64;
-    g.sd_tiles = g.H / 64;
-    g.ed_tiles = g.L / 64;
-    g.up_tiles = g.H / 16;
     return g;
 }
 
 DEVI int queue_len(const StepArgs &a, const Geo &g, int q, int n_active) {
     const StreamPlan &p = a.p.st;
     switch (q) {
-        case SQ_X16: return g.ns ? g.B * p.s_sgu : 0;
-        case SQ_RT: return g.rt_groups * p.s_rt;
-        case SQ_DN: return g.dn_tiles * p.s_dn;
-        case SQ_SGU: return g.ns ? g.sgu_tiles * p.s_sgu : 0;
-        case SQ_EGU: return n_active * g.egu_tiles * p.s_egu;
-        case SQ_SD: return g.ns ? g.sd_tiles * p.s_sd : 0;
-        case SQ_EDOWN: return n_active * g.ed_tiles;
-        case SQ_UP: return g.up_tiles * p.s_up;
+        case SQ_RT: return g.E / 16 * p.s_rt;
+        case SQ_DN: return g.L / 16 * p.s_dn;
+        case SQ_SGU: return g.ns ? g.Is / 16 * p.s_sgu : 0;
+        case SQ_EGU: return n_active * (g.I / 16) * p.s_egu;
+        case SQ_SD: return g.ns ? g.H / 16 * p.s_sd : 0;
+        case SQ_EDOWN: return n_active * (g.L / 16);
+        case SQ_UP: return g.H / 16 * p.s_up;
     }
     return 0;
-}
-
-DEVI int item_stages(const StepArgs &a, const Geo &g, int q) {
-    const StreamPlan &p = a.p.st;
-    switch (q) {
-        case SQ_RT: return p.kr_rt / 128;
-        case SQ_DN: return p.kr_dn / 128;
-        case SQ_SGU: return 2 * (p.kr_sgu / 128);
-        case SQ_EGU: return 2 * (p.kr_egu / 128);
-        case SQ_SD: return p.kr_sd / 128;
-        case SQ_EDOWN: return g.I / 128;
-        case SQ_UP: return p.kr_up / 128;
-    }
-    return 0;
-}
-
-// ---------------------------------------------------------------------------------------------
-// stage issue: weights (always) and the activation columns (when their block is final)
-
-// Activation part of a stage: column c of the slot is 128 k of global row src(c) starting at k0.
-// ASYNC: cp.async into the stage's copy group; else synchronous L2 loads and shared stores.
-template <bool ASYNC, class Src>
-DEVI void copy_act_cols(unsigned char *slot, int ncols, int pitch, bool swizzle, Src src) {
-    const int lane = threadIdx.x & 31;
-    for (int p = lane; p < ncols * 16; p += 32) {
-        const int c = p >> 4, u = p & 15;
-        unsigned char *dst = slot + kSlotAct + c * pitch + 16 * (swizzle ? swz2(u) : u);
-        const uint16_t *s = src(c) + 8 * u;
-        if (ASYNC)
-            cp16(smem_addr(dst), s);
-        else
-            *reinterpret_cast<uint4 *>(dst) = __ldcg(reinterpret_cast<const uint4 *>(s));
-    }
-}
-
-template <bool ASYNC>
-DEVI void copy_exp(unsigned char *slot, int idx, const int *src) {
-    if (ASYNC)
-        cp4(smem_addr(slot + kSlotExp + 4 * idx), src);
-    else
-        *reinterpret_cast<int *>(slot + kSlotExp + 4 * idx) = __ldcg(src);
 }
 
 struct Item {
-    int a, b, ks;  // kind-specific: (group|tile|slot j, tile, k split)
+    int a, b, ks;  // row tile (or active slot j and tile b), K split
 };
 
-DEVI Item decode_item(const StepArgs &a, const Geo &g, int q, int it) {
+// item it of queue q; stages: bf16 128 k each, MXFP4 512 k each (gate and up alternate in pairs)
+DEVI Item decode_item(const StepArgs &a, const Geo &g, int q, int it, int *n_stages) {
     const StreamPlan &p = a.p.st;
     Item r = {0, 0, 0};
     switch (q) {
-        case SQ_X16: r.a = it / p.s_sgu; r.ks = it % p.s_sgu; break;                 // token, block
-        case SQ_RT: r.a = it / p.s_rt; r.ks = it % p.s_rt; break;                    // group
-        case SQ_DN: r.a = it / p.s_dn; r.ks = it % p.s_dn; break;                    // tile
-        case SQ_SGU: r.a = it / p.s_sgu; r.ks = it % p.s_sgu; break;                 // tile
+        case SQ_RT: r.a = it / p.s_rt; r.ks = it % p.s_rt; *n_stages = p.kr_rt / 128; break;
+        case SQ_DN: r.a = it / p.s_dn; r.ks = it % p.s_dn; *n_stages = p.kr_dn / 128; break;
+        case SQ_SGU: r.a = it / p.s_sgu; r.ks = it % p.s_sgu; *n_stages = 2 * (p.kr_sgu / 512); break;
         case SQ_EGU: {
-            const int jt = it / p.s_egu;
-            r.ks = it % p.s_egu; r.a = jt / g.egu_tiles; r.b = jt % g.egu_tiles;     // slot j, tile
+            const int jt = it / p.s_egu, tiles = g.I / 16;
+            r.ks = it % p.s_egu; r.a = jt / tiles; r.b = jt % tiles; *n_stages = 2 * (p.kr_egu / 512);
             break;
         }
-        case SQ_SD: r.a = it / p.s_sd; r.ks = it % p.s_sd; break;                    // tile
-        case SQ_EDOWN: r.a = it / g.ed_tiles; r.b = it % g.ed_tiles; break;          // slot j, tile
-        case SQ_UP: r.ks = it / g.up_tiles; r.a = it % g.up_tiles; break;            // tile, K-range major
+        case SQ_SD: r.a = it / p.s_sd; r.ks = it % p.s_sd; *n_stages = p.kr_sd / 512; break;
+        case SQ_EDOWN: r.a = it / (g.L / 16); r.b = it % (g.L / 16); *n_stages = g.I / 512; break;
+        case SQ_UP: r.ks = it / (g.H / 16); r.a = it % (g.H / 16); *n_stages = p.kr_up / 128; break;  // K major
+        default: *n_stages = 0; break;
     }
     return r;
 }
 
-// dependency of the activation block of an item
-DEVI int item_dep(int q, const Item &t) {
-    switch (q) {
-        case SQ_SGU: return kDepX16 + t.ks;
-        case SQ_EGU: return kDepH16 + t.ks;
-        case SQ_SD: return kDepSh16 + t.ks;
-        case SQ_EDOWN: return kDepA16 + t.a;
-        case SQ_UP: return kDepYl + t.ks;
-    }
-    return kDepNone;
-}
+// ---------------------------------------------------------------------------------------------
+// stage issue: lane r < 16 copies weight row r of the stage (256 B); for MXFP4, lane 16 + r copies
+// the row's 16 scale bytes.  The per-lane sources are computed once per item.
 
-DEVI bool dep_known(const StSmem &sm, int dep) {
-    return dep < 0 || ((*(volatile const unsigned *)&sm.dep_ready[dep >> 5]) >> (dep & 31) & 1u);
-}
-
-// global flag and target that make a dependency final
-DEVI void dep_flag(const StepArgs &a, const Geo &g, int dep, const unsigned **flag, unsigned *target) {
-    const StreamPlan &p = a.p.st;
-    const unsigned *ctl = a.ws.ctl;
-    if (dep >= kDepA16) { *flag = ctl + p.c_a16 + (dep - kDepA16); *target = 1u; }
-    else if (dep >= kDepYl) { *flag = ctl + p.c_yl + (dep - kDepYl); *target = (unsigned)(g.B * (p.kr_up / 64)); }
-    else if (dep >= kDepSh16) { *flag = ctl + p.c_sh16 + (dep - kDepSh16); *target = 1u; }
-    else if (dep >= kDepH16) { *flag = ctl + p.c_h16 + (dep - kDepH16); *target = 1u; }
-    else { *flag = ctl + p.c_x16 + dep; *target = (unsigned)g.B; }
-}
-
-// activation columns (and exponents) of stage c of item t of queue q
-template <bool ASYNC>
-DEVI void copy_act(const StepArgs &a, const Geo &g, const StSmem &sm, unsigned char *slot, int q, const Item &t,
-                   int c) {
-    const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31;
-    switch (q) {
-        case SQ_RT: {
-            const int k0 = t.ks * p.kr_rt + 128 * c;
-            copy_act_cols<ASYNC>(slot, g.B, kPitchB16, false, [&](int col) { return a.x + (size_t)col * g.H + k0; });
-            break;
-        }
-        case SQ_DN: {
-            const int k0 = t.ks * p.kr_dn + 128 * c;
-            copy_act_cols<ASYNC>(slot, g.B, kPitchB16, false, [&](int col) { return a.x + (size_t)col * g.H + k0; });
-            break;
-        }
-        case SQ_UP: {
-            const int k0 = t.ks * p.kr_up + 128 * c;
-            copy_act_cols<ASYNC>(slot, 2 * g.B, kPitchB16, false,
-                                 [&](int col) { return (const uint16_t *)a.ws.ylat16 + (size_t)col * g.L + k0; });
-            break;
-        }
-        case SQ_SGU: {
-            const int k0 = t.ks * p.kr_sgu + 128 * (c >> 1);
-            copy_act_cols<ASYNC>(slot, g.B, kPitchF16, true,
-                                 [&](int col) { return (const uint16_t *)a.ws.x16 + (size_t)col * g.H + k0; });
-            if (lane < g.B) copy_exp<ASYNC>(slot, lane, a.ws.x16e + t.ks * 4 + lane);
-            break;
-        }
-        case SQ_EGU: {
-            const int k0 = t.ks * p.kr_egu + 128 * (c >> 1);
-            const int cnt = sm.act_cnt[t.a], off = sm.act_off[t.a];
-            copy_act_cols<ASYNC>(slot, 2 * cnt, kPitchF16, true, [&](int col) {
-                const int tok = sm.ent[off + (col >> 1)] / g.K;
-                return (const uint16_t *)a.ws.h16 + (size_t)(2 * tok + (col & 1)) * g.L + k0;
-            });
-            if (lane < cnt) copy_exp<ASYNC>(slot, lane, a.ws.h16e + t.ks * 4 + sm.ent[off + lane] / g.K);
-            break;
-        }
-        case SQ_SD: {
-            const int k0 = t.ks * p.kr_sd + 128 * c;
-            copy_act_cols<ASYNC>(slot, 2 * g.B, kPitchF16, true,
-                                 [&](int col) { return (const uint16_t *)a.ws.sh16 + (size_t)col * g.Is + k0; });
-            if (lane < g.B) copy_exp<ASYNC>(slot, lane, a.ws.sh16e + t.ks * 4 + lane);
-            break;
-        }
-        case SQ_EDOWN: {
-            const int k0 = 128 * c;
-            const int cnt = sm.act_cnt[t.a], off = sm.act_off[t.a];
-            copy_act_cols<ASYNC>(slot, 2 * cnt, kPitchF16, true, [&](int col) {
-                const int ent = sm.ent[off + (col >> 1)];
-                return (const uint16_t *)a.ws.a16 + (size_t)(2 * ent + (col & 1)) * g.I + k0;
-            });
-            if (lane < cnt) copy_exp<ASYNC>(slot, lane, a.ws.a16e + t.a * 4 + lane);
-            break;
-        }
-    }
-}
-
-// Per-lane copy plan of the item being issued, computed once per item: every stage's copies are
-// then the plan's pointers plus a per-stage offset (a few instructions per 16-byte copy).
 struct IssuePlan {
-    const unsigned char *w;       // lane's weight piece 0, stage 0, matrix 0
-    const unsigned char *s;       // MXFP4: lane's scale row, stage 0, matrix 0; bf16: a valid address
-    long long dw, ds;             // MXFP4 pairs: byte offset of the up matrix from the gate matrix
-    int wpi, spi;                 // bytes between the lane's weight pieces / its two scale rows
-    unsigned valid;               // bf16: bit i set when piece i's row exists
-    uint32_t dst;                 // lane's piece-0 offset in a slot
-    const unsigned char *a0, *a1; // lane's activation pieces at stage 0 (null: none)
-    uint32_t adst0, adst1;
-    const int *ex;                // lane's exponent source (null: none)
-    bool fp4, pair;
+    const unsigned char *src;  // this lane's copy source at stage 0 (matrix 0)
+    long long dmat;            // MXFP4 gate/up pairs: offset of the up matrix's matching source
+    int step;                  // bytes the source advances per stage of one matrix
+    unsigned bytes;            // bytes of this lane's copy
+    uint32_t dst;              // its offset in a slot
+    unsigned expect;           // bytes of one stage
+    bool pair;
 };
-
-// activation column c of item t (its source row at the item's first k), for c < ncols
-DEVI const uint16_t *act_col(const StepArgs &a, const Geo &g, const StSmem &sm, int q, const Item &t, int c) {
-    const StreamPlan &p = a.p.st;
-    switch (q) {
-        case SQ_RT: return a.x + (size_t)c * g.H + t.ks * p.kr_rt;
-        case SQ_DN: return a.x + (size_t)c * g.H + t.ks * p.kr_dn;
-        case SQ_UP: return a.ws.ylat16 + (size_t)c * g.L + t.ks * p.kr_up;
-        case SQ_SGU: return a.ws.x16 + (size_t)c * g.H + t.ks * p.kr_sgu;
-        case SQ_EGU:
-            return a.ws.h16 + (size_t)(2 * (sm.ent[sm.act_off[t.a] + (c >> 1)] / g.K) + (c & 1)) * g.L + t.ks * p.kr_egu;
-        case SQ_SD: return a.ws.sh16 + (size_t)c * g.Is + t.ks * p.kr_sd;
-        default: return a.ws.a16 + (size_t)(2 * sm.ent[sm.act_off[t.a] + (c >> 1)] + (c & 1)) * g.I;  // SQ_EDOWN
-    }
-}
 
 DEVI IssuePlan make_plan(const StepArgs &a, const Geo &g, const StSmem &sm, int q, const Item &t) {
     const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, r = lane & 15;
     IssuePlan P;
-    P.dw = P.ds = 0;
-    P.ex = nullptr;
-    P.fp4 = !(q == SQ_RT || q == SQ_DN || q == SQ_UP);
+    P.dmat = 0;
     P.pair = (q == SQ_SGU || q == SQ_EGU);
-    if (!P.fp4) {
+    if (q == SQ_RT || q == SQ_DN || q == SQ_UP) {
         const uint16_t *W = q == SQ_RT ? a.w.router : q == SQ_DN ? a.w.w_dn : a.w.w_up;
         const int ld = q == SQ_UP ? g.L : g.H;
-        const int nrows = q == SQ_RT ? g.E : q == SQ_DN ? g.L : g.H;
         const int k0 = t.ks * (q == SQ_RT ? p.kr_rt : q == SQ_DN ? p.kr_dn : p.kr_up);
-        const int r0 = lane >> 4, u = lane & 15, row = 16 * t.a + r0;
-        P.w = reinterpret_cast<const unsigned char *>(W + (size_t)(row < nrows ? row : 0) * ld + k0 + 8 * u);
-        P.s = reinterpret_cast<const unsigned char *>(W);
-        P.wpi = 2 * ld * 2;
-        P.spi = 0;
-        P.valid = 0u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) P.valid |= (row + 2 * i < nrows ? 1u : 0u) << i;
-        P.dst = r0 * 256 + 16 * (u ^ ((r0 & 1) << 2));
+        P.src = reinterpret_cast<const unsigned char *>(W + (size_t)(16 * t.a + r) * ld + k0);
+        P.step = 256;
+        P.bytes = lane < 16 ? 256u : 0u;
+        P.dst = r * 256;
+        P.expect = 16 * 256;
+        return P;
+    }
+    const uint8_t *Q, *S;
+    size_t ldq, lds, row0;
+    int k0;
+    if (q == SQ_SGU) {
+        Q = a.w.sh_gate_q; S = a.w.sh_gate_s; ldq = g.H / 2; lds = g.H / 32; row0 = (size_t)16 * t.a;
+        k0 = t.ks * p.kr_sgu;
+        P.dmat = lane < 16 ? (long long)(a.w.sh_up_q - a.w.sh_gate_q) : (long long)(a.w.sh_up_s - a.w.sh_gate_s);
+    } else if (q == SQ_EGU) {
+        Q = a.w.gate_q; S = a.w.gate_s; ldq = g.L / 2; lds = g.L / 32;
+        row0 = (size_t)sm.act_e[t.a] * g.I + 16 * t.b;
+        k0 = t.ks * p.kr_egu;
+        P.dmat = lane < 16 ? (long long)(a.w.up_q - a.w.gate_q) : (long long)(a.w.up_s - a.w.gate_s);
+    } else if (q == SQ_SD) {
+        Q = a.w.sh_down_q; S = a.w.sh_down_s; ldq = g.Is / 2; lds = g.Is / 32; row0 = (size_t)16 * t.a;
+        k0 = t.ks * p.kr_sd;
+    } else {  // SQ_EDOWN
+        Q = a.w.down_q; S = a.w.down_s; ldq = g.I / 2; lds = g.I / 32;
+        row0 = (size_t)sm.act_e[t.a] * g.L + 16 * t.b;
+        k0 = 0;
+    }
+    if (lane < 16) {
+        P.src = Q + (row0 + r) * ldq + k0 / 2;
+        P.step = 256;
+        P.bytes = 256;
+        P.dst = r * 256;
     } else {
-        const uint8_t *Q, *S;
-        size_t ldq, lds, row0;
-        int k0;
-        if (q == SQ_SGU) {
-            Q = a.w.sh_gate_q; S = a.w.sh_gate_s; ldq = g.H / 2; lds = g.H / 32; row0 = (size_t)64 * t.a;
-            k0 = t.ks * p.kr_sgu;
-            P.dw = a.w.sh_up_q - a.w.sh_gate_q;
-            P.ds = a.w.sh_up_s - a.w.sh_gate_s;
-        } else if (q == SQ_EGU) {
-            Q = a.w.gate_q; S = a.w.gate_s; ldq = g.L / 2; lds = g.L / 32;
-            row0 = (size_t)sm.act_e[t.a] * g.I + 64 * t.b;
-            k0 = t.ks * p.kr_egu;
-            P.dw = a.w.up_q - a.w.gate_q;
-            P.ds = a.w.up_s - a.w.gate_s;
-        } else if (q == SQ_SD) {
-            Q = a.w.sh_down_q; S = a.w.sh_down_s; ldq = g.Is / 2; lds = g.Is / 32; row0 = (size_t)64 * t.a;
-            k0 = t.ks * p.kr_sd;
-        } else {  // SQ_EDOWN
-            Q = a.w.down_q; S = a.w.down_s; ldq = g.I / 2; lds = g.I / 32;
-            row0 = (size_t)sm.act_e[t.a] * g.L + 64 * t.b;
-            k0 = 0;
-        }
-        P.w = Q + (row0 + (lane >> 2)) * ldq + k0 / 2 + 16 * (lane & 3);
-        P.s = S + (row0 + lane) * lds + k0 / 32;
-        P.wpi = (int)(8 * ldq);
-        P.spi = (int)(32 * lds);
-        P.valid = 0xffu;
-        P.dst = (lane >> 2) * 64 + 16 * (lane & 3);
+        P.src = S + (row0 + r) * lds + k0 / 32;
+        P.step = 16;
+        P.bytes = 16;
+        P.dst = kSlotSc + r * 16;
     }
-    // activation pieces of this lane (lane + 32j for j < 2) and its exponent
-    int ncols, pitch = kPitchF16;
-    bool swz = true;
-    switch (q) {
-        case SQ_RT: case SQ_DN: ncols = g.B; pitch = kPitchB16; swz = false; break;
-        case SQ_UP: ncols = 2 * g.B; pitch = kPitchB16; swz = false; break;
-        case SQ_SGU: ncols = g.B; break;
-        case SQ_SD: ncols = 2 * g.B; break;
-        default: ncols = 2 * sm.act_cnt[t.a]; break;  // SQ_EGU, SQ_EDOWN
-    }
-    if (q == SQ_SGU && lane < g.B) P.ex = a.ws.x16e + t.ks * 4 + lane;
-    if (q == SQ_SD && lane < g.B) P.ex = a.ws.sh16e + t.ks * 4 + lane;
-    if (q == SQ_EGU && lane < sm.act_cnt[t.a]) P.ex = a.ws.h16e + t.ks * 4 + sm.ent[sm.act_off[t.a] + lane] / g.K;
-    if (q == SQ_EDOWN && lane < sm.act_cnt[t.a]) P.ex = a.ws.a16e + t.a * 4 + lane;
-    P.a0 = P.a1 = nullptr;
-    P.adst0 = P.adst1 = 0;
-    {
-        const int c = lane >> 4, u = lane & 15;
-        if (c < ncols) {
-            P.a0 = reinterpret_cast<const unsigned char *>(act_col(a, g, sm, q, t, c) + 8 * u);
-            P.adst0 = kSlotAct + c * pitch + 16 * (swz ? swz2(u) : u);
-        }
-        if (c + 2 < ncols) {
-            P.a1 = reinterpret_cast<const unsigned char *>(act_col(a, g, sm, q, t, c + 2) + 8 * u);
-            P.adst1 = kSlotAct + (c + 2) * pitch + 16 * (swz ? swz2(u) : u);
-        }
-    }
+    P.expect = 16 * 256 + 16 * 16;
     return P;
 }
 
-// stage c of the planned item: weights always, the activation part when `act`
-DEVI void issue_planned(const IssuePlan &P, uint32_t slot, int c, bool act) {
-    const int lane = threadIdx.x & 31;
+DEVI void issue_stage(const IssuePlan &P, unsigned char *slot, unsigned long long *bar, int c) {
     const int kk = P.pair ? (c >> 1) : c;
-    const bool up = P.pair && (c & 1);
-    if (P.fp4) {
-        const unsigned char *b = P.w + (up ? P.dw : 0) + 64 * kk;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cp16(slot + P.dst + 512 * i, b + i * P.wpi);
-        const unsigned char *sb = P.s + (up ? P.ds : 0) + 4 * kk;
-        cp4(slot + kSlotSc + 4 * lane, sb);
-        cp4(slot + kSlotSc + 4 * (lane + 32), sb + P.spi);
-    } else {
-        const unsigned char *b = P.w + 256 * kk;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const bool ok = (P.valid >> i) & 1u;
-            cp16_zfill(slot + P.dst + 512 * i, ok ? b + i * P.wpi : P.s, ok);
-        }
-    }
-    if (act) {
-        const int ka = 256 * kk;
-        if (P.a0) cp16(slot + P.adst0, P.a0 + ka);
-        if (P.a1) cp16(slot + P.adst1, P.a1 + ka);
-        if (P.ex) cp4(slot + kSlotExp + 4 * lane, P.ex);
+    if ((threadIdx.x & 31) == 0) mbar_arrive_expect_tx(bar, P.expect);
+    __syncwarp();
+    if (P.bytes) {
+        const unsigned char *src = P.src + (P.pair && (c & 1) ? P.dmat : 0) + (long long)P.step * kk;
+        bulk_copy(smem_addr(slot) + P.dst, src, P.bytes, bar);
     }
 }
 
 // ---------------------------------------------------------------------------------------------
-// stage compute
+// stage compute (weights from the slot, activation columns from the CTA's staging)
 
-// bf16: 16 rows x 128 k against up to 4 staged columns; two accumulator chains
-DEVI void mma_stage_bf16(const unsigned char *slot, int ncols, float (&acc0)[4], float (&acc1)[4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, sw = (g & 1) << 2;
-    const unsigned char *ra = slot + g * 256, *rb = slot + (g + 8) * 256;
-    const unsigned char *xc = slot + kSlotAct + (g < ncols ? g : 0) * kPitchB16;
+// bf16: 16 rows x 128 k; B column g is staged column col (or zero when col < 0)
+DEVI void mma_stage_bf16(const unsigned char *slot, const uint16_t *xs, int pitch, int kofs, int col,
+                         float (&acc0)[4], float (&acc1)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const unsigned char *ra = slot + g * 256 + 16 * q, *rb = ra + 8 * 256;
+    const uint16_t *xr = xs + (size_t)(col >= 0 ? col : 0) * pitch + kofs + 8 * q;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int u = 4 * r + q, uw = 16 * (u ^ sw);
-        const uint4 A = *reinterpret_cast<const uint4 *>(ra + uw);
-        const uint4 Bm = *reinterpret_cast<const uint4 *>(rb + uw);
-        uint4 xb = *reinterpret_cast<const uint4 *>(xc + 16 * u);
-        if (g >= ncols) xb = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 A = *reinterpret_cast<const uint4 *>(ra + 64 * r);
+        const uint4 Bm = *reinterpret_cast<const uint4 *>(rb + 64 * r);
+        uint4 xb = *reinterpret_cast<const uint4 *>(xr + 32 * r);
+        if (col < 0) xb = make_uint4(0u, 0u, 0u, 0u);
         mma_bf16(acc0, A.x, Bm.x, A.y, Bm.y, xb.x, xb.y);
         mma_bf16(acc1, A.z, Bm.z, A.w, Bm.w, xb.z, xb.w);
     }
@@ -451,23 +255,21 @@ DEVI void mma_stage_bf16(const unsigned char *slot, int ncols, float (&acc0)[4],
 
 // router: 16 rows (two 8-row groups) x 128 k in fp64 (slot q of step s of a 32-k chunk holds
 // k = 8q + s); column g is token g
-DEVI void mma_stage_router(const unsigned char *slot, int B, double (&c)[2][2], double (&d)[2][2]) {
+DEVI void mma_stage_router(const unsigned char *slot, const uint16_t *xs, int pitch, int kofs, int B,
+                           double (&c)[2][2], double (&d)[2][2]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const unsigned char *xc = slot + kSlotAct + (g < B ? g : 0) * kPitchB16;
+    const uint16_t *xr = xs + (size_t)(g < B ? g : 0) * pitch + kofs + 8 * q;
 #pragma unroll
-    for (int G = 0; G < 2; ++G) {
-        const int row = 8 * G + g, sw = (row & 1) << 2;
-        const unsigned char *ra = slot + row * 256;
+    for (int r = 0; r < 4; ++r) {
+        uint4 xb = *reinterpret_cast<const uint4 *>(xr + 32 * r);
+        if (g >= B) xb = make_uint4(0u, 0u, 0u, 0u);
+        const double xv[8] = {bf16_lo(xb.x), bf16_hi(xb.x), bf16_lo(xb.y), bf16_hi(xb.y),
+                              bf16_lo(xb.z), bf16_hi(xb.z), bf16_lo(xb.w), bf16_hi(xb.w)};
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            const int u = 4 * r + q;
-            const uint4 A = *reinterpret_cast<const uint4 *>(ra + 16 * (u ^ sw));
-            uint4 xb = *reinterpret_cast<const uint4 *>(xc + 16 * u);
-            if (g >= B) xb = make_uint4(0u, 0u, 0u, 0u);
+        for (int G = 0; G < 2; ++G) {
+            const uint4 A = *reinterpret_cast<const uint4 *>(slot + (8 * G + g) * 256 + 64 * r + 16 * q);
             const double av[8] = {bf16_lo(A.x), bf16_hi(A.x), bf16_lo(A.y), bf16_hi(A.y),
                                   bf16_lo(A.z), bf16_hi(A.z), bf16_lo(A.w), bf16_hi(A.w)};
-            const double xv[8] = {bf16_lo(xb.x), bf16_hi(xb.x), bf16_lo(xb.y), bf16_hi(xb.y),
-                                  bf16_lo(xb.z), bf16_hi(xb.z), bf16_lo(xb.w), bf16_hi(xb.w)};
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
                 mma_f64(c[G][0], c[G][1], av[2 * s], xv[2 * s]);
@@ -477,39 +279,38 @@ DEVI void mma_stage_router(const unsigned char *slot, int B, double (&c)[2][2], 
     }
 }
 
-// MXFP4: 64 rows (four 16-row tiles) x 128 k; lane quad q owns 32-element block q of each row;
-// word w of its 16 code bytes holds MMA steps 2w, 2w+1 against activation unit 4q + w
-DEVI void mma_stage_fp4(const unsigned char *slot, int ncols, float (&acc)[4][4]) {
+// MXFP4: 16 rows x 512 k (4 rounds of 128 k); lane quad q owns 32-element block 4r + q of each
+// row; word w of its 16 code bytes holds MMA steps 2w, 2w+1 against staged unit kofs/8 + 16r +
+// 4q + w (fp16 staging layout, swizzled); two accumulator chains
+DEVI void mma_stage_fp4(const unsigned char *slot, const uint16_t *xs, int pitch, int kofs, int col,
+                        float (&acc0)[4], float (&acc1)[4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3, sh = 8 * q;
-    uint4 v[4];
-    const unsigned char *xc = slot + kSlotAct + (g < ncols ? g : 0) * kPitchF16;
+    const uint16_t *xc = xs + (size_t)(col >= 0 ? col : 0) * pitch;
+    const int ubase = kofs / 8 + 4 * q, flip = q >> 1;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        v[w] = *reinterpret_cast<const uint4 *>(xc + 16 * swz2(4 * q + w));
-        if (g >= ncols) v[w] = make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        const int r0 = 16 * t + g, r1 = r0 + 8;
-        const uint4 c0 = *reinterpret_cast<const uint4 *>(slot + r0 * 64 + 16 * q);
-        const uint4 c1 = *reinterpret_cast<const uint4 *>(slot + r1 * 64 + 16 * q);
-        const uint32_t s0 = *reinterpret_cast<const uint32_t *>(slot + kSlotSc + 4 * r0);
-        const uint32_t s1 = *reinterpret_cast<const uint32_t *>(slot + kSlotSc + 4 * r1);
+    for (int r = 0; r < 4; ++r) {
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(slot + g * 256 + 64 * r + 16 * q);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(slot + (g + 8) * 256 + 64 * r + 16 * q);
+        const uint32_t s0 = *reinterpret_cast<const uint32_t *>(slot + kSlotSc + g * 16 + 4 * r);
+        const uint32_t s1 = *reinterpret_cast<const uint32_t *>(slot + kSlotSc + (g + 8) * 16 + 4 * r);
         const uint32_t f0 = e8m0_to_f16x2((s0 >> sh) & 0xffu), f1 = e8m0_to_f16x2((s1 >> sh) & 0xffu);
         const uint32_t w0[4] = {c0.x, c0.y, c0.z, c0.w}, w1[4] = {c1.x, c1.y, c1.z, c1.w};
+        const int u = ubase + 16 * r;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
+            uint4 v = *reinterpret_cast<const uint4 *>(xc + 8 * ((u + w) ^ flip));
+            if (col < 0) v = make_uint4(0u, 0u, 0u, 0u);
             uint32_t d0[4], d1[4];
             fp4_decode_word(w0[w], f0, d0);
             fp4_decode_word(w1[w], f1, d1);
-            mma_f16(acc[t], d0[0], d1[0], d0[1], d1[1], v[w].x, v[w].y);
-            mma_f16(acc[t], d0[2], d1[2], d0[3], d1[3], v[w].z, v[w].w);
+            mma_f16(acc0, d0[0], d1[0], d0[1], d1[1], v.x, v.y);
+            mma_f16(acc1, d0[2], d1[2], d0[3], d1[3], v.z, v.w);
         }
     }
 }
 
 // ---------------------------------------------------------------------------------------------
-// tickets, flags, conversions
+// tickets and flags
 
 DEVI bool warp_last_of(unsigned *counter, unsigned expected) {
     __threadfence();
@@ -539,42 +340,6 @@ DEVI void warp_publish(unsigned *flag, unsigned v) {
     __threadfence();
     __syncwarp();
     if ((threadIdx.x & 31) == 0) atomicExch(flag, v);
-}
-
-DEVI float warp_max(float m) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    return m;
-}
-
-// fp32 src[0..n) -> fp16 hi/lo rows dst_hi/dst_lo scaled by 2^-e, e from the block's max |v|;
-// n <= 1024 and a multiple of 64 (every load is issued before the first use)
-constexpr int kConvMax = 1024;
-DEVI int warp_to_f16_hilo(const float *src, uint16_t *dst_hi, uint16_t *dst_lo, int n) {
-    const int lane = threadIdx.x & 31;
-    float2 v[kConvMax / 64];
-    float m = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kConvMax / 64; ++j) {
-        const int i = 64 * j + 2 * lane;
-        v[j] = i < n ? __ldcg(reinterpret_cast<const float2 *>(src + i)) : make_float2(0.0f, 0.0f);
-    }
-#pragma unroll
-    for (int j = 0; j < kConvMax / 64; ++j) m = fmaxf(m, fmaxf(fabsf(v[j].x), fabsf(v[j].y)));
-    const int e = prescale_shift(warp_max(m));
-    const float sc = exp2i(-e);
-#pragma unroll
-    for (int j = 0; j < kConvMax / 64; ++j) {
-        const int i = 64 * j + 2 * lane;
-        if (i < n) {
-            const float x0 = v[j].x * sc, x1 = v[j].y * sc;
-            const uint32_t hi = pack_f16x2(x0, x1);
-            const uint32_t lo = pack_f16x2(x0 - f16_lo(hi), x1 - f16_hi(hi));
-            *reinterpret_cast<uint32_t *>(dst_hi + i) = hi;
-            *reinterpret_cast<uint32_t *>(dst_lo + i) = lo;
-        }
-    }
-    return e;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -692,7 +457,7 @@ DEVI void st_buckets(const StepArgs &a, const Geo &g, StSmem &sm) {
     warp_publish(a.ws.ctl + CTL_ROUTE_READY, 1u);
 }
 
-// the CTA's copy of the routing tables (first warp to need it loads it)
+// the CTA's copy of the routing tables (first warp to need it loads it; an earlier launch made it)
 DEVI bool ensure_routing(const StepArgs &a, StSmem &sm) {
     const int lane = threadIdx.x & 31;
     volatile int *state = &sm.route_state;
@@ -702,7 +467,7 @@ DEVI bool ensure_routing(const StepArgs &a, StSmem &sm) {
     mine = __shfl_sync(0xffffffffu, mine, 0);
     if (mine) {
         if (!warp_wait_geq(a, a.ws.ctl + CTL_ROUTE_READY, 1u)) {
-            if (lane == 0) atomicExch(&sm.route_state, 3);  // aborted
+            if (lane == 0) atomicExch(&sm.route_state, 3);
             return false;
         }
         const int n = __ldcg(a.ws.n_active);
@@ -713,14 +478,11 @@ DEVI bool ensure_routing(const StepArgs &a, StSmem &sm) {
         }
         for (int p = lane; p < a.B * a.d.k && p < kMaxActive; p += 32) sm.ent[p] = __ldcg(a.ws.entries + p);
         if (lane == 0) sm.n_active = n;
-        if (a.ws.trace && lane == 0)
-            a.ws.trace[((size_t)blockIdx.x * kTraceRowsPerSm + (threadIdx.x >> 5)) * kTraceStamps + 12] = global_ns();
         __threadfence_block();
         __syncwarp();
         if (lane == 0) atomicExch(&sm.route_state, 2);
         return true;
     }
-    // another warp of this CTA loads it
     const unsigned long long t0 = global_ns();
     for (;;) {
         const int s = *state;
@@ -741,10 +503,11 @@ DEVI bool ensure_routing(const StepArgs &a, StSmem &sm) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// epilogues (after the last stage of an item)
+// epilogues (after the last stage of an item); accumulator entry j of a lane is row g (j < 2) or
+// g + 8 (j >= 2), MMA column 2q + (j & 1)
 
 struct Acc {
-    float f[2][4][4];     // [gate|up][row tile][4] for MXFP4; f[0][0..1] chains for bf16
+    float f[2][2][4];  // [gate|up][chain][4]
     double c[2][2], d[2][2];
 };
 
@@ -752,35 +515,14 @@ DEVI void acc_zero(Acc &r) {
 #pragma unroll
     for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int t = 0; t < 4; ++t)
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) r.f[m][t][j] = 0.0f;
+            for (int j = 0; j < 4; ++j) r.f[m][h][j] = 0.0f;
 #pragma unroll
     for (int G = 0; G < 2; ++G) r.c[G][0] = r.c[G][1] = r.d[G][0] = r.d[G][1] = 0.0;
 }
 
-// x16 block (token, 512 k): bf16 x -> fp16 x * 2^-e
-DEVI void st_x16(const StepArgs &a, const Geo &g, int it) {
-    const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31, t = it / p.s_sgu, kb = it % p.s_sgu, k0 = kb * p.kr_sgu;
-    const uint16_t *src = a.x + (size_t)t * g.H + k0;
-    float m = 0.0f;
-    for (int i = 2 * lane; i < p.kr_sgu; i += 64) {
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(src + i);
-        m = fmaxf(m, fmaxf(fabsf(bf16_lo(v)), fabsf(bf16_hi(v))));
-    }
-    const int e = prescale_shift(warp_max(m));
-    const float sc = exp2i(-e);
-    uint16_t *dst = a.ws.x16 + (size_t)t * g.H + k0;
-    for (int i = 2 * lane; i < p.kr_sgu; i += 64) {
-        const uint32_t v = *reinterpret_cast<const uint32_t *>(src + i);
-        *reinterpret_cast<uint32_t *>(dst + i) = pack_f16x2(bf16_lo(v) * sc, bf16_hi(v) * sc);
-    }
-    if (lane == 0) a.ws.x16e[kb * 4 + t] = e;
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) atomicAdd(a.ws.ctl + p.c_x16 + kb, 1u);
-}
+DEVI float accv(const Acc &r, int m, int j) { return r.f[m][0][j] + r.f[m][1][j]; }
 
 DEVI void epi_router(const StepArgs &a, const Geo &g, StSmem &sm, const Item &t, Acc &r) {
     const StreamPlan &p = a.p.st;
@@ -789,40 +531,30 @@ DEVI void epi_router(const StepArgs &a, const Geo &g, StSmem &sm, const Item &t,
 #pragma unroll
     for (int G = 0; G < 2; ++G) {
         const int row = 16 * t.a + 8 * G + gg;
-        if (row < g.E) {
-            if (2 * q < g.B) part[(size_t)(2 * q) * g.E + row] = r.c[G][0] + r.d[G][0];
-            if (2 * q + 1 < g.B) part[(size_t)(2 * q + 1) * g.E + row] = r.c[G][1] + r.d[G][1];
-        }
+        if (2 * q < g.B) part[(size_t)(2 * q) * g.E + row] = r.c[G][0] + r.d[G][0];
+        if (2 * q + 1 < g.B) part[(size_t)(2 * q + 1) * g.E + row] = r.c[G][1] + r.d[G][1];
     }
     if (!warp_last_of(a.ws.ctl + p.c_rt_tk + t.a, (unsigned)p.s_rt)) return;
     for (int i = lane; i < 16 * g.B; i += 32) {
         const int b = i >> 4, row = 16 * t.a + (i & 15);
-        if (row < g.E) {
-            const float lg = (float)sum_splits<double, 16>(a.ws.st_rt_part + (size_t)b * g.E + row, (size_t)2 * g.E, p.s_rt);
-            a.ws.logits[(size_t)b * g.E + row] = lg;
-            // top-k key: fp32 sigmoid score (computed in double) bits + 1; 0 marks "no expert"
-            const float sc = (float)(1.0 / (1.0 + exp(-(double)lg)));
-            a.ws.st_key[(size_t)b * g.E + row] = (sc >= 0.0f ? __float_as_uint(sc) : 0u) + 1u;
-        }
+        const float lg = (float)sum_splits<double, 16>(a.ws.st_rt_part + (size_t)b * g.E + row, (size_t)2 * g.E, p.s_rt);
+        a.ws.logits[(size_t)b * g.E + row] = lg;
+        // top-k key: fp32 sigmoid score (computed in double) bits + 1; 0 marks "no expert"
+        const float sc = (float)(1.0 / (1.0 + exp(-(double)lg)));
+        a.ws.st_key[(size_t)b * g.E + row] = (sc >= 0.0f ? __float_as_uint(sc) : 0u) + 1u;
     }
     if (a.flags & kFlagTestStall) return;  // the routing never completes: its waits must time out
-    if (!warp_count_reaches(a.ws.ctl + CTL_RT_DONE, (unsigned)g.rt_groups)) return;
+    if (!warp_count_reaches(a.ws.ctl + CTL_RT_DONE, (unsigned)(g.E / 16))) return;
     unsigned long long *tr =
         a.ws.trace ? a.ws.trace + ((size_t)blockIdx.x * kTraceRowsPerSm + (threadIdx.x >> 5)) * kTraceStamps : nullptr;
     if (tr && lane == 0) tr[14] = global_ns();
-    const long long c0 = clock64();
     for (int b = 0; b < g.B; ++b) st_topk_token(a, g, sm, b);
-    const long long c1 = clock64();
     if (tr && lane == 0) tr[15] = global_ns();
     st_buckets(a, g, sm);
-    const long long c2 = clock64();
-    if (tr && lane == 0) {
-        tr[11] = global_ns();
-        tr[8] = c1 - c0;
-        tr[13] = c2 - c1;
-    }
+    if (tr && lane == 0) tr[11] = global_ns();
 }
 
+// 16-row split-K tile of B token columns (x columns are tokens: column 2q + j is token 2q + j)
 DEVI void epi_dn(const StepArgs &a, const Geo &g, const Item &t, Acc &r) {
     const StreamPlan &p = a.p.st;
     const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
@@ -831,36 +563,145 @@ DEVI void epi_dn(const StepArgs &a, const Geo &g, const Item &t, Acc &r) {
 #pragma unroll
     for (int j = 0; j < 2; ++j)
         if (2 * q + j < g.B) {
-            part[(size_t)(2 * q + j) * g.L + row] = r.f[0][0][j] + r.f[0][1][j];
-            part[(size_t)(2 * q + j) * g.L + row + 8] = r.f[0][0][2 + j] + r.f[0][1][2 + j];
+            part[(size_t)(2 * q + j) * g.L + row] = accv(r, 0, j);
+            part[(size_t)(2 * q + j) * g.L + row + 8] = accv(r, 0, 2 + j);
         }
     if (!warp_last_of(a.ws.ctl + p.c_dn_tk + t.a, (unsigned)p.s_dn)) return;
     for (int i = lane; i < 16 * g.B; i += 32) {
         const int b = i >> 4, rr = 16 * t.a + (i & 15);
         a.ws.h[(size_t)b * g.L + rr] = sum_splits(a.ws.st_dn_part + (size_t)b * g.L + rr, (size_t)2 * g.L, p.s_dn);
     }
-    const int kb = (16 * t.a) / p.kr_egu;
-    if (!warp_count_reaches(a.ws.ctl + p.c_dnb + kb, (unsigned)(p.kr_egu / 16))) return;
-    for (int b = 0; b < g.B; ++b) {
-        const int e = warp_to_f16_hilo(a.ws.h + (size_t)b * g.L + kb * p.kr_egu,
-                                       a.ws.h16 + (size_t)(2 * b) * g.L + kb * p.kr_egu,
-                                       a.ws.h16 + (size_t)(2 * b + 1) * g.L + kb * p.kr_egu, p.kr_egu);
-        if (lane == 0) a.ws.h16e[kb * 4 + b] = e;
-    }
-    warp_publish(a.ws.ctl + p.c_h16 + kb, 1u);
 }
 
+// shared gate/up: x16 columns are tokens, scaled by 2^-shift[token]
+DEVI void epi_sgu(const StepArgs &a, const Geo &g, const StSmem &sm, const Item &t, Acc &r) {
+    const StreamPlan &p = a.p.st;
+    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
+    float *part = a.ws.st_sgu_part + (size_t)t.ks * 2 * 2 * g.Is;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int b = 2 * q + j;
+        if (b < g.B) {
+            const float sc = exp2i(sm.shift[b]);
+            float *pg = part + (size_t)b * 2 * g.Is, *pu = pg + g.Is;
+            const int row = 16 * t.a + gg;
+            pg[row] = accv(r, 0, j) * sc;
+            pg[row + 8] = accv(r, 0, 2 + j) * sc;
+            pu[row] = accv(r, 1, j) * sc;
+            pu[row + 8] = accv(r, 1, 2 + j) * sc;
+        }
+    }
+    if (!warp_last_of(a.ws.ctl + p.c_sgu_tk + t.a, (unsigned)p.s_sgu)) return;
+    const size_t st = (size_t)2 * 2 * g.Is;
+    for (int i = lane; i < 16 * g.B; i += 32) {
+        const int b = i >> 4, rr = 16 * t.a + (i & 15);
+        const float *pb = a.ws.st_sgu_part + (size_t)b * 2 * g.Is;
+        const float gs = sum_splits(pb + rr, st, p.s_sgu), us = sum_splits(pb + g.Is + rr, st, p.s_sgu);
+        a.ws.sh_a[(size_t)b * g.Is + rr] = gs / (1.0f + expf(-gs)) * us;
+    }
+}
+
+// expert gate/up: columns 2m, 2m+1 are entry m's hi and lo parts (h of its token)
+DEVI void epi_egu(const StepArgs &a, const Geo &g, const StSmem &sm, const Item &t, Acc &r) {
+    const StreamPlan &p = a.p.st;
+    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
+    const int cnt = sm.act_cnt[t.a], off = sm.act_off[t.a];
+    const int nent = g.B * g.K;
+    if (q < cnt) {
+        const int ent = sm.ent[off + q];
+        const float sc = exp2i(sm.shift[ent / g.K]);
+        float *pg = a.ws.st_egu_part + ((size_t)t.ks * nent + ent) * 2 * g.I, *pu = pg + g.I;
+        const int row = 16 * t.b + gg;
+        pg[row] = (accv(r, 0, 0) + accv(r, 0, 1)) * sc;
+        pg[row + 8] = (accv(r, 0, 2) + accv(r, 0, 3)) * sc;
+        pu[row] = (accv(r, 1, 0) + accv(r, 1, 1)) * sc;
+        pu[row + 8] = (accv(r, 1, 2) + accv(r, 1, 3)) * sc;
+    }
+    if (!warp_last_of(a.ws.ctl + p.c_egu_tk + t.a * (g.I / 16) + t.b, (unsigned)p.s_egu)) return;
+    const size_t st = (size_t)nent * 2 * g.I;
+    for (int i = lane; i < 16 * cnt; i += 32) {
+        const int m = i >> 4, rr = 16 * t.b + (i & 15);
+        const int ent = sm.ent[off + m];
+        const float *pb = a.ws.st_egu_part + (size_t)ent * 2 * g.I;
+        const float gs = sum_splits(pb + rr, st, p.s_egu), us = sum_splits(pb + g.I + rr, st, p.s_egu);
+        a.ws.a[(size_t)ent * g.I + rr] = gs / (1.0f + expf(-gs)) * us;
+    }
+}
+
+// shared down: columns 2q, 2q+1 are token q's hi and lo parts
+DEVI void epi_sd(const StepArgs &a, const Geo &g, const StSmem &sm, const Item &t, Acc &r) {
+    const StreamPlan &p = a.p.st;
+    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
+    float *part = a.ws.st_sd_part + (size_t)t.ks * 2 * g.H;
+    if (q < g.B) {
+        const float sc = exp2i(sm.shift[g.B + q]);
+        const int row = 16 * t.a + gg;
+        part[(size_t)q * g.H + row] = (accv(r, 0, 0) + accv(r, 0, 1)) * sc;
+        part[(size_t)q * g.H + row + 8] = (accv(r, 0, 2) + accv(r, 0, 3)) * sc;
+    }
+    if (!warp_last_of(a.ws.ctl + p.c_sd_tk + t.a, (unsigned)p.s_sd)) return;
+    for (int i = lane; i < 16 * g.B; i += 32) {
+        const int b = i >> 4, rr = 16 * t.a + (i & 15);
+        a.ws.sh[(size_t)b * g.H + rr] = sum_splits(a.ws.st_sd_part + (size_t)b * g.H + rr, (size_t)2 * g.H, p.s_sd);
+    }
+}
+
+// expert down (full K): y rows of the slot's entries; the K-th entry of a (token, tile) combines
+// the token's 16 latent rows in slot order
+DEVI void epi_edown(const StepArgs &a, const Geo &g, const StSmem &sm, const Item &t, Acc &r) {
+    const StreamPlan &p = a.p.st;
+    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
+    const int cnt = sm.act_cnt[t.a], off = sm.act_off[t.a];
+    if (q < cnt) {
+        const int ent = sm.ent[off + q];
+        const float sc = exp2i(sm.shift[(t.a - sm.ed_j0) * g.B + q]);
+        float *y = a.ws.y + (size_t)ent * g.L + 16 * t.b + gg;
+        y[0] = (accv(r, 0, 0) + accv(r, 0, 1)) * sc;
+        y[8] = (accv(r, 0, 2) + accv(r, 0, 3)) * sc;
+    }
+    __threadfence();
+    __syncwarp();
+    unsigned mine = 0;
+    if (lane < cnt) {
+        const int tok = sm.ent[off + lane] / g.K;
+        mine = atomicAdd(a.ws.ctl + p.c_comb + tok * (g.L / 16) + t.b, 1u) == (unsigned)(g.K - 1) ? 1u : 0u;
+    }
+    unsigned todo = __ballot_sync(0xffffffffu, mine != 0);
+    if (todo) __threadfence();
+    while (todo) {
+        const int m = __ffs(todo) - 1;
+        todo &= todo - 1;
+        const int tok = sm.ent[off + m] / g.K;
+        // lane (row i, half h) adds the weighted slots of its parity in slot order
+        const int l = 16 * t.b + (lane & 15), h = lane >> 4;
+        float s = 0.0f;
+        for (int r0 = h; r0 < g.K; r0 += 16) {
+            float wv[8], yv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int rr = r0 + 2 * j;
+                wv[j] = rr < g.K ? __ldcg(a.ws.wts + (size_t)tok * g.K + rr) : 0.0f;
+                yv[j] = rr < g.K ? __ldcg(a.ws.y + ((size_t)tok * g.K + rr) * g.L + l) : 0.0f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) s += wv[j] * yv[j];
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        if (lane < 16) a.ws.ylat[(size_t)tok * g.L + l] = s;
+    }
+}
+
+// W_up: ylat columns 2q, 2q+1 are token q's bf16 hi and lo parts; out = bf16(. + sh)
 DEVI void epi_up(const StepArgs &a, const Geo &g, const Item &t, Acc &r) {
     const StreamPlan &p = a.p.st;
     const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
     float *part = a.ws.st_up_part + (size_t)t.ks * 2 * g.H;
     const int row = 16 * t.a + gg;
-    if (q < g.B) {  // columns 2q, 2q+1: token q's hi and lo parts
-        part[(size_t)q * g.H + row] = (r.f[0][0][0] + r.f[0][1][0]) + (r.f[0][0][1] + r.f[0][1][1]);
-        part[(size_t)q * g.H + row + 8] = (r.f[0][0][2] + r.f[0][1][2]) + (r.f[0][0][3] + r.f[0][1][3]);
+    if (q < g.B) {
+        part[(size_t)q * g.H + row] = accv(r, 0, 0) + accv(r, 0, 1);
+        part[(size_t)q * g.H + row + 8] = accv(r, 0, 2) + accv(r, 0, 3);
     }
     if (!warp_last_of(a.ws.ctl + p.c_up_tk + t.a, (unsigned)p.s_up)) return;
-    if (g.ns && !warp_wait_geq(a, a.ws.ctl + CTL_SD_DONE, (unsigned)g.sd_tiles)) return;
     for (int i = lane; i < 16 * g.B; i += 32) {
         const int b = i >> 4, rr = 16 * t.a + (i & 15);
         const float s = sum_splits(a.ws.st_up_part + (size_t)b * g.H + rr, (size_t)2 * g.H, p.s_up);
@@ -870,165 +711,120 @@ DEVI void epi_up(const StepArgs &a, const Geo &g, const Item &t, Acc &r) {
     }
 }
 
-DEVI void epi_sgu(const StepArgs &a, const Geo &g, const Item &t, Acc &r, const unsigned char *slot) {
-    const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
-    float *part = a.ws.st_sgu_part + (size_t)t.ks * 2 * 2 * g.Is;
-    const int *ex = reinterpret_cast<const int *>(slot + kSlotExp);
+// ---------------------------------------------------------------------------------------------
+// activation staging of a launch (all threads of the CTA)
+
+constexpr int kStageMax = 6;  // 16-byte units (4 fp32 or 8 bf16) each thread stages at most
+
+// fp32 rows -> fp16 hi/lo column pairs: row r (n floats at rows[r]) becomes columns (2r, 2r+1) of the
+// fp16 staging xs (swizzled units), scaled by 2^-shift[base + r] with the shift from the row's max
+// |v|.  Every load is issued before the first use: one L2 round trip.
+DEVI void cta_stage_f32_rows(uint16_t *xs, int pitch, const float *const *rows, int nrows, int n, StSmem &sm,
+                             int base) {
+    const int units = n / 4, total = nrows * units;
+    if ((int)threadIdx.x < nrows) sm.amax[base + threadIdx.x] = 0u;
+    float4 v[kStageMax];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int b = 2 * q + j;  // x16 columns are tokens
-        if (b < g.B) {
-            const float sc = exp2i(ex[b]);
-            float *pg = part + (size_t)b * 2 * g.Is, *pu = pg + g.Is;
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        v[j] = u < total ? __ldcg(reinterpret_cast<const float4 *>(rows[u / units]) + u % units)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
 #pragma unroll
-            for (int tt = 0; tt < 4; ++tt) {
-                const int row = 64 * t.a + 16 * tt + gg;
-                pg[row] = r.f[0][tt][j] * sc;
-                pg[row + 8] = r.f[0][tt][2 + j] * sc;
-                pu[row] = r.f[1][tt][j] * sc;
-                pu[row + 8] = r.f[1][tt][2 + j] * sc;
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        if (u < total) {
+            const float m = fmaxf(fmaxf(fabsf(v[j].x), fabsf(v[j].y)), fmaxf(fabsf(v[j].z), fabsf(v[j].w)));
+            atomicMax(sm.amax + base + u / units, __float_as_uint(m));
+        }
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < nrows) sm.shift[base + threadIdx.x] = prescale_shift(__uint_as_float(sm.amax[base + threadIdx.x]));
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        if (u < total) {
+            const int r = u / units, k = 4 * (u % units);
+            const float sc = exp2i(-sm.shift[base + r]);
+            const float x0 = v[j].x * sc, x1 = v[j].y * sc, x2 = v[j].z * sc, x3 = v[j].w * sc;
+            const uint32_t h01 = pack_f16x2(x0, x1), h23 = pack_f16x2(x2, x3);
+            const uint32_t l01 = pack_f16x2(x0 - f16_lo(h01), x1 - f16_hi(h01));
+            const uint32_t l23 = pack_f16x2(x2 - f16_lo(h23), x3 - f16_hi(h23));
+            const int off = 8 * swz(k >> 3) + (k & 7);
+            *reinterpret_cast<uint2 *>(xs + (size_t)(2 * r) * pitch + off) = make_uint2(h01, h23);
+            *reinterpret_cast<uint2 *>(xs + (size_t)(2 * r + 1) * pitch + off) = make_uint2(l01, l23);
+        }
+    }
+}
+
+// x (B bf16 rows of H): bf16 columns t of xs, and (with a shared expert) fp16 columns t of x16
+// scaled by 2^-shift[t] from the token's max |x|; one L2 round trip
+DEVI void cta_stage_x(uint16_t *xs, uint16_t *x16, const StepArgs &a, const Geo &g, StSmem &sm) {
+    const int units = g.H / 8, total = g.B * units;
+    if ((int)threadIdx.x < g.B) sm.amax[threadIdx.x] = 0u;
+    uint4 v[kStageMax];
+#pragma unroll
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        v[j] = u < total ? *reinterpret_cast<const uint4 *>(a.x + (size_t)u * 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        if (u < total) {
+            const int t = u / units, k = 8 * (u % units);
+            *reinterpret_cast<uint4 *>(xs + (size_t)t * bf16_pitch(g.H) + k) = v[j];
+            if (g.ns) {
+                const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+                float m = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fabsf(bf16_lo(w4[i])), fabsf(bf16_hi(w4[i]))));
+                atomicMax(sm.amax + t, __float_as_uint(m));
             }
         }
     }
-    if (!warp_last_of(a.ws.ctl + p.c_sgu_tk + t.a, (unsigned)p.s_sgu)) return;
-    const size_t st = (size_t)2 * 2 * g.Is;
-    for (int i = lane; i < 64 * g.B; i += 32) {
-        const int b = i >> 6, rr = 64 * t.a + (i & 63);
-        const float *pb = a.ws.st_sgu_part + (size_t)b * 2 * g.Is;
-        const float gs = sum_splits(pb + rr, st, p.s_sgu), us = sum_splits(pb + g.Is + rr, st, p.s_sgu);
-        a.ws.sh_a[(size_t)b * g.Is + rr] = gs / (1.0f + expf(-gs)) * us;
+    if (!g.ns) return;
+    __syncthreads();
+    if ((int)threadIdx.x < g.B) sm.shift[threadIdx.x] = prescale_shift(__uint_as_float(sm.amax[threadIdx.x]));
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        if (u < total) {
+            const int t = u / units, k = 8 * (u % units);
+            const float sc = exp2i(-sm.shift[t]);
+            const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] = pack_f16x2(bf16_lo(w4[i]) * sc, bf16_hi(w4[i]) * sc);
+            *reinterpret_cast<uint4 *>(x16 + (size_t)t * f16_pitch(g.H) + 8 * swz(k >> 3)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
-    const int kb = (64 * t.a) / p.kr_sd;
-    if (!warp_count_reaches(a.ws.ctl + p.c_sgb + kb, (unsigned)(p.kr_sd / 64))) return;
-    for (int b = 0; b < g.B; ++b) {
-        const int e = warp_to_f16_hilo(a.ws.sh_a + (size_t)b * g.Is + kb * p.kr_sd,
-                                       a.ws.sh16 + (size_t)(2 * b) * g.Is + kb * p.kr_sd,
-                                       a.ws.sh16 + (size_t)(2 * b + 1) * g.Is + kb * p.kr_sd, p.kr_sd);
-        if (lane == 0) a.ws.sh16e[kb * 4 + b] = e;
-    }
-    warp_publish(a.ws.ctl + p.c_sh16 + kb, 1u);
 }
 
-DEVI void epi_egu(const StepArgs &a, const Geo &g, const StSmem &sm, const Item &t, Acc &r,
-                  const unsigned char *slot) {
-    const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
-    const int cnt = sm.act_cnt[t.a], off = sm.act_off[t.a];
-    const int nent = g.B * g.K;
-    const int *ex = reinterpret_cast<const int *>(slot + kSlotExp);
-    if (q < cnt) {  // columns 2q, 2q+1: the slot's entry q, hi and lo parts
-        const int ent = sm.ent[off + q];
-        const float sc = exp2i(ex[q]);
-        float *pg = a.ws.st_egu_part + ((size_t)t.ks * nent + ent) * 2 * g.I, *pu = pg + g.I;
+// ylat (B fp32 rows of L) -> bf16 hi/lo columns (2t, 2t+1); one L2 round trip
+DEVI void cta_stage_ylat(uint16_t *xs, const StepArgs &a, const Geo &g) {
+    const int units = g.L / 4, total = g.B * units, pitch = bf16_pitch(g.L);
+    float4 v[kStageMax];
 #pragma unroll
-        for (int tt = 0; tt < 4; ++tt) {
-            const int row = 64 * t.b + 16 * tt + gg;
-            pg[row] = (r.f[0][tt][0] + r.f[0][tt][1]) * sc;
-            pg[row + 8] = (r.f[0][tt][2] + r.f[0][tt][3]) * sc;
-            pu[row] = (r.f[1][tt][0] + r.f[1][tt][1]) * sc;
-            pu[row + 8] = (r.f[1][tt][2] + r.f[1][tt][3]) * sc;
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        v[j] = u < total ? __ldcg(reinterpret_cast<const float4 *>(a.ws.ylat) + u) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < kStageMax; ++j) {
+        const int u = threadIdx.x + j * blockDim.x;
+        if (u < total) {
+            const int t = u / units, k = 4 * (u % units);
+            const uint32_t h01 = pack_bf16x2(v[j].x, v[j].y), h23 = pack_bf16x2(v[j].z, v[j].w);
+            const uint32_t l01 = pack_bf16x2(v[j].x - bf16_lo(h01), v[j].y - bf16_hi(h01));
+            const uint32_t l23 = pack_bf16x2(v[j].z - bf16_lo(h23), v[j].w - bf16_hi(h23));
+            *reinterpret_cast<uint2 *>(xs + (size_t)(2 * t) * pitch + k) = make_uint2(h01, h23);
+            *reinterpret_cast<uint2 *>(xs + (size_t)(2 * t + 1) * pitch + k) = make_uint2(l01, l23);
         }
-    }
-    if (!warp_last_of(a.ws.ctl + p.c_egu_tk + t.a * g.egu_tiles + t.b, (unsigned)p.s_egu)) return;
-    const size_t st = (size_t)nent * 2 * g.I;
-    for (int i = lane; i < 64 * cnt; i += 32) {
-        const int m = i >> 6, rr = 64 * t.b + (i & 63);
-        const int ent = sm.ent[off + m];
-        const float *pb = a.ws.st_egu_part + (size_t)ent * 2 * g.I;
-        const float gs = sum_splits(pb + rr, st, p.s_egu), us = sum_splits(pb + g.I + rr, st, p.s_egu);
-        a.ws.a[(size_t)ent * g.I + rr] = gs / (1.0f + expf(-gs)) * us;
-    }
-    if (!warp_count_reaches(a.ws.ctl + p.c_gu + t.a, (unsigned)g.egu_tiles)) return;
-    for (int m = 0; m < cnt; ++m) {
-        const int ent = sm.ent[off + m];
-        const int e = warp_to_f16_hilo(a.ws.a + (size_t)ent * g.I, a.ws.a16 + (size_t)(2 * ent) * g.I,
-                                       a.ws.a16 + (size_t)(2 * ent + 1) * g.I, g.I);
-        if (lane == 0) a.ws.a16e[t.a * 4 + m] = e;
-    }
-    warp_publish(a.ws.ctl + p.c_a16 + t.a, 1u);
-}
-
-DEVI void epi_sd(const StepArgs &a, const Geo &g, const Item &t, Acc &r, const unsigned char *slot) {
-    const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
-    const int *ex = reinterpret_cast<const int *>(slot + kSlotExp);
-    float *part = a.ws.st_sd_part + (size_t)t.ks * 2 * g.H;
-    if (q < g.B) {
-        const float sc = exp2i(ex[q]);
-#pragma unroll
-        for (int tt = 0; tt < 4; ++tt) {
-            const int row = 64 * t.a + 16 * tt + gg;
-            part[(size_t)q * g.H + row] = (r.f[0][tt][0] + r.f[0][tt][1]) * sc;
-            part[(size_t)q * g.H + row + 8] = (r.f[0][tt][2] + r.f[0][tt][3]) * sc;
-        }
-    }
-    if (!warp_last_of(a.ws.ctl + p.c_sd_tk + t.a, (unsigned)p.s_sd)) return;
-    for (int i = lane; i < 64 * g.B; i += 32) {
-        const int b = i >> 6, rr = 64 * t.a + (i & 63);
-        a.ws.sh[(size_t)b * g.H + rr] = sum_splits(a.ws.st_sd_part + (size_t)b * g.H + rr, (size_t)2 * g.H, p.s_sd);
-    }
-    warp_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
-}
-
-DEVI void epi_edown(const StepArgs &a, const Geo &g, const StSmem &sm, const Item &t, Acc &r,
-                    const unsigned char *slot) {
-    const StreamPlan &p = a.p.st;
-    const int lane = threadIdx.x & 31, gg = lane >> 2, q = lane & 3;
-    const int cnt = sm.act_cnt[t.a], off = sm.act_off[t.a];
-    const int *ex = reinterpret_cast<const int *>(slot + kSlotExp);
-    if (q < cnt) {
-        const int ent = sm.ent[off + q];
-        const float sc = exp2i(ex[q]);
-        float *y = a.ws.y + (size_t)ent * g.L;
-#pragma unroll
-        for (int tt = 0; tt < 4; ++tt) {
-            const int row = 64 * t.b + 16 * tt + gg;
-            y[row] = (r.f[0][tt][0] + r.f[0][tt][1]) * sc;
-            y[row + 8] = (r.f[0][tt][2] + r.f[0][tt][3]) * sc;
-        }
-    }
-    __threadfence();
-    __syncwarp();
-    // one count per entry on its (token, 64-row tile); the K-th combines the token's rows
-    unsigned mine = 0;
-    if (lane < cnt) {
-        const int tok = sm.ent[off + lane] / g.K;
-        mine = atomicAdd(a.ws.ctl + p.c_comb + tok * g.ed_tiles + t.b, 1u) == (unsigned)(g.K - 1) ? 1u : 0u;
-    }
-    unsigned todo = __ballot_sync(0xffffffffu, mine != 0);
-    if (todo) __threadfence();
-    while (todo) {
-        const int m = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const int tok = sm.ent[off + m] / g.K;
-        // ylat rows 64*tile + 2*lane, +1: weighted slot sum in slot order
-        const int l = 64 * t.b + 2 * lane;
-        float s0 = 0.0f, s1 = 0.0f;
-        for (int r0 = 0; r0 < g.K; r0 += 8) {
-            float wv[8];
-            float2 yv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int rr = r0 + j;
-                wv[j] = rr < g.K ? __ldcg(a.ws.wts + (size_t)tok * g.K + rr) : 0.0f;
-                yv[j] = rr < g.K ? __ldcg(reinterpret_cast<const float2 *>(a.ws.y + ((size_t)tok * g.K + rr) * g.L + l))
-                                 : make_float2(0.0f, 0.0f);
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (r0 + j < g.K) {
-                    s0 += wv[j] * yv[j].x;
-                    s1 += wv[j] * yv[j].y;
-                }
-        }
-        a.ws.ylat[(size_t)tok * g.L + l] = s0;
-        a.ws.ylat[(size_t)tok * g.L + l + 1] = s1;
-        const uint32_t hi = pack_bf16x2(s0, s1);
-        const uint32_t lo = pack_bf16x2(s0 - bf16_lo(hi), s1 - bf16_hi(hi));
-        *reinterpret_cast<uint32_t *>(a.ws.ylat16 + (size_t)(2 * tok) * g.L + l) = hi;
-        *reinterpret_cast<uint32_t *>(a.ws.ylat16 + (size_t)(2 * tok + 1) * g.L + l) = lo;
-        warp_signal_add(a.ws.ctl + p.c_yl + (64 * t.b) / p.kr_up, 1u);
     }
 }
 
@@ -1037,9 +833,8 @@ DEVI void epi_edown(const StepArgs &a, const Geo &g, const StSmem &sm, const Ite
 // ---------------------------------------------------------------------------------------------
 // the kernel
 
-// One launch runs queues [q_lo, q_hi); the step is four launches (see launch_stream), and the
-// last one (q_hi == SQ_N) clears the control block for the next step.
-__global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_lo, int q_hi) {
+// Launch `ph` (0..3) of a step; the last one clears the control block for the next step.
+__global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int ph) {
     extern __shared__ __align__(128) unsigned char st_dyn[];
     __shared__ StSmem sm;
     const Geo g = geo(a);
@@ -1047,56 +842,46 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
     unsigned *ctl = a.ws.ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     unsigned char *ring = st_dyn + (size_t)warp * kStStages * kSlotBytes;
+    uint16_t *xs = reinterpret_cast<uint16_t *>(st_dyn + kRingBytes);  // the launch's activations
+    const int q_lo = ph == 0 ? SQ_RT : ph == 1 ? SQ_SD : ph == 2 ? SQ_EDOWN : SQ_UP;
+    const int q_hi = ph == 0 ? SQ_SD : ph == 1 ? SQ_EDOWN : ph == 2 ? SQ_UP : SQ_N;
     unsigned long long *trace =
         a.ws.trace ? a.ws.trace + ((size_t)blockIdx.x * kTraceRowsPerSm + warp) * kTraceStamps : nullptr;
-    auto stamp = [&](int i) {
-        if (trace && lane == 0) trace[i] = global_ns();
-    };
-    if (trace && lane < kTraceStamps) trace[lane] = 0ull;
-    __syncwarp();
-    stamp(0);
-    // row 12 of the SM: start and end of this CTA in each of the step's launches
     unsigned long long *launch_row =
         a.ws.trace ? a.ws.trace + ((size_t)blockIdx.x * kTraceRowsPerSm + 12) * kTraceStamps : nullptr;
-    const int launch_no = q_lo == SQ_X16 ? 0 : q_lo == SQ_EGU ? 1 : q_lo == SQ_EDOWN ? 2 : 3;
-    if (launch_row && threadIdx.x == 0) launch_row[2 * launch_no] = global_ns();
+    if (trace && lane < kTraceStamps && (ph == 0 || (lane != 11 && lane != 14 && lane != 15))) trace[lane] = 0ull;
+    if (trace && lane == 0) trace[0] = global_ns();
+    if (launch_row && threadIdx.x == 0) launch_row[2 * ph] = global_ns();
+    if (a.ws.trace && ph == 0 && threadIdx.x < kTraceStamps)
+        a.ws.trace[((size_t)blockIdx.x * kTraceRowsPerSm + 13) * kTraceStamps + threadIdx.x] = 0ull;
 
-    // after the first launch, every activation block a queue reads was finished by an earlier launch
-    for (int i = threadIdx.x; i < kDepBits / 32; i += blockDim.x) sm.dep_ready[i] = q_lo > SQ_SGU ? ~0u : 0u;
-    cta_take_init(sm.claim);
+    if (lane < kStStages) mbar_init(&sm.bar[warp][lane], 1u);
     if (threadIdx.x == 0) {
         sm.route_state = 0;
         sm.n_active = 0;
+        sm.ed_j0 = 0;
     }
+    cta_take_init(sm.claim);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
 
     // producer state (warp-uniform)
-    int pq = q_lo, pit = -1, pc = 0, pn = 0, pdep = kDepNone;
+    int pq = q_lo, pit = -1, pc = 0, pn = 0;
     Item pitem = {0, 0, 0};
     IssuePlan pplan;
     int n_iss = 0, n_con = 0;
     bool alive = true;
-    int n_active = -1;  // known once the CTA's routing copy is loaded
+    int n_active = -1;
 
-    // items come from this CTA's range of each queue (one lane per warp takes)
     auto claim_next = [&](int q, int n) {
         int v = -1;
         if (lane == 0) v = cta_take(sm.claim, q, n);
         return __shfl_sync(0xffffffffu, v, 0);
     };
-    auto routing_known = [&]() {
-        if (n_active >= 0) return true;
-        if (*(volatile int *)&sm.route_state == 2) {
-            n_active = sm.n_active;
-            return true;
-        }
-        return false;
-    };
-    // next item for the producer; false when none can start now (routing unknown) or all done
-    auto next_item = [&](bool may_block) -> bool {
+    auto next_item = [&](bool routed) -> bool {
         while (pq < q_hi) {
-            if ((pq == SQ_EGU || pq == SQ_EDOWN) && !routing_known()) {
-                if (!may_block) return false;
+            if ((pq == SQ_EGU || pq == SQ_EDOWN) && n_active < 0) {
+                if (!routed) return false;  // before the launch dependency resolves: no routing yet
                 if (!ensure_routing(a, sm)) {
                     alive = false;
                     return false;
@@ -1107,35 +892,28 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
             const int it = n > 0 ? claim_next(pq, n) : -1;
             if (it >= 0) {
                 pit = it;
-                pitem = decode_item(a, g, pq, it);
+                pitem = decode_item(a, g, pq, it, &pn);
                 pc = 0;
-                pn = item_stages(a, g, pq);
                 pplan = make_plan(a, g, sm, pq, pitem);
-                pdep = item_dep(pq, pitem);
                 return true;
             }
             ++pq;
         }
         return false;
     };
-    // issue stages until the ring is full or nothing more can start without waiting
-    auto top_up = [&](bool may_block) {
+    auto top_up = [&](bool routed) {
         while (alive && n_iss - n_con < kStStages) {
             if (pit < 0 || pc == pn) {
                 pit = -1;
-                if (!next_item(may_block && n_iss == n_con)) return;
+                if (!next_item(routed)) return;
             }
             const int s = n_iss % kStStages;
-            unsigned char *slot = ring + (size_t)s * kSlotBytes;
-            const bool act = dep_known(sm, pdep);
-            issue_planned(pplan, smem_addr(slot), pc, act);
-            cp_commit();
+            issue_stage(pplan, ring + (size_t)s * kSlotBytes, &sm.bar[warp][s], pc);
             if (lane == 0) {
                 sm.meta[warp][s].q = pq;
                 sm.meta[warp][s].item = pit;
                 sm.meta[warp][s].c = pc;
                 sm.meta[warp][s].n = pn;
-                sm.meta[warp][s].act = act ? 1 : 0;
             }
             __syncwarp();
             ++pc;
@@ -1143,152 +921,242 @@ __global__ void __launch_bounds__(kStWarps * 32, 1) k_stream(StepArgs a, int q_l
         }
     };
 
-    // fp16 copies of x for the shared gate/up (few items; taken before the rings start)
-    if (g.ns && q_lo <= SQ_X16) {
-        const int n = queue_len(a, g, SQ_X16, 0);
-        for (int it = claim_next(SQ_X16, n); it >= 0; it = claim_next(SQ_X16, n)) st_x16(a, g, it);
+    // The next launch may be scheduled onto SMs as this one's CTAs leave (its weight copies need
+    // nothing of ours); it reads our results only after its griddepcontrol.wait.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // start the copies that need nothing of the previous launches (weights of the queues before
+    // the routed ones), then wait for the previous launch, stage its results while they fly
+    top_up(false);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (ph == 0) {
+        // x as bf16 (router, W_dn) and as fp16 * 2^-shift[token] (shared gate/up)
+        cta_stage_x(xs, xs + (size_t)g.B * bf16_pitch(g.H), a, g, sm);
+    } else if (ph == 1) {
+        // h (all tokens) and sh_a as fp16 hi/lo columns; shift[t] for h, shift[B + t] for sh_a
+        const float *rows[2 * kStMaxBatch];
+        for (int t = 0; t < g.B; ++t) {
+            rows[t] = a.ws.h + (size_t)t * g.L;
+            rows[g.B + t] = a.ws.sh_a + (size_t)t * g.Is;
+        }
+        cta_stage_f32_rows(xs, f16_pitch(g.L), rows, g.B, g.L, sm, 0);
+        if (g.ns) cta_stage_f32_rows(xs + (size_t)2 * g.B * f16_pitch(g.L), f16_pitch(g.Is), rows + g.B, g.B, g.Is, sm, g.B);
+    } else if (ph == 2) {
+        // a of the entries of the (at most two) experts of this CTA's range, fp16 hi/lo; expert
+        // j0 + e, entry m: columns 2(e B + m) + part, shift[e B + m]
+        __shared__ int s_ok, s_rows[2 * kMaxEdownExperts * kStMaxBatch], s_nr;
+        if (warp == 0) {
+            const bool ok = ensure_routing(a, sm);
+            if (lane == 0) s_ok = ok ? 1 : 0;
+        }
+        __syncthreads();
+        alive = alive && s_ok;
+        const int n = sm.n_active * (g.L / 16);
+        const long long G = gridDim.x, cc = blockIdx.x;
+        const int lo = (int)((long long)n * cc / G), hi = (int)((long long)n * (cc + 1) / G);
+        if (s_ok && hi > lo) {
+            const int j0 = lo / (g.L / 16), j1 = (hi - 1) / (g.L / 16);
+            if (threadIdx.x == 0) {
+                int nr = 0;
+                for (int e = 0; e <= j1 - j0 && e < kMaxEdownExperts; ++e)
+                    for (int m = 0; m < g.B; ++m) {
+                        const int cnt = sm.act_cnt[j0 + e];
+                        s_rows[e * g.B + m] = sm.ent[sm.act_off[j0 + e] + (m < cnt ? m : 0)];
+                        nr = e * g.B + m + 1;
+                    }
+                s_nr = nr;
+                sm.ed_j0 = j0;
+            }
+            __syncthreads();
+            const float *rows[2 * kMaxEdownExperts * kStMaxBatch];
+            for (int i = 0; i < s_nr; ++i) rows[i] = a.ws.a + (size_t)s_rows[i] * g.I;
+            cta_stage_f32_rows(xs, f16_pitch(g.I), rows, s_nr, g.I, sm, 0);
+        }
+    } else {
+        // ylat as bf16 hi/lo columns (2t, 2t+1)
+        cta_stage_ylat(xs, a, g);
     }
-    stamp(1);
+    __syncthreads();
+    if (trace && lane == 0) trace[1] = global_ns();
+    const unsigned long long t_staged = a.ws.trace ? global_ns() : 0ull;
+    unsigned long long *spread =
+        a.ws.trace ? a.ws.trace + ((size_t)blockIdx.x * kTraceRowsPerSm + 14) * kTraceStamps + 4 * ph : nullptr;
+    if (spread && threadIdx.x == 0) {
+        spread[0] = t_staged - launch_row[2 * ph];  // launch start to activations staged
+        spread[1] = 0ull;                           // latest warp finish after staging
+        spread[2] = ~0ull;                          // earliest warp finish after staging
+    }
+    __syncthreads();
 
     Acc acc;
     acc_zero(acc);
-    Item cit = {0, 0, 0};  // the item being consumed
-    long long cyc_issue = 0, cyc_data = 0, cyc_dep = 0, cyc_compute = 0, cyc_epi = 0;
+    Item cit = {0, 0, 0};
+    long long cyc_issue = 0, cyc_data = 0, cyc_compute = 0, cyc_epi = 0;
     for (;;) {
         const long long ti0 = trace ? clock64() : 0;
         top_up(true);
         const long long ti1 = trace ? clock64() : 0;
         cyc_issue += ti1 - ti0;
-        if (!alive || n_con == n_iss) break;  // aborted, or every queue is drained
+        if (!alive || n_con == n_iss) break;  // aborted, or every queue of this launch is drained
         const int s = n_con % kStStages;
         unsigned char *slot = ring + (size_t)s * kSlotBytes;
-        cp_wait(n_iss - n_con - 1);
-        __syncwarp();
-        const long long td0 = trace ? clock64() : 0;
-        cyc_data += td0 - ti1;
+        if (!slot_wait(a, &sm.bar[warp][s], (unsigned)((n_con / kStStages) & 1))) {
+            alive = false;
+            break;
+        }
+        const long long td = trace ? clock64() : 0;
+        cyc_data += td - ti1;
         const SlotMeta m = sm.meta[warp][s];
-        if (m.c == 0) cit = decode_item(a, g, m.q, m.item);
+        if (m.c == 0) {
+            int ns_;
+            cit = decode_item(a, g, m.q, m.item, &ns_);
+            acc_zero(acc);
+        }
         const Item it = cit;
-        if (!m.act) {
-            // the activation block was not final when the weights were issued: wait for it, then
-            // copy the activation part of every issued stage that waits on the same block (those
-            // copies write the slots' activation areas only, never bytes still in flight)
-            const int dep = item_dep(m.q, it);
-            if (!dep_known(sm, dep)) {
-                const unsigned *flag;
-                unsigned target;
-                dep_flag(a, g, dep, &flag, &target);
-                if (!warp_wait_geq(a, flag, target)) {
-                    alive = false;
-                    break;
-                }
-                if (lane == 0) atomicOr(&sm.dep_ready[dep >> 5], 1u << (dep & 31));
-            }
-            for (int k = n_con; k < n_iss; ++k) {
-                const int s2 = k % kStStages;
-                const SlotMeta m2 = sm.meta[warp][s2];
-                if (m2.act) continue;
-                const Item it2 = decode_item(a, g, m2.q, m2.item);
-                if (item_dep(m2.q, it2) != dep) continue;
-                copy_act<false>(a, g, sm, ring + (size_t)s2 * kSlotBytes, m2.q, it2, m2.c);
-                __syncwarp();
-                if (lane == 0) sm.meta[warp][s2].act = 1;
-            }
-            __syncwarp();
-        }
-        if (trace) cyc_dep += clock64() - td0;
-        if (m.c == 0) acc_zero(acc);
-        const long long tc0 = trace ? clock64() : 0;
-        const bool upm = m.c & 1;
+        const int gcol = lane >> 2;
         switch (m.q) {
-            case SQ_RT: mma_stage_router(slot, g.B, acc.c, acc.d); break;
-            case SQ_DN: mma_stage_bf16(slot, g.B, acc.f[0][0], acc.f[0][1]); break;
-            case SQ_UP: mma_stage_bf16(slot, 2 * g.B, acc.f[0][0], acc.f[0][1]); break;
-            case SQ_SGU:
-                if (upm) mma_stage_fp4(slot, g.B, acc.f[1]);
-                else mma_stage_fp4(slot, g.B, acc.f[0]);
+            case SQ_RT:
+                mma_stage_router(slot, xs, bf16_pitch(g.H), it.ks * p.kr_rt + 128 * m.c, g.B, acc.c, acc.d);
                 break;
-            case SQ_EGU:
-                if (upm) mma_stage_fp4(slot, 2 * sm.act_cnt[it.a], acc.f[1]);
-                else mma_stage_fp4(slot, 2 * sm.act_cnt[it.a], acc.f[0]);
+            case SQ_DN:
+                mma_stage_bf16(slot, xs, bf16_pitch(g.H), it.ks * p.kr_dn + 128 * m.c, gcol < g.B ? gcol : -1,
+                               acc.f[0][0], acc.f[0][1]);
                 break;
-            case SQ_SD: mma_stage_fp4(slot, 2 * g.B, acc.f[0]); break;
-            case SQ_EDOWN: mma_stage_fp4(slot, 2 * sm.act_cnt[it.a], acc.f[0]); break;
+            case SQ_UP:
+                mma_stage_bf16(slot, xs, bf16_pitch(g.L), it.ks * p.kr_up + 128 * m.c, gcol < 2 * g.B ? gcol : -1,
+                               acc.f[0][0], acc.f[0][1]);
+                break;
+            case SQ_SGU: {
+                const uint16_t *x16 = xs + (size_t)g.B * bf16_pitch(g.H);
+                const int kofs = it.ks * p.kr_sgu + 512 * (m.c >> 1), col = gcol < g.B ? gcol : -1;
+                if (m.c & 1) mma_stage_fp4(slot, x16, f16_pitch(g.H), kofs, col, acc.f[1][0], acc.f[1][1]);
+                else mma_stage_fp4(slot, x16, f16_pitch(g.H), kofs, col, acc.f[0][0], acc.f[0][1]);
+                break;
+            }
+            case SQ_EGU: {
+                // MMA column gcol: entry gcol/2 of the slot, hi (even) or lo (odd) part of its token's h
+                const int cnt = sm.act_cnt[it.a];
+                const int col = (gcol >> 1) < cnt ? 2 * (sm.ent[sm.act_off[it.a] + (gcol >> 1)] / g.K) + (gcol & 1) : -1;
+                const int kofs = it.ks * p.kr_egu + 512 * (m.c >> 1);
+                if (m.c & 1) mma_stage_fp4(slot, xs, f16_pitch(g.L), kofs, col, acc.f[1][0], acc.f[1][1]);
+                else mma_stage_fp4(slot, xs, f16_pitch(g.L), kofs, col, acc.f[0][0], acc.f[0][1]);
+                break;
+            }
+            case SQ_SD: {
+                const uint16_t *s16 = xs + (size_t)2 * g.B * f16_pitch(g.L);
+                mma_stage_fp4(slot, s16, f16_pitch(g.Is), it.ks * p.kr_sd + 512 * m.c, gcol < 2 * g.B ? gcol : -1,
+                              acc.f[0][0], acc.f[0][1]);
+                break;
+            }
+            case SQ_EDOWN: {
+                const int cnt = sm.act_cnt[it.a];
+                const int col = gcol < 2 * cnt ? 2 * (it.a - sm.ed_j0) * g.B + gcol : -1;
+                mma_stage_fp4(slot, xs, f16_pitch(g.I), 512 * m.c, col, acc.f[0][0], acc.f[0][1]);
+                break;
+            }
         }
-        __syncwarp();
+        __syncwarp();  // every lane is done with the slot before it is refilled
         const long long tc1 = trace ? clock64() : 0;
-        cyc_compute += tc1 - tc0;
+        cyc_compute += tc1 - td;
         if (m.c == m.n - 1) {
             switch (m.q) {
                 case SQ_RT: epi_router(a, g, sm, it, acc); break;
                 case SQ_DN: epi_dn(a, g, it, acc); break;
                 case SQ_UP: epi_up(a, g, it, acc); break;
-                case SQ_SGU: epi_sgu(a, g, it, acc, slot); break;
-                case SQ_EGU: epi_egu(a, g, sm, it, acc, slot); break;
-                case SQ_SD: epi_sd(a, g, it, acc, slot); break;
-                case SQ_EDOWN: epi_edown(a, g, sm, it, acc, slot); break;
+                case SQ_SGU: epi_sgu(a, g, sm, it, acc); break;
+                case SQ_EGU: epi_egu(a, g, sm, it, acc); break;
+                case SQ_SD: epi_sd(a, g, sm, it, acc); break;
+                case SQ_EDOWN: epi_edown(a, g, sm, it, acc); break;
             }
             __syncwarp();
             if (trace) cyc_epi += clock64() - tc1;
         }
         ++n_con;
     }
-    cp_wait(0);  // nothing of this warp's may still land in shared memory
-    __syncwarp();
-    stamp(9);
+    // an aborted warp still owns copies in flight: let them land before the CTA leaves
+    for (; n_con < n_iss; ++n_con)
+        if (!slot_wait(a, &sm.bar[warp][n_con % kStStages], (unsigned)((n_con / kStStages) & 1))) break;
+    if (spread && lane == 0) {
+        const unsigned long long dt = global_ns() - t_staged;
+        atomicMax(spread + 1, dt);
+        atomicMin(spread + 2, dt);
+    }
     if (trace && lane == 0) {
         trace[2] = cyc_issue;
         trace[3] = cyc_data;
-        trace[4] = cyc_dep;
         trace[5] = cyc_compute;
         trace[6] = cyc_epi;
-        trace[7] = n_con;
+        trace[7] = n_iss;
+        trace[9] = global_ns();
+        // row 13 of the SM: this launch's cycle sums over the CTA's warps (issue, data, compute,
+        // epilogue), 4 stamps per launch
+        unsigned long long *sums = a.ws.trace + ((size_t)blockIdx.x * kTraceRowsPerSm + 13) * kTraceStamps + 4 * ph;
+        atomicAdd(sums + 0, (unsigned long long)cyc_issue);
+        atomicAdd(sums + 1, (unsigned long long)cyc_data);
+        atomicAdd(sums + 2, (unsigned long long)cyc_compute);
+        atomicAdd(sums + 3, (unsigned long long)cyc_epi);
     }
 
-    // leave; the last CTA out clears the control block for the next step
+    // leave; the last CTA out of the last launch clears the control block for the next step
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
-        sm.exit_last = (atomicAdd(ctl + CTL_EXIT, 1u) == gridDim.x - 1) ? 1 : 0;
+        sm.exit_last = (atomicAdd(ctl + CTL_QHEAD + ph, 1u) == gridDim.x - 1) ? 1 : 0;  // per-launch exit count
     }
     __syncthreads();
-    stamp(10);
-    if (launch_row && threadIdx.x == 0) launch_row[2 * launch_no + 1] = global_ns();
+    if (trace && lane == 0) trace[10] = global_ns();
+    if (launch_row && threadIdx.x == 0) launch_row[2 * ph + 1] = global_ns();
     if (sm.exit_last) {
         __threadfence();
-        if (q_hi == SQ_N) {
+        if (ph == kStreamLaunches - 1) {
             for (int i = threadIdx.x; i < CTL_FIXED; i += blockDim.x) ctl[i] = 0u;
             for (int i = p.c_rt_tk + threadIdx.x; i < p.words; i += blockDim.x) ctl[i] = 0u;
-        } else if (threadIdx.x == 0) {
-            ctl[CTL_EXIT] = 0u;  // the next launch counts its own CTAs; everything else carries over
         }
     }
 }
 
-bool stream_supports(const Dims &d, int B) {
-    if (B < 1 || B > kStMaxBatch || d.k > 32 || d.k > d.E || d.E > 1024 || B * d.k > kMaxActive) return false;
-    if (d.H % 128 || d.L % 128 || d.I % 128 || d.I > kConvMax || (d.n_shared && d.Is % 128)) return false;
-    StreamPlan sp;
-    stream_plan(d, sp, 0);
-    return sp.s_sgu <= 64 && sp.s_egu <= 16 && sp.kr_egu <= kConvMax && sp.s_sd <= 16 && sp.kr_sd <= kConvMax &&
-           sp.s_up <= 32;
+// ---------------------------------------------------------------------------------------------
+// host side
+
+// dynamic shared memory: the rings, then the largest activation staging of the four launches
+static size_t stream_smem(const Dims &d, int B) {
+    size_t act = (size_t)B * bf16_pitch(d.H) * 2 + (d.n_shared ? (size_t)B * f16_pitch(d.H) * 2 : 0);
+    act = std::max(act, (size_t)2 * B * f16_pitch(d.L) * 2 + (d.n_shared ? (size_t)2 * B * f16_pitch(d.Is) * 2 : 0));
+    act = std::max(act, (size_t)2 * kMaxEdownExperts * B * f16_pitch(d.I) * 2);
+    act = std::max(act, (size_t)2 * B * bf16_pitch(d.L) * 2);
+    return (size_t)kRingBytes + act;
 }
 
-// largest multiple of 128 that is <= pref and divides K (K is a multiple of 128)
-static int pick_range(int K, int pref) {
-    for (int r = pref - pref % 128; r >= 128; r -= 128)
+constexpr size_t kStSmemLimit = 216 * 1024;  // dynamic; the static part is a few KB
+
+bool stream_supports(const Dims &d, int B) {
+    if (B < 1 || B > kStMaxBatch || d.k > 32 || d.k > d.E || d.E > 1024 || B * d.k > kMaxActive) return false;
+    // whole MXFP4 stages (512 k, 16-byte scale rows) and bf16 stages (128 k); 16-row tiles
+    if (d.H % 512 || d.L % 512 || d.I % 512 || (d.n_shared && d.Is % 512) || d.E % 16) return false;
+    // a CTA's expert-down range (n_active * L/16 items over the grid) spans at most two experts
+    // as long as there are no more active experts than CTAs (>= 1 per SM, and n_active <= 64)
+    // batched staging: at most kStageMax 16-byte units per thread in every launch
+    const int cap = kStageMax * kStWarps * 32;
+    if (B * d.H / 8 > cap || B * d.L / 4 > cap || (d.n_shared && B * d.Is / 4 > cap) ||
+        kMaxEdownExperts * B * d.I / 4 > cap)
+        return false;
+    return stream_smem(d, B) <= kStSmemLimit;
+}
+
+// largest multiple of `unit` that is <= pref and divides K (K is a multiple of unit)
+static int pick_range(int K, int pref, int unit) {
+    for (int r = pref - pref % unit; r >= unit; r -= unit)
         if (K % r == 0) return r;
-    return 128;
+    return unit;
 }
 
 void stream_plan(const Dims &d, StreamPlan &sp, int ctl_base) {
-    const int Is = d.n_shared ? d.Is : 128;
-    sp.kr_rt = pick_range(d.H, 512);
-    sp.kr_dn = pick_range(d.H, 896);
-    sp.kr_sgu = pick_range(d.H, 512);
-    sp.kr_egu = pick_range(d.L, 512);
-    sp.kr_sd = pick_range(Is, 512);
-    sp.kr_up = pick_range(d.L, 256);
+    const int Is = d.n_shared ? d.Is : 512;
+    sp.kr_rt = pick_range(d.H, 512, 128);
+    sp.kr_dn = pick_range(d.H, 512, 128);
+    sp.kr_sgu = pick_range(d.H, 512, 512);
+    sp.kr_egu = pick_range(d.L, 512, 512);
+    sp.kr_sd = pick_range(Is, 512, 512);
+    sp.kr_up = pick_range(d.L, 256, 128);
     sp.s_rt = d.H / sp.kr_rt;
     sp.s_dn = d.H / sp.kr_dn;
     sp.s_sgu = d.H / sp.kr_sgu;
@@ -1298,47 +1166,39 @@ void stream_plan(const Dims &d, StreamPlan &sp, int ctl_base) {
     int c = ctl_base;
     sp.c_rt_tk = c; c += (d.E + 15) / 16;
     sp.c_dn_tk = c; c += d.L / 16;
-    sp.c_dnb = c; c += sp.s_egu;
-    sp.c_h16 = c; c += sp.s_egu;
-    sp.c_x16 = c; c += sp.s_sgu;
-    sp.c_sgu_tk = c; c += Is / 64;
-    sp.c_sgb = c; c += sp.s_sd;
-    sp.c_sh16 = c; c += sp.s_sd;
-    sp.c_egu_tk = c; c += d.E * (d.I / 64);
-    sp.c_gu = c; c += d.E;
-    sp.c_a16 = c; c += d.E;
-    sp.c_sd_tk = c; c += d.H / 64;
-    sp.c_comb = c; c += kStMaxBatch * (d.L / 64);
-    sp.c_yl = c; c += sp.s_up;
+    sp.c_sgu_tk = c; c += Is / 16;
+    sp.c_egu_tk = c; c += d.E * (d.I / 16);
+    sp.c_sd_tk = c; c += d.H / 16;
+    sp.c_comb = c; c += kStMaxBatch * (d.L / 16);
     sp.c_up_tk = c; c += d.H / 16;
     sp.words = c;
 }
 
 // The step as four launches, each of which only runs work whose inputs the previous launches
-// finished: (x16, router and top-k, W_dn, shared gate/up), (expert gate/up, shared down),
-// (expert down and combine), (W_up).  Inside a launch no warp waits on another's results, so
-// every warp streams; a stage's activation block is always final when it is issued.
+// finished (see the top of this file).
 cudaError_t launch_stream(const StepArgs &a, cudaStream_t s, int n_sm) {
-    static const int bounds[5] = {SQ_X16, SQ_EGU, SQ_EDOWN, SQ_UP, SQ_N};
     cudaError_t e = cudaSuccess;
+    const size_t smem = stream_smem(a.d, a.B);
     for (int ph = 0; ph < kStreamLaunches && e == cudaSuccess; ++ph) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(n_sm);
         cfg.blockDim = dim3(kStWarps * 32);
-        cfg.dynamicSmemBytes = kStDynSmem;
+        cfg.dynamicSmemBytes = smem;
         cfg.stream = s;
+        // launches 2..4 may start as SMs free up (they wait for the previous launch's results on
+        // the device); the first one waits for the previous step like any stream-ordered launch
         cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeCooperative;
-        attr[0].val.cooperative = 1;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, k_stream, a, bounds[ph], bounds[ph + 1]);
+        cfg.numAttrs = ph > 0 ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, k_stream, a, ph);
     }
     return e;
 }
 
 cudaError_t init_stream_attributes() {
-    return cudaFuncSetAttribute(k_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, kStDynSmem);
+    return cudaFuncSetAttribute(k_stream, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStSmemLimit);
 }
 
 }  // namespace moedec

@@ -10,6 +10,7 @@ Workloads (the five shapes the layer is exercised on):
 name               shape
 =================  ====================================================================
 tiny_b1            H=512, L=256, E=64, k=4, I=256, I_s=256, B=1
+mid_b2             H=1024, L=512, E=128, k=8, I=512, I_s=512, B=2 (perturbed second token)
 full_b1            H=7168, L=2048, E=896, k=16, I=1024, I_s=2048, B=1
 full_b2            full size, B=2; token 1 = bf16(token 0 + 0.1 N(0,1))
 full_b16           full size, B=16, independent N(0,1) tokens
@@ -108,6 +109,8 @@ class Dims:
 
 TINY = Dims(hidden=512, latent=256, n_experts=64, top_k=4, expert_inter=256, shared_inter=256)
 FULL = Dims(hidden=7168, latent=2048, n_experts=896, top_k=16, expert_inter=1024, shared_inter=2048)
+# a small layer whose every dimension is a multiple of 512 (the streaming schedule's unit)
+MID = Dims(hidden=1024, latent=512, n_experts=128, top_k=8, expert_inter=512, shared_inter=512)
 
 
 @dataclass(frozen=True)
@@ -131,6 +134,8 @@ HOT_BETA_B64 = 20.0
 
 WORKLOADS = {
     "tiny_b1": Workload("tiny_b1", TINY, 1, 1000, description="tiny latent-MoE layer, B=1"),
+    "mid_b2": Workload("mid_b2", MID, 2, 1005, tokens="perturbed",
+                       description="small layer (dims multiples of 512), B=2, token 1 = token 0 + 0.1 N(0,1)"),
     "full_b1": Workload("full_b1", FULL, 1, 1001, description="full-size layer, B=1"),
     "full_b2": Workload("full_b2", FULL, 2, 1002, tokens="perturbed",
                         description="full-size layer, B=2, token 1 = token 0 + 0.1 N(0,1)"),

@@ -11,8 +11,8 @@ import pytest
 
 import oracle
 import synth
-from tests.harness import (assert_close, assert_logits_match, layer_dims, rel_errors, run_layer, to_device,
-                           upload_weights)
+from tests.harness import (assert_close, assert_logits_match, bf16_tensor_to_f32, layer_dims, rel_errors, run_layer,
+                           to_device, upload_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +55,57 @@ def _check_step(w, W, x, layer, tokens=None, check_all_routing=True):
         assert_close(taps["up"][t], r["out"][0] - r["sh"][0], f"up[{t}]")
         assert_close(out[t], r["out"][0], f"out[{t}]")
     return out, idx
+
+
+# ---- mid-size layer (every dimension a multiple of 512: the streaming schedule runs on it) -----
+
+@pytest.fixture(scope="module")
+def mid(torch_cuda):
+    w = synth.WORKLOADS["mid_b2"]
+    W = synth.layer_weights(w, 0)
+    return w, W, upload_weights(W)
+
+
+@pytest.mark.parametrize("B", [1, 2])
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_mid_parity(mid, B, schedule):
+    w, W, W_dev = mid
+    x = synth.tokens(w, batch=B)
+    layer = _make_layer(w, W_dev, max_batch=B, schedule=schedule)
+    _check_step(w, W, x, layer)
+    if schedule == "stream":
+        assert layer.kernels_per_step(B) == 4  # the streaming kernel ran (4 launches per step)
+
+
+@pytest.mark.parametrize("schedule", ["fused", "stream"])
+def test_mid_back_to_back_and_graph(mid, torch_cuda, schedule):
+    # consecutive steps of different tokens, eager and replayed from a CUDA graph, agree with a
+    # fresh handle's single step (the control block is clean between steps)
+    torch = torch_cuda
+    w, W, W_dev = mid
+    layer = _make_layer(w, W_dev, max_batch=2, schedule=schedule)
+    xs = [to_device(synth.tokens(w, step=s, batch=2)) for s in range(3)]
+    ref = [run_layer(_make_layer(w, W_dev, max_batch=2, schedule=schedule), synth.tokens(w, step=s, batch=2))[0]
+           for s in range(3)]
+    outs = [torch.empty_like(x) for x in xs]
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for x, o in zip(xs, outs):
+            layer.step(x, out=o, stream=stream)
+    torch.cuda.synchronize()
+    for o, r in zip(outs, ref):
+        assert np.array_equal(bf16_tensor_to_f32(o), r)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        for x, o in zip(xs, outs):
+            layer.step(x, out=o, stream=stream)
+    for o in outs:
+        o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    for o, r in zip(outs, ref):
+        assert np.array_equal(bf16_tensor_to_f32(o), r)
+    del g
 
 
 # ---- tiny layer -------------------------------------------------------------------------------
