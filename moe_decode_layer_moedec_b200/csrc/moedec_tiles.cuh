@@ -275,15 +275,28 @@ DEVI void tile_foreach(const float (&acc)[NT][4], int ntok, F fn) {
 // ---------------------------------------------------------------------------------------------
 // staging
 
+// Every staging helper issues a batch of its thread's loads before the first store, so that a call
+// costs about one L2 round trip per batch rather than one per element of its loop.
+constexpr int kStageBatch = 4;   // 16-byte loads (bf16 sources)
+constexpr int kStageBatchF = 2;  // 32-byte loads (fp32 sources)
+
 // bf16 tokens x[b][k0 .. k0+kc) -> xs[col b][0..kc) (bf16 layout), columns [ntok, ncols_pad) zero.
 DEVI void stage_bf16(uint16_t *xs, int pitch, const uint16_t *x, size_t ldx, int ntok, int ncols_pad, int k0, int kc,
                       int tid = threadIdx.x, int nthr = blockDim.x) {
-    const int units = kc / 8;
-    for (int i = tid; i < ncols_pad * units; i += nthr) {
-        const int col = i / units, u = i % units;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (col < ntok) v = *reinterpret_cast<const uint4 *>(x + (size_t)col * ldx + k0 + 8 * u);
-        *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * u) = v;
+    const int units = kc / 8, total = ncols_pad * units;
+    for (int i0 = tid; i0 < total; i0 += kStageBatch * nthr) {
+        uint4 v[kStageBatch];
+#pragma unroll
+        for (int j = 0; j < kStageBatch; ++j) {
+            const int i = i0 + j * nthr, col = i / units, u = i % units;
+            v[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < total && col < ntok) v[j] = *reinterpret_cast<const uint4 *>(x + (size_t)col * ldx + k0 + 8 * u);
+        }
+#pragma unroll
+        for (int j = 0; j < kStageBatch; ++j) {
+            const int i = i0 + j * nthr, col = i / units, u = i % units;
+            if (i < total) *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * u) = v[j];
+        }
     }
 }
 
@@ -292,24 +305,40 @@ DEVI void stage_bf16(uint16_t *xs, int pitch, const uint16_t *x, size_t ldx, int
 template <bool SPLIT, class RowOf>
 DEVI void stage_f16_from_f32(uint16_t *xs, int pitch, const float *src, size_t lds, int ntok, RowOf rowof,
                              const int *shift, int k0, int kc, int tid = threadIdx.x, int nthr = blockDim.x) {
-    const int units = kc / 8;
-    for (int i = tid; i < ntok * units; i += nthr) {
-        const int t = i / units, u = i % units;
-        const float *p = src + (size_t)rowof(t) * lds + k0 + 8 * u;
-        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(p));
-        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
-        const float sc = exp2i(-shift[t]);
-        const float v[8] = {v0.x * sc, v0.y * sc, v0.z * sc, v0.w * sc, v1.x * sc, v1.y * sc, v1.z * sc, v1.w * sc};
-        uint32_t hi[4], lo[4];
+    const int units = kc / 8, total = ntok * units;
+    for (int i0 = tid; i0 < total; i0 += kStageBatchF * nthr) {
+        float4 v0[kStageBatchF], v1[kStageBatchF];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            hi[j] = pack_f16x2(v[2 * j], v[2 * j + 1]);
-            if (SPLIT) lo[j] = pack_f16x2(v[2 * j] - f16_lo(hi[j]), v[2 * j + 1] - f16_hi(hi[j]));
+        for (int j = 0; j < kStageBatchF; ++j) {
+            const int i = i0 + j * nthr;
+            if (i < total) {
+                const int t = i / units, u = i % units;
+                const float *p = src + (size_t)rowof(t) * lds + k0 + 8 * u;
+                v0[j] = __ldcg(reinterpret_cast<const float4 *>(p));
+                v1[j] = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
+            }
         }
-        const int col = SPLIT ? 2 * t : t;
-        *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * swz(u)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        if (SPLIT)
-            *reinterpret_cast<uint4 *>(xs + (size_t)(col + 1) * pitch + 8 * swz(u)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+        for (int j = 0; j < kStageBatchF; ++j) {
+            const int i = i0 + j * nthr;
+            if (i < total) {
+                const int t = i / units, u = i % units;
+                const float sc = exp2i(-shift[t]);
+                const float v[8] = {v0[j].x * sc, v0[j].y * sc, v0[j].z * sc, v0[j].w * sc,
+                                    v1[j].x * sc, v1[j].y * sc, v1[j].z * sc, v1[j].w * sc};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    hi[q] = pack_f16x2(v[2 * q], v[2 * q + 1]);
+                    if (SPLIT) lo[q] = pack_f16x2(v[2 * q] - f16_lo(hi[q]), v[2 * q + 1] - f16_hi(hi[q]));
+                }
+                const int col = SPLIT ? 2 * t : t;
+                *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * swz(u)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                if (SPLIT)
+                    *reinterpret_cast<uint4 *>(xs + (size_t)(col + 1) * pitch + 8 * swz(u)) =
+                        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
     }
 }
 
@@ -317,37 +346,62 @@ DEVI void stage_f16_from_f32(uint16_t *xs, int pitch, const float *src, size_t l
 // column's maximum), fp16 layout, swizzled.
 DEVI void stage_f16_from_bf16(uint16_t *xs, int pitch, const uint16_t *x, size_t ldx, int ntok, const int *shift,
                               int k0, int kc, int tid = threadIdx.x, int nthr = blockDim.x) {
-    const int units = kc / 8;
-    for (int i = tid; i < ntok * units; i += nthr) {
-        const int t = i / units, u = i % units;
-        const uint4 v = *reinterpret_cast<const uint4 *>(x + (size_t)t * ldx + k0 + 8 * u);
-        const float sc = exp2i(-shift[t]);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
+    const int units = kc / 8, total = ntok * units;
+    for (int i0 = tid; i0 < total; i0 += kStageBatch * nthr) {
+        uint4 v[kStageBatch];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) o[j] = pack_f16x2(bf16_lo(w[j]) * sc, bf16_hi(w[j]) * sc);
-        *reinterpret_cast<uint4 *>(xs + (size_t)t * pitch + 8 * swz(u)) = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < kStageBatch; ++j) {
+            const int i = i0 + j * nthr, t = i / units, u = i % units;
+            v[j] = i < total ? *reinterpret_cast<const uint4 *>(x + (size_t)t * ldx + k0 + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < kStageBatch; ++j) {
+            const int i = i0 + j * nthr, t = i / units, u = i % units;
+            if (i < total) {
+                const float sc = exp2i(-shift[t]);
+                const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+                uint32_t o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) o[q] = pack_f16x2(bf16_lo(w[q]) * sc, bf16_hi(w[q]) * sc);
+                *reinterpret_cast<uint4 *>(xs + (size_t)t * pitch + 8 * swz(u)) = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+        }
     }
 }
 
 // fp32 vectors -> bf16 hi/lo column pairs (bf16 layout): column 2i = bf16(v), 2i+1 = bf16(v - hi).
 DEVI void stage_bf16split_from_f32(uint16_t *xs, int pitch, const float *src, size_t lds, int ntok, int k0, int kc,
                                    int tid = threadIdx.x, int nthr = blockDim.x) {
-    const int units = kc / 8;
-    for (int i = tid; i < ntok * units; i += nthr) {
-        const int t = i / units, u = i % units;
-        const float *p = src + (size_t)t * lds + k0 + 8 * u;
-        const float4 v0 = __ldcg(reinterpret_cast<const float4 *>(p));
-        const float4 v1 = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
-        const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        uint32_t hi[4], lo[4];
+    const int units = kc / 8, total = ntok * units;
+    for (int i0 = tid; i0 < total; i0 += kStageBatchF * nthr) {
+        float4 v0[kStageBatchF], v1[kStageBatchF];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            hi[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-            lo[j] = pack_bf16x2(v[2 * j] - bf16_lo(hi[j]), v[2 * j + 1] - bf16_hi(hi[j]));
+        for (int j = 0; j < kStageBatchF; ++j) {
+            const int i = i0 + j * nthr;
+            if (i < total) {
+                const int t = i / units, u = i % units;
+                const float *p = src + (size_t)t * lds + k0 + 8 * u;
+                v0[j] = __ldcg(reinterpret_cast<const float4 *>(p));
+                v1[j] = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
+            }
         }
-        *reinterpret_cast<uint4 *>(xs + (size_t)(2 * t) * pitch + 8 * u) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(xs + (size_t)(2 * t + 1) * pitch + 8 * u) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+        for (int j = 0; j < kStageBatchF; ++j) {
+            const int i = i0 + j * nthr;
+            if (i < total) {
+                const int t = i / units, u = i % units;
+                const float v[8] = {v0[j].x, v0[j].y, v0[j].z, v0[j].w, v1[j].x, v1[j].y, v1[j].z, v1[j].w};
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    hi[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+                    lo[q] = pack_bf16x2(v[2 * q] - bf16_lo(hi[q]), v[2 * q + 1] - bf16_hi(hi[q]));
+                }
+                *reinterpret_cast<uint4 *>(xs + (size_t)(2 * t) * pitch + 8 * u) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(xs + (size_t)(2 * t + 1) * pitch + 8 * u) =
+                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
     }
 }
 
