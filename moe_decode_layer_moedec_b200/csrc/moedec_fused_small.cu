@@ -12,16 +12,20 @@
 // full K) in shared memory once.  K splits of a tile are added by the warp that finishes last
 // (per-tile ticket), in split order; routed experts read the staged columns of their own tokens.
 //
-// Phases, in order (each CTA claims items from one queue at a time):
-//   router       8 rows x K/4            fp64 MMAs                    -> logits (per 8 rows)
+// The grid is split in two groups of CTAs.  The routed chain (most CTAs) runs, in order:
+//   router       8 rows x K/16           fp64 MMAs                    -> logits (per 8 rows)
 //   top-k        one CTA per token       waits: all logits            -> routing, buckets
-//   W_dn         16 rows x K/4           bf16 MMAs                    -> h rows, max |h|
-//   shared g/u   16 rows x K/4, g and u  MXFP4, x staged as fp16      -> sh_a rows, max |sh_a|
+//   W_dn         16 rows x K/16          bf16 MMAs (not the top-k CTAs) -> h rows, max |h|
 //   expert g/u   16 rows of one expert   waits: buckets, all of h     -> a rows, max |a|
-//   shared down  16 rows x K/2           waits: all of sh_a           -> sh rows
 //   expert down  16 rows of one expert   waits: its g/u rows          -> y rows; completing a token's
 //                                                                        16 rows combines them (ylat)
-//   W_up         16 rows x K/2           waits: ylat, sh              -> out rows
+//   W_up         16 rows x K/8           waits: ylat, sh              -> out rows
+// and the shared expert (an eighth of the grid) runs beside it:
+//   shared g/u   16 rows x K/8, g and u  MXFP4, x staged as fp16      -> sh_a rows, max |sh_a|
+//   shared down  16 rows x K/4           waits: all of sh_a           -> sh rows
+// Every phase entry is a CTA-wide barrier (the phase's activations are staged once per CTA), so
+// the shared parts, which nothing on the chain needs before W_up, must not sit between the
+// chain's phases: a CTA there would hold the chain until its slowest shared item ends.
 #include <algorithm>
 
 #include "moedec_items.cuh"
@@ -509,12 +513,22 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     const int n_sgu = a.d.n_shared ? Is / 16 * a.p.s_sgu : 0, n_sd = a.d.n_shared ? H / 16 * a.p.s_sd : 0;
     const int n_up = H / 16 * a.p.s_up;
 
+    // The shared expert runs on its own CTAs (the last G_sh of the grid), so that the routed
+    // chain (router -> top-k -> expert gate/up -> expert down -> W_up) never waits for the
+    // CTA-wide phase entries of the shared parts; a CTA's items come from its static range of
+    // its group's queues.
+    const int G = gridDim.x;
+    const int G_sh = a.d.n_shared ? max(1, G * kSmallSharedPer64 / 64) : 0, G_m = G - G_sh;
+    // the top-k CTAs (one per token) take no W_dn items: all of h is awaited right after routing
+    const int n_tk = B < G_m ? B : 0;
+    const int c_m = blockIdx.x, c_sh = (int)blockIdx.x - G_m;
+    const bool sh_cta = c_sh >= 0;
     // warps take items of queue qi until this CTA's range of it runs dry
-    auto warp_queue = [&](int qi, int n, auto body) {
+    auto warp_queue = [&](int qi, int n, int c, int g, auto body) {
         int ok = 1;
         for (;;) {
             int it = -1;
-            if (lane == 0) it = cta_take(claim, qi, n);
+            if (lane == 0) it = cta_take(claim, qi, n, c, g);
             it = __shfl_sync(0xffffffffu, it, 0);
             if (it < 0) break;
             if (!body(it)) {
@@ -530,20 +544,11 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     };
 
     cta_take_init(claim);
-    // router and W_dn read x as bf16
-    stage_x_bf16();
-    warp_queue(QS_ROUTER, n_rt, [&](int it) { w_router(a, it, xs); return true; });
-    stamp(1);
-    __syncthreads();
-    for (int it = blockIdx.x; alive && it < B; it += gridDim.x) alive = item_topk<true>(a, it, topk, (unsigned)((E + 7) / 8));
-    stamp(2);
-    if (alive) warp_queue(QS_DN, n_dn, [&](int it) { w_dn(a, it, xs); return true; });
-    stamp(3);
-    __syncthreads();
-    // shared gate/up read x as fp16 with a per-token exponent over all of H
-    if (alive && n_sgu) {
+    if (sh_cta) {
+        // ---- shared expert CTAs: gate/up on x, then down on sh_a (off the routed chain) ----
         if (threadIdx.x < B) s_amax[threadIdx.x] = 0u;
         __syncthreads();
+        // x as fp16 with a per-token exponent over all of H
         for (int i = threadIdx.x; i < B * (H / 8); i += blockDim.x) {
             const int t = i / (H / 8), u = i % (H / 8);
             const uint4 v = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * H + 8 * u);
@@ -558,56 +563,67 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         __syncthreads();
         stage_f16_from_bf16(xs, f16_pitch(H), a.x, H, B, s_shift, 0, H);
         __syncthreads();
-        warp_queue(QS_SGU, n_sgu, [&](int it) { w_sgu(a, it, xs, s_shift); return true; });
-    }
-    stamp(4);
-    // expert gate/up: routing and all of h final; stage h of every token (fp16 hi/lo)
-    if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
-    if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)(L / 16), &s_ok);
-    stamp(5);
-    if (alive) {
-        if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
-        __syncthreads();
-        stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, B, [](int t) { return t; }, s_shift, 0, L);
-        __syncthreads();
-        const int n = __ldcg(a.ws.n_active) * (I / 16) * a.p.s_egu;
-        warp_queue(QS_EGU, n, [&](int it) { w_egu(a, it, xs, s_shift); return true; });
-    }
-    stamp(6);
-    // shared down: all of sh_a final; stage it (fp16 hi/lo)
-    if (alive && n_sd) {
+        warp_queue(QS_SGU, n_sgu, c_sh, G_sh, [&](int it) { w_sgu(a, it, xs, s_shift); return true; });
+        stamp(4);
+        // shared down: all of sh_a final; stage it (fp16 hi/lo)
         alive = cta_wait_geq(a, ctl + CTL_SGU_DONE, (unsigned)(Is / 16), &s_ok);
         if (alive) {
             if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_shamax + threadIdx.x)));
             __syncthreads();
             stage_f16_from_f32<true>(xs, f16_pitch(Is), a.ws.sh_a, Is, B, [](int t) { return t; }, s_shift, 0, Is);
             __syncthreads();
-            warp_queue(QS_SD, n_sd, [&](int it) { w_sd(a, it, xs, s_shift); return true; });
+            warp_queue(QS_SD, n_sd, c_sh, G_sh, [&](int it) { w_sd(a, it, xs, s_shift); return true; });
         }
-    }
-    stamp(7);
-    // expert down (per-warp staging of the expert's entries)
-    if (alive) {
+        stamp(7);
+    } else {
+        // ---- routed chain CTAs ----
+        // router and W_dn read x as bf16
+        stage_x_bf16();
+        warp_queue(QS_ROUTER, n_rt, c_m, G_m, [&](int it) { w_router(a, it, xs); return true; });
+        stamp(1);
         __syncthreads();
-        const int n = __ldcg(a.ws.n_active) * (L / 16);
-        const int kc = kKChunk < I ? kKChunk : I;
-        uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(kc);
-        const int ok = warp_queue(QS_EDOWN, n, [&](int it) { return w_edown(a, it, ws); });
-        alive = __syncthreads_and(ok) != 0;
-    }
-    stamp(8);
-    // W_up: every ylat block final for every token, and all of sh; stage ylat (bf16 hi/lo)
-    if (alive) {
-        int ok = 1;
-        for (int blk = threadIdx.x; blk < L / 16; blk += blockDim.x)
-            ok &= wait_geq(a, ctl + a.p.ctl_ylat + blk, (unsigned)B) ? 1 : 0;
-        if (threadIdx.x == 0 && a.d.n_shared) ok &= wait_geq(a, ctl + CTL_SD_DONE, (unsigned)(H / 16)) ? 1 : 0;
-        __threadfence();
-        alive = __syncthreads_and(ok) != 0;
+        for (int it = c_m; alive && it < B; it += G_m) alive = item_topk<true>(a, it, topk, (unsigned)((E + 7) / 8), trace ? a.ws.trace + (size_t)(G + blockIdx.x) * kTraceStamps : nullptr);
+        stamp(2);
+        if (alive && c_m >= n_tk)
+            warp_queue(QS_DN, n_dn, c_m - n_tk, G_m - n_tk, [&](int it) { w_dn(a, it, xs); return true; });
+        stamp(3);
+        // expert gate/up: routing and all of h final; stage h of every token (fp16 hi/lo)
+        if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
+        stamp(11);
+        if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)(L / 16), &s_ok);
+        stamp(5);
         if (alive) {
-            stage_bf16split_from_f32(xs, bf16_pitch(L), a.ws.ylat, L, B, 0, L);
+            if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
             __syncthreads();
-            warp_queue(QS_UP, n_up, [&](int it) { w_up(a, it, xs); return true; });
+            stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, B, [](int t) { return t; }, s_shift, 0, L);
+            __syncthreads();
+            const int n = __ldcg(a.ws.n_active) * (I / 16) * a.p.s_egu;
+            warp_queue(QS_EGU, n, c_m, G_m, [&](int it) { w_egu(a, it, xs, s_shift); return true; });
+        }
+        stamp(6);
+        // expert down (per-warp staging of the expert's entries)
+        if (alive) {
+            __syncthreads();
+            const int n = __ldcg(a.ws.n_active) * (L / 16);
+            const int kc = kKChunk < I ? kKChunk : I;
+            uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(kc);
+            const int ok = warp_queue(QS_EDOWN, n, c_m, G_m, [&](int it) { return w_edown(a, it, ws); });
+            alive = __syncthreads_and(ok) != 0;
+        }
+        stamp(8);
+        // W_up: every ylat block final for every token, and all of sh; stage ylat (bf16 hi/lo)
+        if (alive) {
+            int ok = 1;
+            for (int blk = threadIdx.x; blk < L / 16; blk += blockDim.x)
+                ok &= wait_geq(a, ctl + a.p.ctl_ylat + blk, (unsigned)B) ? 1 : 0;
+            if (threadIdx.x == 0 && a.d.n_shared) ok &= wait_geq(a, ctl + CTL_SD_DONE, (unsigned)(H / 16)) ? 1 : 0;
+            __threadfence();
+            alive = __syncthreads_and(ok) != 0;
+            if (alive) {
+                stage_bf16split_from_f32(xs, bf16_pitch(L), a.ws.ylat, L, B, 0, L);
+                __syncthreads();
+                warp_queue(QS_UP, n_up, c_m, G_m, [&](int it) { w_up(a, it, xs); return true; });
+            }
         }
     }
     stamp(9);

@@ -18,6 +18,8 @@ constexpr int kKChunk = 512;       // activation staging chunk along K
 constexpr int kExpertTokGroup = 16;  // tokens of one expert per pass (two 8-column n-tiles)
 constexpr int kMaxCtasPerSm = 2;  // persistent kernels: CTAs per SM at most
 constexpr int kTraceRowsPerSm = 16;  // trace rows per SM (one per CTA, or one per warp)
+// 64ths of the small-batch grid that run the shared expert (the rest run the routed chain)
+constexpr int kSmallSharedPer64 = 8;
 // Largest K splits of the small-batch step's warp items (router, W_dn, shared gate/up, expert
 // gate/up, shared down, W_up); the plan takes the largest count <= these that divides K evenly.
 constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmallSplitEgu = 2, kSmallSplitSd = 4,

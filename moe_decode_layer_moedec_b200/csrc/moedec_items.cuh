@@ -103,14 +103,16 @@ DEVI void cta_take_init(CtaTake &t) {
     for (int i = threadIdx.x; i < 8; i += blockDim.x) t.next[i] = 0;
 }
 
-// next item of queue q (n items) of this CTA's range for the calling thread (one lane per
-// warp), or -1 once the range is used up
-DEVI int cta_take(CtaTake &t, int q, int n) {
-    const long long G = gridDim.x, c = blockIdx.x;
+// next item of queue q (n items) of the range [n c / G, n (c + 1) / G) that CTA c of a group of
+// G CTAs owns, for the calling thread (one lane per warp), or -1 once the range is used up
+DEVI int cta_take(CtaTake &t, int q, int n, int c, int G) {
     const int lo = (int)((long long)n * c / G), hi = (int)((long long)n * (c + 1) / G);
     const int k = atomicAdd(t.next + q, 1);
     return lo + k < hi ? lo + k : -1;
 }
+
+// the same over the whole grid
+DEVI int cta_take(CtaTake &t, int q, int n) { return cta_take(t, q, n, (int)blockIdx.x, (int)gridDim.x); }
 
 // ---------------------------------------------------------------------------------------------
 // router: one router row block x K range (fp64 MMAs); the block's last CTA publishes logits
@@ -180,32 +182,46 @@ struct TopkSmem {
 
 // FUSED: first wait until CTL_RT_DONE reaches rt_done (the schedule's count of router signals).
 template <bool FUSED>
-DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u) {
+DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u, unsigned long long *stamps = nullptr) {
     const int E = a.d.E, K = a.d.k, B = a.B;
     if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, rt_done, &t.ok)) return false;
+    // optional trace (global ns): logits complete, keys, K-th key, selection, routing written,
+    // expert masks, buckets written, buckets published
+    auto stamp = [&](int i) {
+        if (stamps && threadIdx.x == 0) stamps[i] = global_ns();
+    };
+    stamp(0);
     const int tid = threadIdx.x;
-    // thread tid owns experts 4*tid .. 4*tid+3 (index order follows thread order)
+    // thread tid owns experts 4*tid .. 4*tid+3 (index order follows thread order); all four
+    // logits are loaded before the first score is computed (one memory round trip, not four)
     unsigned key[4];
     bool valid[4];
+    float lg[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const int e = 4 * tid + i;
-        valid[i] = e < E;
-        key[i] = 0u;
-        if (valid[i]) {
-            const float lg = __ldcg(a.ws.logits + (size_t)b * E + e);
-            const float sc = (float)(1.0 / (1.0 + exp(-(double)lg)));
-            key[i] = sc >= 0.0f ? __float_as_uint(sc) : 0u;  // non-negative fp32 orders like its bits
-        }
+        valid[i] = 4 * tid + i < E;
+        lg[i] = valid[i] ? __ldcg(a.ws.logits + (size_t)b * E + 4 * tid + i) : 0.0f;
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float sc = (float)(1.0 / (1.0 + exp(-(double)lg[i])));
+        key[i] = valid[i] && sc >= 0.0f ? __float_as_uint(sc) : 0u;  // non-negative fp32 orders like its bits
+    }
+    stamp(1);
     // radix select of the K-th largest key, 8 bits at a time from the top
     unsigned prefix = 0u, mask = 0u, want = (unsigned)K;
     for (int shift = 24; shift >= 0; shift -= 8) {
         if (tid < 256) t.hist[tid] = 0u;
         __syncthreads();
+        // warp-aggregated counts: sigmoid scores share their top bits, so most keys of a pass
+        // fall into one or two bins and per-key shared atomics would serialise on them
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (valid[i] && (key[i] & mask) == prefix) atomicAdd(&t.hist[(key[i] >> shift) & 255u], 1u);
+        for (int i = 0; i < 4; ++i) {
+            const bool in = valid[i] && (key[i] & mask) == prefix;
+            const unsigned bin = in ? (key[i] >> shift) & 255u : 0xffffffffu;
+            const unsigned peers = __match_any_sync(0xffffffffu, bin);
+            if (in && __ffs(peers) - 1 == (tid & 31)) atomicAdd(&t.hist[bin], (unsigned)__popc(peers));
+        }
         __syncthreads();
         if (tid < 32) {
             // lane l holds bins 8l..8l+7; find the bin d holding the want-th largest key
@@ -240,6 +256,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
         mask |= 255u << shift;
         want = t.want;
     }
+    stamp(2);
     const unsigned T = prefix;  // the K-th largest key; `want` keys equal to T are taken
     int n_eq = 0;
 #pragma unroll
@@ -264,6 +281,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
             ++pos;
         }
     __syncthreads();
+    stamp(3);
     if (tid < K) {
         const unsigned mk = t.key[tid];
         const int me = t.e[tid];
@@ -281,17 +299,21 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
             a.ws.wts[(size_t)b * K + r] = t.rank_s[r] / S;
         }
     }
-    // the last token's CTA groups the B*K selections by expert
-    if (!cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
+    stamp(4);
+    // the last token's CTA groups the B*K selections by expert (with one token, this CTA: its
+    // selections are still in shared memory)
+    if (B > 1 && !cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
+    auto sel_e = [&](int i) { return B > 1 ? __ldcg(a.ws.idx + i) : t.rank_e[i]; };
     for (int i = tid; i < E; i += blockDim.x) t.mask[i] = 0ull;
     __syncthreads();
     for (int i = tid; i < B * K; i += blockDim.x) {
-        const int ex = __ldcg(a.ws.idx + i);
+        const int ex = sel_e(i);
         if (ex >= 0 && ex < E) atomicOr(&t.mask[ex], 1ull << (i / K));
         else atomicOr(a.ws.err, kErrBucket);
         a.ws.a_amax[i] = 0u;
     }
     __syncthreads();
+    stamp(5);
     int cnt[4], n_act_t = 0, n_ent_t = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -318,11 +340,13 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
     if (tid == 0) *a.ws.n_active = n_act;
     __syncthreads();
     for (int i = tid; i < B * K; i += blockDim.x) {
-        const int ex = __ldcg(a.ws.idx + i), tb = i / K;
+        const int ex = sel_e(i), tb = i / K;
         if (ex < 0 || ex >= E) continue;
         a.ws.entries[t.off[ex] + __popcll(t.mask[ex] & ((1ull << tb) - 1ull))] = i;
     }
+    stamp(6);
     if (FUSED) cta_signal_add(a.ws.ctl + CTL_ROUTE_READY, 1u);
+    stamp(7);
     return true;
 }
 
