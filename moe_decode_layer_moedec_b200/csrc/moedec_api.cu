@@ -87,6 +87,7 @@ void layout(moedec_handle *h, char *base) {
     Work &w = h->ws;
     w.rt_part = c.take<double>((size_t)std::max(p.rt.splits, kSmallSplitRt) * B * d.E);
     w.logits = c.take<float>(B * d.E);
+    w.rt_acc = c.take<double>(std::min<size_t>(B, kSmallMaxBatch) * d.E);
     w.dn_part = c.take<float>((size_t)std::max(p.dn.splits, kSmallSplitDn) * B * d.L);
     w.h = c.take<float>(B * d.L);
     w.h_shift = c.take<int>(B);
@@ -194,6 +195,8 @@ int read_device_error(moedec_handle *h, cudaStream_t s) {
     if (e != cudaSuccess) return record_cuda(h, e);
     if (v == 0) return MOEDEC_OK;
     cudaMemsetAsync(h->ws.err, 0, sizeof(unsigned), s);
+    // an aborted small-batch step may have left router sums behind: they are zero at rest
+    cudaMemsetAsync(h->ws.rt_acc, 0, std::min<size_t>(h->d.max_batch, kSmallMaxBatch) * h->d.E * sizeof(double), s);
     cudaStreamSynchronize(s);
     return (v & kErrTimeout) ? MOEDEC_ERR_TIMEOUT : MOEDEC_ERR_DEVICE;
 }

@@ -17,12 +17,12 @@
 //   top-k        one CTA per token       waits: all logits            -> routing, buckets
 //   W_dn         16 rows x K/16          bf16 MMAs (not the top-k CTAs) -> h rows, max |h|
 //   expert g/u   16 rows of one expert   waits: buckets, all of h     -> a rows, max |a|
-//   expert down  16 rows of one expert   waits: its g/u rows          -> y rows; completing a token's
-//                                                                        16 rows combines them (ylat)
-//   W_up         16 rows x K/8           waits: ylat, sh              -> out rows
+//   expert down  16 rows of one expert   waits: its g/u rows          -> w * y rows added into ylat
+//                                                                        (fp32 reductions)
+//   W_up         16 rows x K/4           waits: ylat, sh              -> out rows
 // and the shared expert (an eighth of the grid) runs beside it:
 //   shared g/u   16 rows x K/8, g and u  MXFP4, x staged as fp16      -> sh_a rows, max |sh_a|
-//   shared down  16 rows x K/4           waits: all of sh_a           -> sh rows
+//   shared down  16 rows x K             waits: all of sh_a           -> sh rows
 // Every phase entry is a CTA-wide barrier (the phase's activations are staged once per CTA), so
 // the shared parts, which nothing on the chain needs before W_up, must not sit between the
 // chain's phases: a CTA there would hold the chain until its slowest shared item ends.
@@ -167,7 +167,7 @@ DEVI bool warp_ticket_last(unsigned *counter, unsigned expected) {
 
 // router: 8 rows x K/s_rt (fp64 m8n8k4; slot q of step s of chunk c holds k = 32c + 8q + s)
 DEVI void w_router(const StepArgs &a, int item, const uint16_t *xs) {
-    const int E = a.d.E, H = a.d.H, B = a.B, maxB = a.d.max_batch;
+    const int E = a.d.E, H = a.d.H, B = a.B;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int rg = item / a.p.s_rt, ks = item % a.p.s_rt;
     const int row = rg * 8 + g;
@@ -203,16 +203,12 @@ DEVI void w_router(const StepArgs &a, int item, const uint16_t *xs) {
     }
     c0 += d0;
     c1 += d1;
+    // the K splits of a logit meet in fp64 reductions (the top-k rounds the sum to fp32 once
+    // every router item has signalled, and clears the accumulator for the next step)
     if (row_ok) {
-        if (2 * q < B) a.ws.rt_part[((size_t)ks * maxB + 2 * q) * E + row] = c0;
-        if (2 * q + 1 < B) a.ws.rt_part[((size_t)ks * maxB + 2 * q + 1) * E + row] = c1;
+        if (2 * q < B) atomicAdd(a.ws.rt_acc + (size_t)(2 * q) * E + row, c0);
+        if (2 * q + 1 < B) atomicAdd(a.ws.rt_acc + (size_t)(2 * q + 1) * E + row, c1);
     }
-    if (!warp_ticket_last(a.ws.ctl + a.p.ctl_tk + rg, a.p.s_rt)) return;
-    if (row_ok)
-        for (int j = 0; j < 2; ++j) {
-            const int b = 2 * q + j;
-            if (b < B) a.ws.logits[(size_t)b * E + row] = (float)sum_splits(a.ws.rt_part + (size_t)b * E + row, (size_t)maxB * E, a.p.s_rt);
-        }
     if (!(a.flags & kFlagTestStall)) warp_signal_add(a.ws.ctl + CTL_RT_DONE, 1u);
 }
 
@@ -292,29 +288,53 @@ DEVI void w_sgu(const StepArgs &a, int item, const uint16_t *xs16, const int *xs
     warp_signal_add(a.ws.ctl + CTL_SGU_DONE, 1u);
 }
 
+// The step's expert buckets, copied into shared memory once per CTA when the routing is out
+// (the routed items read them from there instead of paying a global round trip each).
+struct RouteSmem {
+    int n_active;
+    int e[kSmallMaxBatch * kMaxTopK], cnt[kSmallMaxBatch * kMaxTopK], off[kSmallMaxBatch * kMaxTopK];
+    int ent[kSmallMaxBatch * kMaxTopK];
+    float w[kSmallMaxBatch * kMaxTopK];  // routing weight of each entry
+};
+
+// all threads; every load is issued before the first use (one round trip); a barrier must follow
+DEVI void cta_load_routing(const StepArgs &a, RouteSmem &r) {
+    const int n = a.B * a.d.k;  // >= n_active
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int e = __ldcg(a.ws.active_e + i), c = __ldcg(a.ws.active_cnt + i), o = __ldcg(a.ws.active_off + i);
+        const int en = __ldcg(a.ws.entries + i);
+        const float w = __ldcg(a.ws.wts + i);
+        r.e[i] = e;
+        r.cnt[i] = c;
+        r.off[i] = o;
+        r.ent[i] = en;
+        r.w[i] = w;
+    }
+    if (threadIdx.x == 0) r.n_active = __ldcg(a.ws.n_active);
+}
+
 // this warp's entries of active expert slot j: ent[i] for i < cnt (lane i holds entry i)
 struct Entries {
     int e, cnt, my_ent;
 };
 
-DEVI Entries warp_entries(const StepArgs &a, int j) {
+DEVI Entries warp_entries(const RouteSmem &rt, int j) {
     const int lane = threadIdx.x & 31;
     Entries r;
-    r.e = __ldcg(a.ws.active_e + j);
-    r.cnt = __ldcg(a.ws.active_cnt + j);
-    const int off = __ldcg(a.ws.active_off + j);
-    r.my_ent = lane < r.cnt ? __ldcg(a.ws.entries + off + lane) : 0;
+    r.e = rt.e[j];
+    r.cnt = rt.cnt[j];
+    r.my_ent = lane < r.cnt ? rt.ent[rt.off[j] + lane] : 0;
     return r;
 }
 
 // expert gate/up: 16 rows of active expert slot j x K/s_egu; h of all tokens staged as fp16
 // hi/lo columns (2b, 2b+1) with a per-token exponent; the last split applies silu(gate) * up
-DEVI void w_egu(const StepArgs &a, int item, const uint16_t *hs, const int *hshift) {
+DEVI void w_egu(const StepArgs &a, const RouteSmem &rt, int item, const uint16_t *hs, const int *hshift) {
     const int L = a.d.L, I = a.d.I, K = a.d.k, S = a.p.s_egu;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int tiles = I / 16, ks = item % S, jt = item / S, j = jt / tiles, row0 = (jt % tiles) * 16;
     const int KW = L / S, k0 = ks * KW;
-    const Entries en = warp_entries(a, j);
+    const Entries en = warp_entries(rt, j);
     // MMA column g: entry g/2, hi (g even) or lo (g odd) part of its token's staged h
     const int ent_g = __shfl_sync(0xffffffffu, en.my_ent, (g >> 1) & 31);
     const int col = (g >> 1) < en.cnt ? 2 * (ent_g / K) + (g & 1) : -1;
@@ -366,6 +386,15 @@ DEVI void w_sd(const StepArgs &a, int item, const uint16_t *ss, const int *sshif
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, dummy[4];
     s_fp4<5, false>(a.w.sh_down_q, a.w.sh_down_s, nullptr, nullptr, Is / 2, Is / 32, row0, k0, KW / 128, ss,
                     f16_pitch(Is), k0, g < 2 * B ? g : -1, acc, dummy);
+    if (a.p.s_sd == 1) {  // the item covers all of K: the tile is final here (no partials, no ticket)
+        if (q < B) {
+            const float sc = exp2i(sshift[q]);
+            a.ws.sh[(size_t)q * H + row0 + g] = (acc[0] + acc[1]) * sc;
+            a.ws.sh[(size_t)q * H + row0 + g + 8] = (acc[2] + acc[3]) * sc;
+        }
+        warp_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
+        return;
+    }
     float *part = a.ws.sd_part + (size_t)ks * maxB * H;
     if (q < B) {
         part[(size_t)q * H + row0 + g] = acc[0] + acc[1];
@@ -383,34 +412,16 @@ DEVI void w_sd(const StepArgs &a, int item, const uint16_t *ss, const int *sshif
     warp_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
 }
 
-// ylat[b][row0 + i], i < 16, combined by one warp: lane (i, half) adds the weighted slots of its
-// parity in slot order, then the two halves are added
-DEVI void warp_combine_rows(const StepArgs &a, int b, int row0) {
-    const int L = a.d.L, K = a.d.k, lane = threadIdx.x & 31, l = row0 + (lane & 15), h = lane >> 4;
-    float s = 0.0f;
-    for (int r0 = h; r0 < K; r0 += 16) {
-        float wv[8], yv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int r = r0 + 2 * j;
-            wv[j] = r < K ? __ldcg(a.ws.wts + (size_t)b * K + r) : 0.0f;
-            yv[j] = r < K ? __ldcg(a.ws.y + ((size_t)b * K + r) * L + l) : 0.0f;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s += wv[j] * yv[j];
-    }
-    s += __shfl_xor_sync(0xffffffffu, s, 16);
-    if (lane < 16) a.ws.ylat[(size_t)b * L + l] = s;
-}
-
 // expert down: 16 rows of L of active expert slot j, full K; a staged per warp (fp16 hi/lo of
-// the expert's entries, 512 k at a time); the warp that completes a token's 16 rows combines them
-DEVI bool w_edown(const StepArgs &a, int item, uint16_t *ws) {
+// the expert's entries, 512 k at a time).  The combine is folded in: each entry's rows, times
+// its routing weight, are added into ylat (fp32 reductions, so the order of the K slots of a
+// token is not fixed), and the tile's ylat count grows by the number of entries.
+DEVI bool w_edown(const StepArgs &a, const RouteSmem &rt, int item, uint16_t *ws) {
     const int L = a.d.L, I = a.d.I, K = a.d.k;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int tiles = L / 16, j = item / tiles, tile = item % tiles, row0 = tile * 16;
     if (!warp_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(I / 16))) return false;
-    const Entries en = warp_entries(a, j);
+    const Entries en = warp_entries(rt, j);
     __shared__ int s_ent[kWarps][kMaxTopK], s_shift[kWarps][kMaxTopK];  // cnt <= B <= 4
     const int warp = threadIdx.x >> 5;
     __syncwarp();
@@ -431,25 +442,13 @@ DEVI bool w_edown(const StepArgs &a, int item, uint16_t *ws) {
                         f16_pitch(kc), 0, g < 2 * en.cnt ? g : -1, acc, dummy);
     }
     if (q < en.cnt) {
-        const float sc = exp2i(s_shift[warp][q]);
-        float *dst = a.ws.y + (size_t)s_ent[warp][q] * L + row0;
-        dst[g] = (acc[0] + acc[1]) * sc;
-        dst[g + 8] = (acc[2] + acc[3]) * sc;
+        const int ent = s_ent[warp][q];
+        const float ws_ = rt.w[ent] * exp2i(s_shift[warp][q]);
+        float *dst = a.ws.ylat + (size_t)(ent / K) * L + row0;
+        atomicAdd(dst + g, (acc[0] + acc[1]) * ws_);
+        atomicAdd(dst + g + 8, (acc[2] + acc[3]) * ws_);
     }
-    __threadfence();
-    __syncwarp();
-    bool mine = false;
-    if (lane < en.cnt)
-        mine = atomicAdd(a.ws.ctl + a.p.ctl_comb + (size_t)(en.my_ent / K) * (L / 16) + tile, 1u) == (unsigned)(K - 1);
-    unsigned todo = __ballot_sync(0xffffffffu, mine);
-    if (todo) __threadfence();  // acquire: the other slots' y rows of this block are visible
-    while (todo) {
-        const int tl = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const int b = s_ent[warp][tl] / K;
-        warp_combine_rows(a, b, row0);
-        warp_signal_add(a.ws.ctl + a.p.ctl_ylat + tile, 1u);
-    }
+    warp_signal_add(a.ws.ctl + a.p.ctl_ylat + tile, (unsigned)en.cnt);
     return true;
 }
 
@@ -499,6 +498,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     __shared__ int s_shift[kMaxBatch], s_ok;
     __shared__ unsigned s_amax[kMaxBatch];
     __shared__ CtaTake claim;
+    __shared__ RouteSmem route;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     unsigned *ctl = a.ws.ctl;
     const int H = a.d.H, L = a.d.L, I = a.d.I, Is = a.d.Is, B = a.B, E = a.d.E;
@@ -582,7 +582,10 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         warp_queue(QS_ROUTER, n_rt, c_m, G_m, [&](int it) { w_router(a, it, xs); return true; });
         stamp(1);
         __syncthreads();
-        for (int it = c_m; alive && it < B; it += G_m) alive = item_topk<true>(a, it, topk, (unsigned)((E + 7) / 8), trace ? a.ws.trace + (size_t)(G + blockIdx.x) * kTraceStamps : nullptr);
+        for (int it = c_m; alive && it < B; it += G_m)
+            alive = item_topk<true>(a, it, topk, (unsigned)n_rt,
+                                    trace ? a.ws.trace + (size_t)(G + blockIdx.x) * kTraceStamps : nullptr, a.ws.ylat,
+                                    a.ws.rt_acc);
         stamp(2);
         if (alive && c_m >= n_tk)
             warp_queue(QS_DN, n_dn, c_m - n_tk, G_m - n_tk, [&](int it) { w_dn(a, it, xs); return true; });
@@ -594,28 +597,30 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         stamp(5);
         if (alive) {
             if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
+            cta_load_routing(a, route);
             __syncthreads();
             stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, B, [](int t) { return t; }, s_shift, 0, L);
             __syncthreads();
-            const int n = __ldcg(a.ws.n_active) * (I / 16) * a.p.s_egu;
-            warp_queue(QS_EGU, n, c_m, G_m, [&](int it) { w_egu(a, it, xs, s_shift); return true; });
+            const int n = route.n_active * (I / 16) * a.p.s_egu;
+            warp_queue(QS_EGU, n, c_m, G_m, [&](int it) { w_egu(a, route, it, xs, s_shift); return true; });
         }
         stamp(6);
         // expert down (per-warp staging of the expert's entries)
         if (alive) {
             __syncthreads();
-            const int n = __ldcg(a.ws.n_active) * (L / 16);
+            const int n = route.n_active * (L / 16);
             const int kc = kKChunk < I ? kKChunk : I;
             uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(kc);
-            const int ok = warp_queue(QS_EDOWN, n, c_m, G_m, [&](int it) { return w_edown(a, it, ws); });
+            const int ok = warp_queue(QS_EDOWN, n, c_m, G_m, [&](int it) { return w_edown(a, route, it, ws); });
             alive = __syncthreads_and(ok) != 0;
         }
         stamp(8);
-        // W_up: every ylat block final for every token, and all of sh; stage ylat (bf16 hi/lo)
+        // W_up: every ylat block complete (all B*k entries added), and all of sh; stage ylat
+        // (bf16 hi/lo)
         if (alive) {
             int ok = 1;
             for (int blk = threadIdx.x; blk < L / 16; blk += blockDim.x)
-                ok &= wait_geq(a, ctl + a.p.ctl_ylat + blk, (unsigned)B) ? 1 : 0;
+                ok &= wait_geq(a, ctl + a.p.ctl_ylat + blk, (unsigned)(B * a.d.k)) ? 1 : 0;
             if (threadIdx.x == 0 && a.d.n_shared) ok &= wait_geq(a, ctl + CTL_SD_DONE, (unsigned)(H / 16)) ? 1 : 0;
             __threadfence();
             alive = __syncthreads_and(ok) != 0;

@@ -22,8 +22,8 @@ constexpr int kTraceRowsPerSm = 16;  // trace rows per SM (one per CTA, or one p
 constexpr int kSmallSharedPer64 = 8;
 // Largest K splits of the small-batch step's warp items (router, W_dn, shared gate/up, expert
 // gate/up, shared down, W_up); the plan takes the largest count <= these that divides K evenly.
-constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmallSplitEgu = 2, kSmallSplitSd = 4,
-              kSmallSplitUp = 8;
+constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmallSplitEgu = 2, kSmallSplitSd = 1,
+              kSmallSplitUp = 4;
 constexpr int kSmallMaxBatch = 4;  // tokens of the small-batch step
 constexpr int kTraceStamps = 16;     // MOEDEC_TRACE_STAMPS
 
@@ -93,6 +93,7 @@ enum CtlWord {
 // Device workspace of one handle (all sized for max_batch).
 struct Work {
     double *rt_part;    // [rt.splits][maxB][E]   router partial sums (fp64)
+    double *rt_acc;     // [min(maxB, 4)][E] small-batch router sums (fp64 reductions; zero at rest)
     float *logits;      // [maxB][E]
     float *dn_part;     // [dn.splits][maxB][L]
     float *h;           // [maxB][L]

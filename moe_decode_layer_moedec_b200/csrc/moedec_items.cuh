@@ -180,13 +180,36 @@ struct TopkSmem {
     int off[kMaxExperts];
 };
 
+// Warp maximum of the lanes' N packed words; the lane holding it clears it (words are unique
+// apart from 0, which only ever ties with another 0).  Returns the maximum to every lane.  Two
+// warp reductions (high halves, then the low halves of the lanes that hold the highest high
+// half) instead of a shuffle tree: the rounds of a selection are a dependent chain.
+template <int N>
+DEVI unsigned long long warp_take_best(unsigned long long (&w)[N]) {
+    unsigned long long m = w[0];
+#pragma unroll
+    for (int i = 1; i < N; ++i) m = w[i] > m ? w[i] : m;
+    const unsigned hi = __reduce_max_sync(0xffffffffu, (unsigned)(m >> 32));
+    const unsigned lo = __reduce_max_sync(0xffffffffu, (unsigned)(m >> 32) == hi ? (unsigned)m : 0u);
+    const unsigned long long best = ((unsigned long long)hi << 32) | lo;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+        if (w[i] == best) w[i] = 0ull;
+    return best;
+}
+
 // FUSED: first wait until CTL_RT_DONE reaches rt_done (the schedule's count of router signals).
+// zero_rows: when given, the token's row of it ([B][L]) is zeroed before the routing is
+// published (the small-batch step adds the expert outputs into ylat).
+// acc64: when given, the logits are the fp64 sums there ([B][E]): they are rounded to fp32 into
+// ws.logits and the accumulator is cleared; otherwise ws.logits already holds them.
 template <bool FUSED>
-DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u, unsigned long long *stamps = nullptr) {
+DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u, unsigned long long *stamps = nullptr,
+                    float *zero_rows = nullptr, double *acc64 = nullptr) {
     const int E = a.d.E, K = a.d.k, B = a.B;
     if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, rt_done, &t.ok)) return false;
-    // optional trace (global ns): logits complete, keys, K-th key, selection, routing written,
-    // expert masks, buckets written, buckets published
+    // optional trace (global ns): logits complete, keys, warp candidates, ranked, routing
+    // written, expert masks, buckets written, buckets published
     auto stamp = [&](int i) {
         if (stamps && threadIdx.x == 0) stamps[i] = global_ns();
     };
@@ -197,10 +220,27 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
     unsigned key[4];
     bool valid[4];
     float lg[4];
+    if (acc64) {
+        double v[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        valid[i] = 4 * tid + i < E;
-        lg[i] = valid[i] ? __ldcg(a.ws.logits + (size_t)b * E + 4 * tid + i) : 0.0f;
+        for (int i = 0; i < 4; ++i) {
+            valid[i] = 4 * tid + i < E;
+            v[i] = valid[i] ? __ldcg(acc64 + (size_t)b * E + 4 * tid + i) : 0.0;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            lg[i] = (float)v[i];
+            if (valid[i]) {
+                a.ws.logits[(size_t)b * E + 4 * tid + i] = lg[i];
+                acc64[(size_t)b * E + 4 * tid + i] = 0.0;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            valid[i] = 4 * tid + i < E;
+            lg[i] = valid[i] ? __ldcg(a.ws.logits + (size_t)b * E + 4 * tid + i) : 0.0f;
+        }
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -208,102 +248,72 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
         key[i] = valid[i] && sc >= 0.0f ? __float_as_uint(sc) : 0u;  // non-negative fp32 orders like its bits
     }
     stamp(1);
-    // radix select of the K-th largest key, 8 bits at a time from the top
-    unsigned prefix = 0u, mask = 0u, want = (unsigned)K;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        if (tid < 256) t.hist[tid] = 0u;
-        __syncthreads();
-        // warp-aggregated counts: sigmoid scores share their top bits, so most keys of a pass
-        // fall into one or two bins and per-key shared atomics would serialise on them
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const bool in = valid[i] && (key[i] & mask) == prefix;
-            const unsigned bin = in ? (key[i] >> shift) & 255u : 0xffffffffu;
-            const unsigned peers = __match_any_sync(0xffffffffu, bin);
-            if (in && __ffs(peers) - 1 == (tid & 31)) atomicAdd(&t.hist[bin], (unsigned)__popc(peers));
-        }
-        __syncthreads();
-        if (tid < 32) {
-            // lane l holds bins 8l..8l+7; find the bin d holding the want-th largest key
-            unsigned c[8], tot = 0u;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                c[j] = t.hist[8 * tid + j];
-                tot += c[j];
-            }
-            unsigned sfx = tot;  // inclusive suffix sum over lanes tid..31
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const unsigned v = __shfl_down_sync(0xffffffffu, sfx, o);
-                if (tid + o < 32) sfx += v;
-            }
-            const unsigned above = sfx - tot;  // keys in the bins of higher lanes (higher digits)
-            if (above < want && want <= above + tot) {
-                unsigned acc = above;
-#pragma unroll
-                for (int j = 7; j >= 0; --j) {
-                    if (acc + c[j] >= want) {
-                        t.digit = 8u * tid + j;
-                        t.want = want - acc;
-                        break;
-                    }
-                    acc += c[j];
-                }
-            }
-        }
-        __syncthreads();
-        prefix |= t.digit << shift;
-        mask |= 255u << shift;
-        want = t.want;
-    }
-    stamp(2);
-    const unsigned T = prefix;  // the K-th largest key; `want` keys equal to T are taken
-    int n_eq = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) n_eq += (valid[i] && key[i] == T) ? 1 : 0;
-    int tot;
-    int eq_rank = block_exclusive_scan(n_eq, t.warp, &tot);
-    bool sel[4];
-    int n_sel = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool eq = valid[i] && key[i] == T;
-        sel[i] = (valid[i] && key[i] > T) || (eq && eq_rank < (int)want);
-        eq_rank += eq ? 1 : 0;
-        n_sel += sel[i] ? 1 : 0;
-    }
-    int pos = block_exclusive_scan(n_sel, t.warp, &tot);
+    // Selection on packed words (score bits << 32 | ~expert): a larger word ranks first (higher
+    // score, then lower expert index), 0 is no expert.  Each warp takes its K best, best first, by
+    // K rounds of a warp maximum whose holder drops the word; warp 0 then ranks the warps'
+    // candidates the same way and so emits the top K in rank order.
+    const int lane = tid & 31, warp = tid >> 5, nw = (int)(blockDim.x >> 5);
+    unsigned long long P[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        if (sel[i]) {
-            t.key[pos] = key[i];
-            t.e[pos] = 4 * tid + i;
-            ++pos;
-        }
-    __syncthreads();
-    stamp(3);
-    if (tid < K) {
-        const unsigned mk = t.key[tid];
-        const int me = t.e[tid];
-        int rank = 0;
-        for (int j = 0; j < K; ++j) rank += (t.key[j] > mk) || (t.key[j] == mk && t.e[j] < me);
-        t.rank_e[rank] = me;
-        t.rank_s[rank] = __uint_as_float(mk);
+        P[i] = valid[i] ? ((unsigned long long)key[i] << 32) | (0xffffffffu - (unsigned)(4 * tid + i)) : 0ull;
+    unsigned long long *cand = t.mask;  // nw * K candidates; the expert masks are built after
+    for (int r = 0; r < K; ++r) {
+        const unsigned long long m = warp_take_best(P);
+        if (lane == 0) cand[warp * K + r] = m;
     }
     __syncthreads();
-    if (tid == 0) {
-        float S = 0.0f;
-        for (int r = 0; r < K; ++r) S += t.rank_s[r];
+    stamp(2);
+    if (warp == 0) {
+        unsigned long long C[8];  // nw * K <= 8 * 32 candidates
+#pragma unroll
+        for (int i = 0; i < 8; ++i) C[i] = lane + 32 * i < nw * K ? cand[lane + 32 * i] : 0ull;
+        float S = 0.0f;  // sum of the selected scores in rank order
         for (int r = 0; r < K; ++r) {
-            a.ws.idx[(size_t)b * K + r] = t.rank_e[r];
-            a.ws.wts[(size_t)b * K + r] = t.rank_s[r] / S;
+            const unsigned long long m = warp_take_best(C);
+            if (lane == 0) {
+                const float sc = __uint_as_float((unsigned)(m >> 32));
+                t.rank_e[r] = (int)(0xffffffffu - (unsigned)(m & 0xffffffffull));
+                t.rank_s[r] = sc;
+                S += sc;
+            }
+        }
+        S = __shfl_sync(0xffffffffu, S, 0);
+        __syncwarp();
+        stamp(3);
+        if (lane < K) {
+            a.ws.idx[(size_t)b * K + lane] = t.rank_e[lane];
+            a.ws.wts[(size_t)b * K + lane] = t.rank_s[lane] / S;
         }
     }
+    if (zero_rows)
+        for (int i = tid; i < a.d.L / 4; i += blockDim.x)
+            reinterpret_cast<float4 *>(zero_rows + (size_t)b * a.d.L)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
     stamp(4);
-    // the last token's CTA groups the B*K selections by expert (with one token, this CTA: its
-    // selections are still in shared memory)
-    if (B > 1 && !cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
-    auto sel_e = [&](int i) { return B > 1 ? __ldcg(a.ws.idx + i) : t.rank_e[i]; };
+    if (B == 1) {
+        // one token: its K distinct experts are the buckets (one entry each), in expert order
+        if (warp == 0) {
+            const int e = lane < K ? t.rank_e[lane] : 0x7fffffff;
+            int pos = 0;
+            for (int j = 0; j < K; ++j) pos += __shfl_sync(0xffffffffu, e, j) < e ? 1 : 0;
+            if (lane < K) {
+                a.ws.active_e[pos] = e;
+                a.ws.active_cnt[pos] = 1;
+                a.ws.active_off[pos] = pos;
+                a.ws.entries[pos] = lane;
+                a.ws.a_amax[lane] = 0u;
+            }
+            if (lane == 0) *a.ws.n_active = K;
+        }
+        stamp(6);
+        if (FUSED) cta_signal_add(a.ws.ctl + CTL_ROUTE_READY, 1u);
+        stamp(7);
+        return true;
+    }
+    // the last token's CTA groups the B*K selections by expert
+    if (!cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
+    auto sel_e = [&](int i) { return __ldcg(a.ws.idx + i); };
     for (int i = tid; i < E; i += blockDim.x) t.mask[i] = 0ull;
     __syncthreads();
     for (int i = tid; i < B * K; i += blockDim.x) {

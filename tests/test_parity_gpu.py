@@ -94,7 +94,7 @@ def test_mid_back_to_back_and_graph(mid, torch_cuda, schedule):
             layer.step(x, out=o, stream=stream)
     torch.cuda.synchronize()
     for o, r in zip(outs, ref):
-        assert np.array_equal(bf16_tensor_to_f32(o), r)
+        _assert_replays(bf16_tensor_to_f32(o), r, schedule)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
         for x, o in zip(xs, outs):
@@ -104,8 +104,20 @@ def test_mid_back_to_back_and_graph(mid, torch_cuda, schedule):
     g.replay()
     torch.cuda.synchronize()
     for o, r in zip(outs, ref):
-        assert np.array_equal(bf16_tensor_to_f32(o), r)
+        _assert_replays(bf16_tensor_to_f32(o), r, schedule)
     del g
+
+
+def _assert_replays(out, ref, schedule):
+    # The streaming schedule adds its split-K partials in a fixed order: a replay is bitwise
+    # equal.  The small-batch fused schedule adds the expert rows into ylat with fp32 reductions
+    # (the order of a token's k slots is not fixed), so ylat may differ in its last bits and an
+    # output element by at most one bf16 unit in the last place.
+    if schedule == "stream":
+        assert np.array_equal(out, ref)
+        return
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    assert np.all(np.abs(out - ref) <= ulp), np.max(np.abs(out - ref) / ulp)
 
 
 # ---- tiny layer -------------------------------------------------------------------------------
