@@ -28,12 +28,22 @@ namespace moedec {
 // Weight loads and MMAs are pure (no volatile): the compiler may hoist the loads of later rounds
 // ahead of earlier MMAs, which is what keeps enough bytes in flight per warp.
 
-// 16 bytes of static weights: non-coherent path, do not keep in L1 (read once per step).
+// L2 policy for bytes read once per step (the weights): first to be evicted, so that the
+// 148 MB or more of weights a step streams through the 126 MB L2 do not push out what is read
+// again (the step's activations, partial sums, counters and the kernel's own code).
+DEVI uint64_t l2_evict_first() {
+    uint64_t pol;
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 16 bytes of static weights: non-coherent path, do not keep in L1, evict first from L2 (read
+// once per step).
 DEVI uint4 ldg_weights(const void *p) {
     uint4 r;
-    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+        : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+        : "l"(p), "l"(l2_evict_first()));
     return r;
 }
 
@@ -47,7 +57,7 @@ DEVI uint4 ldg_weights_l1(const void *p) {
 // 4 bytes of static weights (4-byte aligned).
 DEVI uint32_t ldg_weights_u32(const void *p) {
     uint32_t r;
-    asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+    asm("ld.global.nc.L1::no_allocate.L2::cache_hint.u32 %0, [%1], %2;" : "=r"(r) : "l"(p), "l"(l2_evict_first()));
     return r;
 }
 

@@ -36,6 +36,13 @@ enum SmallQueue { QS_ROUTER = 0, QS_TOPK, QS_DN, QS_SGU, QS_EGU, QS_SD, QS_EDOWN
 constexpr int kWarps = 8;
 constexpr size_t kSmallSmemLimit = 100 * 1024;  // dynamic shared memory of one CTA (two CTAs per SM)
 
+// K chunk of the expert-down activation staging (per warp: the expert's entries, fp16 hi/lo):
+// all of I when the eight warps' buffers fit, so that an item stages once and streams its
+// weights in one pass; else 512
+__host__ __device__ inline int edown_kc(int I, int B) {
+    return (size_t)kWarps * 2 * B * f16_pitch(I) * 2 <= kSmallSmemLimit ? I : (kKChunk < I ? kKChunk : I);
+}
+
 // ---------------------------------------------------------------------------------------------
 // one 16-row tile x one 8-column token tile; `col` is the staged column that this lane's MMA
 // column (g) reads, or -1 for a zero operand
@@ -432,7 +439,7 @@ DEVI bool w_edown(const StepArgs &a, const RouteSmem &rt, int item, uint16_t *ws
     __syncwarp();
     const size_t eq = (size_t)en.e * L * (I / 2), es = (size_t)en.e * L * (I / 32);
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, dummy[4];
-    const int kc = kKChunk < I ? kKChunk : I;
+    const int kc = edown_kc(I, a.B);
     for (int c0 = 0; c0 < I; c0 += kc) {
         __syncwarp();
         stage_f16_from_f32<true>(ws, f16_pitch(kc), a.ws.a, I, en.cnt, [&](int t) { return s_ent[warp][t]; },
@@ -487,7 +494,7 @@ __host__ __device__ inline size_t fused_small_smem(const StepArgs &a) {
     mx((size_t)B * f16_pitch(a.d.H) * 2);                                 // x, fp16
     mx((size_t)2 * B * f16_pitch(a.d.L) * 2);                             // h, fp16 hi/lo
     mx((size_t)2 * B * f16_pitch(a.d.Is) * 2);                            // sh_a, fp16 hi/lo
-    mx((size_t)kWarps * 2 * B * f16_pitch(kKChunk < a.d.I ? kKChunk : a.d.I) * 2);  // a, per warp
+    mx((size_t)kWarps * 2 * B * f16_pitch(edown_kc(a.d.I, B)) * 2);  // a, per warp
     mx((size_t)2 * B * bf16_pitch(a.d.L) * 2);                            // ylat, bf16 hi/lo
     return m;
 }
@@ -609,8 +616,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         if (alive) {
             __syncthreads();
             const int n = route.n_active * (L / 16);
-            const int kc = kKChunk < I ? kKChunk : I;
-            uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(kc);
+            uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(edown_kc(I, B));
             const int ok = warp_queue(QS_EDOWN, n, c_m, G_m, [&](int it) { return w_edown(a, route, it, ws); });
             alive = __syncthreads_and(ok) != 0;
         }
@@ -660,7 +666,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
 bool fused_small_supports(const Dims &d, int B) {
     // K splits of whole bf16 (32) and MXFP4 (128) rounds; at most 4 tokens so that the hi/lo
     // columns of every part fit one 8-column MMA tile
-    const int kc = kKChunk < d.I ? kKChunk : d.I;
+    const int kc = edown_kc(d.I, B);
     const size_t x16 = (size_t)B * (d.H + 32) * 2, hl = (size_t)2 * B * (d.L + 32) * 2;
     const size_t smem = std::max(std::max(x16, hl), std::max((size_t)2 * B * (d.Is + 16) * 2,
                                                              (size_t)kWarps * 2 * B * (kc + 16) * 2));
