@@ -221,7 +221,11 @@ MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, const uint16
  * capacity in rows in, rows written out.  Synchronises `stream`.  INVALID_ARG without
  * MOEDEC_FLAG_TRACE.
  *   split-K and small-batch kernels, row = CTA: 0 start, 1 router, 2 top-k, 3 W_dn, 4 shared
- *     gate/up, 5 routing wait, 6 expert gate/up, 7 shared down, 8 expert down, 9 W_up, 10 exit.
+ *     gate/up, 5 routing wait, 6 expert gate/up, 7 shared down, 8 expert down, 9 W_up, 10 exit
+ *     (small-batch: 11 routing seen; the shared-expert CTAs stamp 0, 4, 7, 9, 10 only);
+ *     small-batch top-k CTAs also fill row (grid size + CTA): 0 logits complete, 1 scores,
+ *     2 warp candidates, 3 ranked, 4 routing written, 5 expert masks (batch > 1), 6 buckets
+ *     written, 7 buckets published.
  *   streaming kernel (batch <= 2), row = 16 * CTA + warp: 0 start, 1 fp16 copy of x done,
  *     2..6 SM clock cycles spent issuing copies and claiming work, waiting for a stage's data,
  *     waiting for activation blocks, in MMAs, in item epilogues; 7 stages consumed; 9 last stage
