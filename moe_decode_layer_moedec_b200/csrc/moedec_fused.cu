@@ -10,7 +10,7 @@
 //   3 shared gate/up blocks    (sh_a)                              CTA items
 //   4 expert gate/up, 16 rows  waits: buckets, all of h            warp items
 //   5 shared down blocks       waits: all of sh_a                  CTA items
-//   6 expert down, 16 rows     waits: that expert's gate/up items  warp items; combine per token
+//   6 expert down, 16 rows     waits: that expert's gate/up items  warp items; w * y added into ylat
 //   7 W_up row blocks          waits: their ylat rows, all of sh   CTA items; writes out
 //
 // An item only ever waits on items of earlier queues (all of which were claimed by resident CTAs
@@ -61,6 +61,8 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
     __shared__ int s_ok;
     __shared__ int s_ent[8][kExpertTokGroup];
     __shared__ int s_shift[8][kExpertTokGroup];
+    __shared__ float s_w[8][kExpertTokGroup];
+    __shared__ SplitKRoute route;
     __shared__ int s_next;
     unsigned *ctl = a.ws.ctl;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,7 +118,8 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
               [&](int it) { item_router<true>(a, it, smem, &s_flag); return true; });
     stamp(1);
     // 1: top-k
-    cta_queue(Q_TOPK, a.B, [](int) {}, [&](int it) { return item_topk<true>(a, it, topk, (unsigned)a.p.rt.blocks); });
+    cta_queue(Q_TOPK, a.B, [](int) {},
+              [&](int it) { return item_topk<true>(a, it, topk, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat); });
     stamp(2);
     // 2: W_dn
     cta_queue(Q_DN, n_dn, [&](int it) { prefetch_dn(a, it); },
@@ -131,9 +134,12 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
     if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)a.p.dn.blocks, &s_ok);
     stamp(5);
     if (alive) {
-        const int n = __ldcg(a.ws.n_active) * (a.d.I / 16);
+        cta_load_routing(a, route);
+        __syncthreads();
+        const int n = route.n_active * (a.d.I / 16);
         uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)warp * expert_warp_smem(a.B));
-        warp_queue(Q_EGU, n, false, [&](int it) { return warp_expert_item<true, false>(a, xs, it, s_ent[warp], s_shift[warp]); });
+        warp_queue(Q_EGU, n, false,
+                   [&](int it) { return warp_expert_item<true, false>(a, xs, it, s_ent[warp], s_shift[warp], &route); });
     }
     stamp(6);
     // 5: shared down
@@ -143,10 +149,11 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
     // 6: expert down (warp items), each waits on its expert's gate/up rows
     if (alive) {
         __syncthreads();
-        const int n = __ldcg(a.ws.n_active) * (a.d.L / 16);
+        const int n = route.n_active * (a.d.L / 16);
         uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)warp * expert_warp_smem(a.B));
-        const int ok = warp_queue(Q_EDOWN, n, true,
-                                  [&](int it) { return warp_expert_item<true, true>(a, xs, it, s_ent[warp], s_shift[warp]); });
+        const int ok = warp_queue(Q_EDOWN, n, true, [&](int it) {
+            return warp_expert_item<true, true>(a, xs, it, s_ent[warp], s_shift[warp], &route, s_w[warp]);
+        });
         alive = __syncthreads_and(ok) != 0;
     }
     stamp(8);
@@ -202,8 +209,16 @@ cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm) {
 cudaError_t init_fused_attributes() {
     const void *fns[] = {(const void *)k_fused<0>, (const void *)k_fused<1>, (const void *)k_fused<2>,
                          (const void *)k_fused<3>, (const void *)k_fused<4>};
+    int dev = 0, optin = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     for (const void *f : fns) {
-        cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        // all the dynamic shared memory the device allows next to the kernel's static part (the
+        // full-size layer needs at most 132 KB at 64 tokens)
+        cudaFuncAttributes fa;
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, f);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

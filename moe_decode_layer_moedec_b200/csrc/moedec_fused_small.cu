@@ -83,10 +83,16 @@ DEVI void s_bf16(const uint16_t *__restrict__ W, size_t ldw, int row0, int kg, i
     for (int j = 0; j < 4; ++j) acc[j] += acc2[j];
 }
 
-template <int D, bool PAIR>
+struct NoPre {
+    DEVI void operator()() const {}
+};
+
+// pre() runs between the ring's first D rounds of weight loads and their first use: work that
+// the weights do not depend on (a wait, the activation staging) overlaps their flight.
+template <int D, bool PAIR, class Pre = NoPre>
 DEVI void s_fp4(const uint8_t *__restrict__ Qa, const uint8_t *__restrict__ Sa, const uint8_t *__restrict__ Qb,
                 const uint8_t *__restrict__ Sb, size_t ldq, size_t lds, int row0, int kg, int nrounds, const uint16_t *xs,
-                int pitch, int kofs, int col, float (&acc)[4], float (&acc2)[4]) {
+                int pitch, int kofs, int col, float (&acc)[4], float (&acc2)[4], Pre pre = Pre()) {
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const size_t ra = (size_t)(row0 + g), rb = ra + 8;
     const uint8_t *qa0 = Qa + ra * ldq + kg / 2 + 16 * q, *qa1 = Qa + rb * ldq + kg / 2 + 16 * q;
@@ -108,6 +114,7 @@ DEVI void s_fp4(const uint8_t *__restrict__ Qa, const uint8_t *__restrict__ Sa, 
             fp4_load(fa[s], qa0, qa1, sa0, sa1, s);
             if (PAIR) fp4_load(fb[PAIR ? s : 0], qb0, qb1, sb0, sb1, s);
         }
+    pre();
     for (int r0 = 0; r0 < nrounds; r0 += D) {
 #pragma unroll
         for (int s = 0; s < D; ++s) {
@@ -295,30 +302,7 @@ DEVI void w_sgu(const StepArgs &a, int item, const uint16_t *xs16, const int *xs
     warp_signal_add(a.ws.ctl + CTL_SGU_DONE, 1u);
 }
 
-// The step's expert buckets, copied into shared memory once per CTA when the routing is out
-// (the routed items read them from there instead of paying a global round trip each).
-struct RouteSmem {
-    int n_active;
-    int e[kSmallMaxBatch * kMaxTopK], cnt[kSmallMaxBatch * kMaxTopK], off[kSmallMaxBatch * kMaxTopK];
-    int ent[kSmallMaxBatch * kMaxTopK];
-    float w[kSmallMaxBatch * kMaxTopK];  // routing weight of each entry
-};
-
-// all threads; every load is issued before the first use (one round trip); a barrier must follow
-DEVI void cta_load_routing(const StepArgs &a, RouteSmem &r) {
-    const int n = a.B * a.d.k;  // >= n_active
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int e = __ldcg(a.ws.active_e + i), c = __ldcg(a.ws.active_cnt + i), o = __ldcg(a.ws.active_off + i);
-        const int en = __ldcg(a.ws.entries + i);
-        const float w = __ldcg(a.ws.wts + i);
-        r.e[i] = e;
-        r.cnt[i] = c;
-        r.off[i] = o;
-        r.ent[i] = en;
-        r.w[i] = w;
-    }
-    if (threadIdx.x == 0) r.n_active = __ldcg(a.ws.n_active);
-}
+using RouteSmem = RouteTables<kSmallMaxBatch * kMaxTopK, kSmallMaxBatch * kMaxTopK>;
 
 // this warp's entries of active expert slot j: ent[i] for i < cnt (lane i holds entry i)
 struct Entries {
@@ -427,27 +411,36 @@ DEVI bool w_edown(const StepArgs &a, const RouteSmem &rt, int item, uint16_t *ws
     const int L = a.d.L, I = a.d.I, K = a.d.k;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int tiles = L / 16, j = item / tiles, tile = item % tiles, row0 = tile * 16;
-    if (!warp_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(I / 16))) return false;
     const Entries en = warp_entries(rt, j);
     __shared__ int s_ent[kWarps][kMaxTopK], s_shift[kWarps][kMaxTopK];  // cnt <= B <= 4
     const int warp = threadIdx.x >> 5;
-    __syncwarp();
-    if (lane < en.cnt) {
-        s_ent[warp][lane] = en.my_ent;
-        s_shift[warp][lane] = prescale_shift(__uint_as_float(__ldcg(a.ws.a_amax + en.my_ent)));
-    }
-    __syncwarp();
     const size_t eq = (size_t)en.e * L * (I / 2), es = (size_t)en.e * L * (I / 32);
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, dummy[4];
     const int kc = edown_kc(I, a.B);
-    for (int c0 = 0; c0 < I; c0 += kc) {
+    bool ok = true;
+    int c0 = 0;
+    // Only the activations wait for the expert's gate/up items: each pass issues its first
+    // weight loads, then (first pass) waits and takes the entries' exponents, and stages its
+    // K chunk of a.  After an abort the pass still runs on whatever is staged; nothing of it is
+    // published.
+    auto pre = [&]() {
+        if (c0 == 0) {
+            ok = warp_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(I / 16));
+            __syncwarp();
+            if (lane < en.cnt) {
+                s_ent[warp][lane] = en.my_ent;
+                s_shift[warp][lane] = prescale_shift(__uint_as_float(__ldcg(a.ws.a_amax + en.my_ent)));
+            }
+        }
         __syncwarp();
         stage_f16_from_f32<true>(ws, f16_pitch(kc), a.ws.a, I, en.cnt, [&](int t) { return s_ent[warp][t]; },
                                  s_shift[warp], c0, kc, lane, 32);
         __syncwarp();
+    };
+    for (; c0 < I; c0 += kc)
         s_fp4<5, false>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I / 2, I / 32, row0, c0, kc / 128, ws,
-                        f16_pitch(kc), 0, g < 2 * en.cnt ? g : -1, acc, dummy);
-    }
+                        f16_pitch(kc), 0, g < 2 * en.cnt ? g : -1, acc, dummy, pre);
+    if (!ok) return false;
     if (q < en.cnt) {
         const int ent = s_ent[warp][q];
         const float ws_ = rt.w[ent] * exp2i(s_shift[warp][q]);

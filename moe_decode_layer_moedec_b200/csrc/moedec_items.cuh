@@ -378,6 +378,44 @@ DEVI float combine_value(const StepArgs &a, int b, int l) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// The step's expert buckets, copied into shared memory once per CTA when the routing is out, so
+// that the routed items of the fused schedules read them from there instead of paying a global
+// round trip each.  NEXP >= active experts (min(E, B k)), NENT >= entries (B k).
+template <int NEXP, int NENT>
+struct RouteTables {
+    int n_active;
+    int e[NEXP], cnt[NEXP], off[NEXP];
+    int ent[NENT];
+    float w[NENT];  // routing weight of each entry
+};
+
+// all threads; every load is issued before the first use (one round trip); a barrier must follow
+template <int NEXP, int NENT>
+DEVI void cta_load_routing(const StepArgs &a, RouteTables<NEXP, NENT> &r) {
+    const int n = a.B * a.d.k, n_exp = n < a.d.E ? n : a.d.E;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        int e = 0, c = 0, o = 0;
+        if (i < n_exp) {
+            e = __ldcg(a.ws.active_e + i);
+            c = __ldcg(a.ws.active_cnt + i);
+            o = __ldcg(a.ws.active_off + i);
+        }
+        const int en = __ldcg(a.ws.entries + i);
+        const float w = __ldcg(a.ws.wts + i);
+        if (i < n_exp) {
+            r.e[i] = e;
+            r.cnt[i] = c;
+            r.off[i] = o;
+        }
+        r.ent[i] = en;
+        r.w[i] = w;
+    }
+    if (threadIdx.x == 0) r.n_active = __ldcg(a.ws.n_active);
+}
+
+using SplitKRoute = RouteTables<kMaxExperts, kMaxBatch * kMaxTopK>;
+
+// ---------------------------------------------------------------------------------------------
 // routed experts: one warp = 16 rows of one active expert for up to 16 of its tokens
 
 template <int NT, bool SPLIT>
@@ -453,10 +491,12 @@ DEVI void warp_expert_gu(const StepArgs &a, uint16_t *xs, int e, int tile, const
     }
 }
 
-// y rows of 16-row block `tile` for the warp's tokens; FUSED also combines each token's latent
-// rows once all its top-k slots have written them (counter per token and 16-row block).
+// y rows of 16-row block `tile` for the warp's tokens.  FUSED folds the combine in: each
+// token's rows, times its routing weight (ent_w), are added into ylat with fp32 reductions and
+// the block's ylat count grows by the number of tokens (complete at B k).
 template <bool FUSED, int NT, bool SPLIT>
-DEVI void warp_expert_down(const StepArgs &a, uint16_t *xs, int e, int tile, const int *ent, const int *shift, int ntok) {
+DEVI void warp_expert_down(const StepArgs &a, uint16_t *xs, int e, int tile, const int *ent, const int *shift, int ntok,
+                           const float *ent_w = nullptr) {
     const int L = a.d.L, I = a.d.I, K = a.d.k, lane = threadIdx.x & 31;
     const int ncols = SPLIT ? 2 * ntok : ntok;
     const int pitch = f16_pitch(kKChunk);
@@ -471,52 +511,53 @@ DEVI void warp_expert_down(const StepArgs &a, uint16_t *xs, int e, int tile, con
         tile_fp4<NT, false>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I / 2, I / 32, row0, kc0, kc / 128, xs,
                             pitch, 0, ncols, acc, acc);
     }
+    if (FUSED) {
+        tile_foreach<NT, SPLIT>(acc, ntok, [&](int t, int r, float v) {
+            atomicAdd(a.ws.ylat + (size_t)(ent[t] / K) * L + row0 + r, v * exp2i(shift[t]) * ent_w[t]);
+        });
+        warp_signal_add(a.ws.ctl + a.p.ctl_ylat + tile, (unsigned)ntok);
+        return;
+    }
     tile_foreach<NT, SPLIT>(acc, ntok, [&](int t, int r, float v) {
         a.ws.y[(size_t)ent[t] * L + row0 + r] = v * exp2i(shift[t]);
     });
-    if (!FUSED) return;
-    __threadfence();
-    __syncwarp();
-    unsigned *comb = a.ws.ctl + a.p.ctl_comb;
-    const int nblk = L / 16;
-    bool mine = false;
-    if (lane < ntok) {
-        const int b = ent[lane] / K;
-        mine = atomicAdd(comb + (size_t)b * nblk + tile, 1u) == (unsigned)(K - 1);
-    }
-    unsigned todo = __ballot_sync(0xffffffffu, mine);
-    if (todo) __threadfence();  // acquire: the other slots' y rows are visible
-    while (todo) {
-        const int tl = __ffs(todo) - 1;
-        todo &= todo - 1;
-        const int b = ent[tl] / K;
-        if (lane < 16) a.ws.ylat[(size_t)b * L + row0 + lane] = combine_value(a, b, row0 + lane);
-        warp_signal_add(a.ws.ctl + a.p.ctl_ylat + tile, 1u);
-    }
 }
 
 // One warp item: 16 rows (`tile`) of active expert slot j, all its tokens in groups of 16.
 // Returns false if the fused step was aborted while waiting.
+// rt (FUSED): the routing tables in shared memory; w_ent / w_shift / w_w: the warp's scratch
+// for a group's entries, exponents and (down) routing weights.
 template <bool FUSED, bool DOWN>
-DEVI bool warp_expert_item(const StepArgs &a, uint16_t *xs, int item, int *w_ent, int *w_shift) {
+DEVI bool warp_expert_item(const StepArgs &a, uint16_t *xs, int item, int *w_ent, int *w_shift,
+                           const SplitKRoute *rt = nullptr, float *w_w = nullptr) {
     const int tiles = (DOWN ? a.d.L : a.d.I) / 16;
     const int j = item / tiles, tile = item % tiles, lane = threadIdx.x & 31, K = a.d.k;
     if (FUSED && DOWN && !warp_wait_geq(a, a.ws.ctl + a.p.ctl_gu + j, (unsigned)(a.d.I / 16))) return false;
-    const int e = __ldcg(a.ws.active_e + j), cnt = __ldcg(a.ws.active_cnt + j), off = __ldcg(a.ws.active_off + j);
+    int e, cnt, off;
+    if (FUSED) {
+        e = rt->e[j];
+        cnt = rt->cnt[j];
+        off = rt->off[j];
+    } else {
+        e = __ldcg(a.ws.active_e + j);
+        cnt = __ldcg(a.ws.active_cnt + j);
+        off = __ldcg(a.ws.active_off + j);
+    }
     for (int t0 = 0; t0 < cnt; t0 += kExpertTokGroup) {
         const int ntok = min(kExpertTokGroup, cnt - t0);
         __syncwarp();
         if (lane < ntok) {
-            const int ent = __ldcg(a.ws.entries + off + t0 + lane);
+            const int ent = FUSED ? rt->ent[off + t0 + lane] : __ldcg(a.ws.entries + off + t0 + lane);
             w_ent[lane] = ent;
+            if (FUSED && DOWN) w_w[lane] = rt->w[ent];
             const unsigned amax = DOWN ? __ldcg(a.ws.a_amax + ent) : __ldcg(a.ws.ctl + a.p.ctl_hamax + ent / K);
             w_shift[lane] = prescale_shift(__uint_as_float(amax));
         }
         __syncwarp();
         if (DOWN) {
-            if (ntok <= 4) warp_expert_down<FUSED, 1, true>(a, xs, e, tile, w_ent, w_shift, ntok);
-            else if (ntok <= 8) warp_expert_down<FUSED, 1, false>(a, xs, e, tile, w_ent, w_shift, ntok);
-            else warp_expert_down<FUSED, 2, false>(a, xs, e, tile, w_ent, w_shift, ntok);
+            if (ntok <= 4) warp_expert_down<FUSED, 1, true>(a, xs, e, tile, w_ent, w_shift, ntok, w_w);
+            else if (ntok <= 8) warp_expert_down<FUSED, 1, false>(a, xs, e, tile, w_ent, w_shift, ntok, w_w);
+            else warp_expert_down<FUSED, 2, false>(a, xs, e, tile, w_ent, w_shift, ntok, w_w);
         } else {
             if (ntok <= 4) warp_expert_gu<1, true>(a, xs, e, tile, w_ent, w_shift, ntok);
             else if (ntok <= 8) warp_expert_gu<1, false>(a, xs, e, tile, w_ent, w_shift, ntok);
@@ -558,7 +599,7 @@ DEVI bool item_up(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
         const int nblk = KR / 16;
         int ok = 1;
         if (threadIdx.x < nblk) {
-            ok = wait_geq(a, a.ws.ctl + a.p.ctl_ylat + k0 / 16 + threadIdx.x, (unsigned)B) ? 1 : 0;
+            ok = wait_geq(a, a.ws.ctl + a.p.ctl_ylat + k0 / 16 + threadIdx.x, (unsigned)(B * a.d.k)) ? 1 : 0;
             __threadfence();
         }
         if (!__syncthreads_and(ok)) return false;

@@ -94,7 +94,7 @@ def test_mid_back_to_back_and_graph(mid, torch_cuda, schedule):
             layer.step(x, out=o, stream=stream)
     torch.cuda.synchronize()
     for o, r in zip(outs, ref):
-        _assert_replays(bf16_tensor_to_f32(o), r, schedule)
+        _assert_replays(bf16_tensor_to_f32(o), r, exact=schedule == "stream")
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
         for x, o in zip(xs, outs):
@@ -104,16 +104,16 @@ def test_mid_back_to_back_and_graph(mid, torch_cuda, schedule):
     g.replay()
     torch.cuda.synchronize()
     for o, r in zip(outs, ref):
-        _assert_replays(bf16_tensor_to_f32(o), r, schedule)
+        _assert_replays(bf16_tensor_to_f32(o), r, exact=schedule == "stream")
     del g
 
 
-def _assert_replays(out, ref, schedule):
-    # The streaming schedule adds its split-K partials in a fixed order: a replay is bitwise
-    # equal.  The small-batch fused schedule adds the expert rows into ylat with fp32 reductions
-    # (the order of a token's k slots is not fixed), so ylat may differ in its last bits and an
-    # output element by at most one bf16 unit in the last place.
-    if schedule == "stream":
+def _assert_replays(out, ref, exact):
+    # The streaming and multi-kernel schedules add split-K partials and the k slots in a fixed
+    # order: a replay is bitwise equal (exact).  The fused schedules add the expert rows into
+    # ylat with fp32 reductions (the order of a token's k slots is not fixed), so ylat may differ
+    # in its last bits and an output element by at most one bf16 unit in the last place.
+    if exact:
         assert np.array_equal(out, ref)
         return
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
@@ -157,9 +157,18 @@ def test_tiny_deterministic(tiny, schedule):
     x = synth.tokens(w, batch=8)
     a = run_layer(layer, x)
     b = run_layer(layer, x)
-    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    assert np.array_equal(a[1], b[1])
+    # At 8 tokens only the multi-kernel schedule adds the k slots in a fixed order; the fused
+    # split-K kernel (also taken by "stream" above 2 tokens) adds them into ylat with fp32
+    # reductions: ylat and what follows from it agree to rounding, the rest bitwise.
+    exact = schedule == "multi"
+    _assert_replays(a[0], b[0], exact)
     for k in a[3]:
-        assert np.array_equal(a[3][k], b[3][k]), k
+        if not exact and k in ("ylat", "up"):
+            r, _ = rel_errors(a[3][k], b[3][k])
+            assert r < 1e-5, (k, r)
+        else:
+            assert np.array_equal(a[3][k], b[3][k]), k
 
 
 @pytest.mark.parametrize("schedule", SCHEDULES)
