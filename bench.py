@@ -12,7 +12,8 @@ prints one JSON line.  Under torchrun every rank runs an independent replica (th
 not shard; no collective touches the data path); value = all ranks' steps / max time.
 
 --impl reference times the CPU oracle (the plain fp64 C implementation) on this host's cores
-for a bounded sample of the same workload; it is the baseline the driver divides by.
+for a bounded sample of the same workload, on the same metric and configuration: the reference
+arm that this bench's throughput is compared against.
 """
 from __future__ import annotations
 
