@@ -53,7 +53,7 @@ extern "C" {
 typedef enum moedec_status {
     MOEDEC_OK = 0,
     MOEDEC_ERR_INVALID_ARG = -1,  /* NULL handle/pointer, misaligned pointer, batch < 0, bad abi_version */
-    MOEDEC_ERR_UNSUPPORTED = -2,  /* dimensions or batch outside what this build handles (see moedec_create) */
+    MOEDEC_ERR_UNSUPPORTED = -2,  /* dimensions or batch outside what this library handles (see moedec_create) */
     MOEDEC_ERR_CUDA = -3,         /* a CUDA runtime call failed; the CUDA error is kept in the handle */
     MOEDEC_ERR_OOM = -4,          /* workspace allocation failed */
     MOEDEC_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (reported by the next call) */
