@@ -152,6 +152,8 @@ KERNEL_SOURCES = {
                           "moedec_router.cuh", "moedec_internal.h"],
     "fused_step_small": ["moedec_fused_small.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
                          "moedec_router.cuh", "moedec_internal.h"],
+    "fused_step_splitk": ["moedec_fused.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
+                          "moedec_router.cuh", "moedec_internal.h"],
 }
 
 
