@@ -56,6 +56,23 @@ def dist_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
 
 
+def max_over_ranks(v: float, dist, device) -> float:
+    """The largest of every rank's v (v itself without a process group): a multi-rank time is the
+    slowest rank's."""
+    if dist is None:
+        return v
+    import torch
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, steps: int, max_ms: float) -> float:
+    """Whole-job layer-steps/s of `world` independent replicas that each ran `steps` steps, the
+    slowest in max_ms milliseconds."""
+    return world * steps / (max_ms / 1e3)
+
+
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
@@ -354,14 +371,10 @@ def main():
             for _ in range(reps):
                 g_main.replay()
         torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, f"cuda:{local_rank}")
     clocks = clk.summary()
-    if dist:
-        t = torch.tensor([ms], device=f"cuda:{local_rank}", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
     ms_per_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+    value = replica_throughput(world, args.steps, ms)
 
     # per-kernel durations: a second replay of the same K steps with an event pair around every
     # kernel on the stream it runs on (main or side stream)
@@ -409,12 +422,8 @@ def main():
             out_host.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device=f"cuda:{local_rank}", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, f"cuda:{local_rank}")
+    e2e_value = replica_throughput(world, args.steps, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
