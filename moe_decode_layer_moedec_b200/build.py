@@ -35,15 +35,33 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every csrc/*.cu to an object (in parallel, under _build/), then link libmoedec.so."""
     if not force and not _stale():
         return SO
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
-           "-Xcompiler", "-fvisibility=hidden", "-shared", "-cudart", "static", "-I", os.path.join(ROOT, "include"),
-           *sources(), "-o", SO + ".tmp"]
+    from concurrent.futures import ThreadPoolExecutor
+    objdir = os.path.join(ROOT, "_build", "moedec")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
+             "-Xcompiler", "-fvisibility=hidden", "-I", os.path.join(ROOT, "include")]
     if verbose:
-        cmd.insert(-2, "-Xptxas=-v")
-        print(" ".join(cmd), file=sys.stderr)
-    subprocess.check_call(cmd)
+        flags.append("-Xptxas=-v")
+
+    def compile_one(src: str) -> str:
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *flags, "-c", src, "-o", obj]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0 or verbose:
+            sys.stderr.write(r.stdout + r.stderr)
+        if r.returncode != 0:
+            raise subprocess.CalledProcessError(r.returncode, cmd)
+        return obj
+
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
+        objs = list(ex.map(compile_one, srcs))
+    subprocess.check_call([nvcc(), *ARCH, "-shared", "-cudart", "static", *objs, "-o", SO + ".tmp"])
     os.replace(SO + ".tmp", SO)
     return SO
 

@@ -13,8 +13,8 @@ def _declared(header):
 
 
 def test_library_exports_every_declared_symbol():
-    from moe_decode_layer_moedec_b200 import build
-    so = build.build()
+    from tests.conftest import build_library
+    so = build_library()
     lib = ctypes.CDLL(so)
     names = _declared("moedec.h")
     assert {"moedec_create", "moedec_step", "moedec_destroy"} <= set(names)
