@@ -4,12 +4,17 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 A step is one decode layer step (router, top-k, latent down-projection, routed MXFP4 experts,
-combine, up-projection, shared expert) for one batch of tokens.  The timed region replays a
+combine, up-projection, shared expert) for one batch of tokens.  A timed region replays a
 CUDA graph of exactly K steps that cycles through `--layers` layers of distinct seeded weights
 (32 by default, ~99 GB), so every step streams its weights from HBM: the per-step working set
-(>= 148 MB) exceeds the 126 MB L2 and the same layer returns only after 31 others.  Rank 0
-prints one JSON line.  Under torchrun every rank runs an independent replica (the step does
-not shard; no collective touches the data path); value = all ranks' steps / max time.
+(>= 148 MB) exceeds the 126 MB L2 and the same layer returns only after 31 others.  The reported
+time is the median of `--reps` (5) such regions, each bracketed by a synchronise (and a barrier
+under torchrun); every layer's device error word is read after them, so a step that gave up on
+a bounded wait fails the run instead of being timed.  The headline is `--workload` (full_b1);
+`per_config` repeats the measurement for the metric's other batches (B = 2, 16, 64), each over
+32 layers of its own weights.  Rank 0 prints one JSON line.  Under torchrun every rank runs an
+independent replica (the step does not shard; no collective touches the data path); value =
+all ranks' steps / max time.
 
 --impl reference times the CPU oracle (the plain fp64 C implementation) on this host's cores
 for a bounded sample of the same workload, on the same metric and configuration: the reference
@@ -34,6 +39,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "MoE layer-steps/s & µs/step at B=1..64; achieved HBM GB/s vs B200 peak"
+PER_CONFIG = ("full_b1", "full_b2", "full_b16", "full_b64_skewed")  # the metric's batches
 UNIT = "layer-steps/s"
 
 
@@ -47,6 +53,8 @@ def parse():
     p.add_argument("--layers", type=int, default=0, help="distinct layers cycled through (default 32)")
     p.add_argument("--schedule", choices=["fused", "multi", "stream"], default="fused",
                    help="one persistent kernel per step (default) or eight stream-ordered kernels")
+    p.add_argument("--reps", type=int, default=5, help="timed replays of the K-step graph (median)")
+    p.add_argument("--no-per-config", action="store_true", help="skip the B=2/16/64 entries of per_config")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
     return p.parse_args()
@@ -225,7 +233,9 @@ def workload_config(w: synth.Workload, n_layers: int, schedule: str, world: int)
             "top_k": d.top_k, "expert_inter": d.expert_inter, "shared_inter": d.shared_inter,
             "layers_cycled": n_layers,
             "l2": "inputs larger than L2: each step streams one of %d distinct layers (>= 148 MB)" % n_layers,
-            "arith": "MXFP4/bf16 weights, fp16/bf16 tensor-core MMA with fp32 accumulation, fp64 router",
+            "arith": "MXFP4/bf16 weights; tensor-core MMA operands fp16 (MXFP4 parts) and bf16 (dense parts), tokens "
+                     "as hi/lo operand pairs at B <= 4 and for W_up, single fp16 with a per-token power-of-two "
+                     "scale otherwise; fp32 accumulation; router exact products summed in fp64",
             "parallelism": "replicas" if world > 1 else "single GPU", "schedule": schedule}
 
 
@@ -266,29 +276,13 @@ def run_reference(args):
 # ---------------------------------------------------------------------------------------------
 # our arm
 
-def main():
-    args = parse()
-    if args.impl == "reference":
-        return run_reference(args)
-    rank, local_rank, world = dist_env()
+def load_layers(w, n_layers, schedule, local_rank, rank):
+    """n_layers handles of distinct seeded layers of workload w, weights resident in HBM."""
     import torch
-    torch.cuda.set_device(local_rank)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
-                                device_id=torch.device("cuda", local_rank))
-    from moe_decode_layer_moedec_b200 import (FLAG_MULTI_KERNEL, FLAG_SKIP_SCALE_CHECK, FLAG_STREAM, LayerDims,
-                                              MoeDecodeLayer)
-
-    w = synth.WORKLOADS[args.workload]
+    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_SKIP_SCALE_CHECK, FLAG_STREAM, LayerDims, \
+        MoeDecodeLayer
     d = w.dims
-    B = w.batch
-    n_layers = default_layers(w, args.layers)
     dims = LayerDims(d.hidden, d.latent, d.n_experts, d.top_k, d.expert_inter, d.shared_inter, 1)
-
-    # weights of n_layers distinct layers, resident in HBM (created once, outside any timing)
     t0 = time.time()
     layers, dev_weights = [], []
     for l in range(n_layers):
@@ -299,20 +293,97 @@ def main():
             Wd[k] = t.to(f"cuda:{local_rank}", non_blocking=False)
         del W
         flags = 0 if l == 0 else FLAG_SKIP_SCALE_CHECK  # layer 0 runs the create-time scale scan
-        if args.schedule == "multi":
+        if schedule == "multi":
             flags |= FLAG_MULTI_KERNEL
-        if args.schedule == "stream":
+        if schedule == "stream":
             flags |= FLAG_STREAM
-        layers.append(MoeDecodeLayer(dims, Wd, max_batch=B, flags=flags))
+        layers.append(MoeDecodeLayer(dims, Wd, max_batch=w.batch, flags=flags))
         dev_weights.append(Wd)
         if rank == 0 and (l % 8 == 7 or l == n_layers - 1):
-            log(f"[bench] {l + 1}/{n_layers} layers resident ({time.time() - t0:.0f} s)")
-    x_host = torch.from_numpy(synth.tokens(w).view(np.int16)).pin_memory()
-    x = x_host.to(f"cuda:{local_rank}")
-    out = torch.empty_like(x)
-    stream = torch.cuda.Stream()
+            log(f"[bench] {w.name}: {l + 1}/{n_layers} layers resident ({time.time() - t0:.0f} s)")
+    return layers, dev_weights
 
-    # routing of every layer (outside the timed region) -> unique experts touched per step
+
+def check_device_errors(layers, B, stream):
+    """Every layer's sticky device error word: a bounded wait that ran out, or a bad bucket, makes
+    the CTAs leave early and would otherwise be timed as a fast step.  Raises on any."""
+    for L_ in layers:
+        L_.routing(B, stream=stream)
+
+
+class Timed:
+    """Graph replays of `steps` steps over the resident layers, timed with CUDA events on the
+    launching stream; median over `reps` replays, max over ranks."""
+
+    def __init__(self, layers, x, out, stream, steps, warmup, dist, device):
+        import torch
+        self.torch, self.layers, self.x, self.out, self.stream = torch, layers, x, out, stream
+        self.steps, self.warmup, self.dist, self.device = steps, warmup, dist, device
+        n = len(layers)
+        B = x.shape[0]
+        with torch.cuda.stream(stream):
+            for i in range(max(warmup, 3)):   # eager warm-up (module load, caches)
+                layers[i % n].step(x, out=out, stream=stream)
+        torch.cuda.synchronize()
+        check_device_errors(layers, B, stream)
+        self.g_warm = self.capture(max(warmup, 1), 0)
+        self.g_main = self.capture(steps, warmup)
+
+    def capture(self, n_steps, first):
+        torch = self.torch
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
+            for i in range(n_steps):
+                self.layers[(first + i) % len(self.layers)].step(self.x, out=self.out, stream=self.stream)
+        return g
+
+    def replay_ms(self, g):
+        torch = self.torch
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        if self.dist:
+            self.dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(self.stream)
+        with torch.cuda.stream(self.stream):
+            g.replay()
+        ev1.record(self.stream)
+        torch.cuda.synchronize()
+        if self.dist:
+            self.dist.barrier()
+        return ev0.elapsed_time(ev1)
+
+    def run(self, reps, local_rank):
+        """Median ms of `reps` timed replays (each exactly `steps` steps), with untimed replays of
+        the same graph for ~0.5 s on each side so that the clock samples see the step running."""
+        torch = self.torch
+        self.g_warm.replay()
+        torch.cuda.synchronize()
+        t_probe = time.perf_counter()
+        with torch.cuda.stream(self.stream):
+            self.g_main.replay()
+        torch.cuda.synchronize()
+        pad = max(1, min(200, int(0.5 / max(time.perf_counter() - t_probe, 1e-4))))
+        with ClockSampler(local_rank) as clk:
+            with torch.cuda.stream(self.stream):
+                for _ in range(pad):
+                    self.g_main.replay()
+            times = [self.replay_ms(self.g_main) for _ in range(reps)]
+            with torch.cuda.stream(self.stream):
+                for _ in range(pad):
+                    self.g_main.replay()
+            torch.cuda.synchronize()
+        check_device_errors(self.layers, self.x.shape[0], self.stream)
+        ms = max_over_ranks(statistics.median(times), self.dist, self.device)
+        return ms, times, clk.summary()
+
+    def close(self):
+        del self.g_main, self.g_warm
+
+
+def unique_experts(layers, x, out, stream, B):
+    """Mean number of distinct experts a step touches (routing of every layer, untimed)."""
+    import torch
     uniq = []
     with torch.cuda.stream(stream):
         for L_ in layers:
@@ -320,88 +391,82 @@ def main():
             idx, _ = L_.routing(B, stream=stream)
             uniq.append(len(np.unique(idx.cpu().numpy())))
     torch.cuda.synchronize()
-    unique_mean = float(np.mean(uniq))
+    return float(np.mean(uniq))
 
-    def capture(n_steps, first):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
-            for i in range(n_steps):
-                layers[(first + i) % n_layers].step(x, out=out, stream=stream)
-        return g
 
-    # eager warm-up (module load, caches) then the graphs
-    with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            layers[i % n_layers].step(x, out=out, stream=stream)
-    torch.cuda.synchronize()
-    g_warm = capture(max(args.warmup, 1), 0)
-    g_main = capture(args.steps, args.warmup)
-    for L_ in layers:
-        L_.profile(True)
-    g_prof = capture(args.steps, args.warmup)
-    for L_ in layers:
-        L_.profile(False)
+def config_entry(w, ms, times, clocks, steps, world, unique_mean, peak):
+    """One per_config record: time per step, throughput, algorithmic bytes and their HBM fraction."""
+    ms_per_step = ms / steps
+    sb = step_bytes(w.dims, unique_mean, w.batch)
+    return {"workload": w.name, "batch": w.batch, "us_per_step": 1e3 * ms_per_step,
+            "layer_steps_per_s": replica_throughput(world, steps, ms), "unique_experts_per_step": unique_mean,
+            "bytes_per_step": sb, "hbm_gbs": sb / (ms_per_step / 1e3) / 1e9,
+            "hbm_frac": sb / (ms_per_step / 1e3) / 1e9 / peak,
+            "replay_ms": [round(t, 4) for t in times], "clocks": clocks}
 
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g_warm.replay()
-    torch.cuda.synchronize()
-    # untimed replays of the same graph before and after the timed one keep the GPU under load
-    # for ~0.5 s on each side, so that the clock samples are taken while the step runs
-    t_probe = time.perf_counter()
-    with torch.cuda.stream(stream):
-        g_main.replay()
-    torch.cuda.synchronize()
-    reps = max(1, min(200, int(0.5 / max(time.perf_counter() - t_probe, 1e-4))))
-    with ClockSampler(local_rank) as clk:
-        with torch.cuda.stream(stream):
-            for _ in range(reps):
-                g_main.replay()
-        torch.cuda.synchronize()
-        if dist:
-            dist.barrier()
-        torch.cuda.synchronize()
-        ev0.record(stream)
-        with torch.cuda.stream(stream):
-            g_main.replay()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-        if dist:
-            dist.barrier()
-        with torch.cuda.stream(stream):
-            for _ in range(reps):
-                g_main.replay()
-        torch.cuda.synchronize()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), dist, f"cuda:{local_rank}")
-    clocks = clk.summary()
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    rank, local_rank, world = dist_env()
+    import torch
+    torch.cuda.set_device(local_rank)
+    device = f"cuda:{local_rank}"
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+
+    w = synth.WORKLOADS[args.workload]
+    d = w.dims
+    B = w.batch
+    n_layers = default_layers(w, args.layers)
+    peak, peak_src = measured_peak_hbm()
+    layers, dev_weights = load_layers(w, n_layers, args.schedule, local_rank, rank)
+    x_host = torch.from_numpy(synth.tokens(w).view(np.int16)).pin_memory()
+    x = x_host.to(device)
+    out = torch.empty_like(x)
+    stream = torch.cuda.Stream()
+    unique_mean = unique_experts(layers, x, out, stream, B)
+
+    tm = Timed(layers, x, out, stream, args.steps, args.warmup, dist, device)
+    ms, times, clocks = tm.run(args.reps, local_rank)
     ms_per_step = ms / args.steps
     value = replica_throughput(world, args.steps, ms)
+    kps = layers[0].kernels_per_step(B)
 
-    # per-kernel durations: a second replay of the same K steps with an event pair around every
-    # kernel on the stream it runs on (main or side stream)
-    g_warm.replay()
-    ev0.record(stream)
-    with torch.cuda.stream(stream):
-        g_prof.replay()
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    ms_prof = ev0.elapsed_time(ev1)
+    # per-kernel durations: a replay of the same K steps with an event pair around every kernel on
+    # the stream it runs on (main or side stream).  With one kernel per step the dominant kernel's
+    # time per launch is the timed replay's time per step; the bracketed pass (which slows the
+    # kernels it brackets) only splits the time of a multi-kernel step.
+    for L_ in layers:
+        L_.profile(True)
+    g_prof = tm.capture(args.steps, args.warmup)
+    for L_ in layers:
+        L_.profile(False)
+    tm.g_warm.replay()
+    ms_prof = tm.replay_ms(g_prof)
+    check_device_errors(layers, B, stream)
     per_kernel = {}
     for L_ in layers:
         for name, (kms, n) in L_.profile_read().items():
             a, b = per_kernel.get(name, (0.0, 0))
             per_kernel[name] = (a + kms, b + n)
+    del g_prof
     kb = kernel_bytes(d, unique_mean, B)
-    peak, peak_src = measured_peak_hbm()
     if not any(v[0] > 0 for v in per_kernel.values()):
         raise RuntimeError(f"per-kernel profile is empty: {per_kernel}")
     dom = max(per_kernel, key=lambda k: per_kernel[k][0])
     dom_ms, dom_n = per_kernel[dom]
-    dom_avg_s = dom_ms / 1e3 / max(dom_n, 1)
+    dom_avg_s = ms_per_step / 1e3 if kps == 1 else dom_ms / 1e3 / max(dom_n, 1)
     achieved = kb[dom] / dom_avg_s / 1e9
     kernels_table = {k: {"avg_us": 1e3 * v[0] / max(v[1], 1), "launches": v[1],
-                         "share": v[0] / max(sum(x[0] for x in per_kernel.values()), 1e-12),
+                         "share": v[0] / max(sum(x_[0] for x_ in per_kernel.values()), 1e-12),
                          "gbs": kb[k] / (v[0] / 1e3 / max(v[1], 1)) / 1e9 if v[0] > 0 else None}
-                     for k, v in per_kernel.items()}
+                     for k, v in per_kernel.items() if v[1] > 0}
 
     # end to end through the public API: pinned host tokens in, step, result back to pinned host
     out_host = torch.empty_like(x_host).pin_memory()
@@ -422,22 +487,48 @@ def main():
             out_host.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, f"cuda:{local_rank}")
+    check_device_errors(layers, B, stream)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     e2e_value = replica_throughput(world, args.steps, e2e_ms)
+    per_config = {w.name: config_entry(w, ms, times, clocks, args.steps, world, unique_mean, peak)}
+    tm.close()
+    for L_ in layers:
+        L_.close()
+    del layers, dev_weights
+    torch.cuda.empty_cache()
+
+    # the metric's other batches (B = 2, 16, 64), each over its own resident layers, same K and W
+    if not args.no_per_config:
+        for name in PER_CONFIG:
+            if name == w.name:
+                continue
+            wc = synth.WORKLOADS[name]
+            lc, wd = load_layers(wc, default_layers(wc, args.layers), args.schedule, local_rank, rank)
+            xc = torch.from_numpy(synth.tokens(wc).view(np.int16)).to(device)
+            oc = torch.empty_like(xc)
+            uc = unique_experts(lc, xc, oc, stream, wc.batch)
+            tc = Timed(lc, xc, oc, stream, args.steps, args.warmup, dist, device)
+            mc, tsc, cc = tc.run(args.reps, local_rank)
+            per_config[name] = config_entry(wc, mc, tsc, cc, args.steps, world, uc, peak)
+            tc.close()
+            for L_ in lc:
+                L_.close()
+            del lc, wd, xc, oc
+            torch.cuda.empty_cache()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_rate(w, args.cpu_seconds)
 
     sb = step_bytes(d, unique_mean, B)
-    kps = layers[0].kernels_per_step(B)
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
+            "dtype": "f16", "data": "synthetic",
             "config": workload_config(w, n_layers, args.schedule, world),
             "us_per_step": 1e3 * ms_per_step, "unique_experts_per_step": unique_mean,
+            "timed_replays": args.reps, "replay_ms": [round(t, 4) for t in times],
             "step_hbm": {"bytes_per_step": sb, "gbs": sb / (ms_per_step / 1e3) / 1e9,
                          "frac": sb / (ms_per_step / 1e3) / 1e9 / peak, "peak_gbs": peak, "peak": peak_src},
             "clocks": clocks,
@@ -446,15 +537,15 @@ def main():
             "gpu_launches": kps * args.steps,
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(dom, w.name), "bytes_per_launch": kb[dom],
-                         "avg_launch_us": dom_avg_s * 1e6, "peak_source": peak_src},
+                         "avg_launch_us": dom_avg_s * 1e6, "peak_source": peak_src,
+                         "time_source": "timed replay (one kernel per step)" if kps == 1 else
+                                        "per-kernel CUDA events of a bracketed replay"},
             "kernels": kernels_table,
             "profiled_pass_ms_per_step": ms_prof / args.steps,
+            "per_config": per_config,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
-    del g_main, g_prof, g_warm
-    for L_ in layers:
-        L_.close()
     if dist:
         dist.destroy_process_group()
 

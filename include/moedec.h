@@ -162,6 +162,14 @@ MOEDEC_API int moedec_get_taps(moedec_handle *h, float *logits, float *hlat, flo
                                int batch, void *stream);
 
 /*
+ * Router scores of the last step (test tap): scores[b][e] = fp32(1 / (1 + exp(-logit[b][e])))
+ * evaluated in fp64 by the same device function the top-k ranks experts with, written on `stream`
+ * into the caller's device buffer fp32 [batch][E].  batch must equal the last step's batch.
+ * Synchronises `stream` and reports device-side errors like moedec_get_routing.
+ */
+MOEDEC_API int moedec_get_scores(moedec_handle *h, float *scores, int batch, void *stream);
+
+/*
  * Launch counters (host values): launches[i] counts the kernels of variant i issued by this
  * handle since creation; i = 0 the small-batch schedules (batch <= 4), 1 the split-K schedule
  * (batch >= 5).  n_variants in/out.
@@ -198,10 +206,15 @@ MOEDEC_API int moedec_profile_read(moedec_handle *h, double *total_ms, uint64_t 
  * entirely handed to another allocator, and runtimes with a fixed, pre-planned memory budget.
  *   router   bf16 [n_experts][hidden], device, 16-byte aligned      x  bf16 [batch][hidden], device, 16-byte aligned
  *   logits   fp32 [batch][n_experts], device (output)               stream  cudaStream_t as void*
- * Computes logits[b][e] = fp32(sum_j router[e][j] x[b][j]) exactly as moedec_step does (same
- * kernel body and split order, so the values equal moedec_get_taps' logits).  Its split-K scratch
- * is one static 2 MiB device array in the library that every GPU loading the library keeps until
- * the process exits; the call only clears the ticket words it needs (an async memset on `stream`).
+ * Computes logits[b][e] = fp32(sum_j router[e][j] x[b][j]) (exact products, fp64 sums, one
+ * rounding) with the step's router kernel body and its K-split order, so the values are bitwise
+ * equal to moedec_get_taps' logits of a step that runs that body (batches above 4, or
+ * MOEDEC_FLAG_MULTI_KERNEL).  The small-batch step (batch <= 4) adds its K splits with fp64
+ * reductions in arrival order instead, so against its logits the values agree to within one fp32
+ * ulp (they differ only where the exact sum lies within fp64 rounding of an fp32 rounding
+ * boundary).  Its split-K scratch is one static 2 MiB device array in the library that every GPU
+ * loading the library keeps until the process exits; the call only clears the ticket words it
+ * needs (an async memset on `stream`).
  * Limit: (hidden / 512) * batch * n_experts * 8 bytes + 4 KiB <= 2 MiB (hidden a multiple of 512;
  * 256 or 128 when it is not, with proportionally more splits); beyond it the call returns
  * MOEDEC_ERR_UNSUPPORTED.  With hidden 7168 and 896 experts that allows batch <= 20.

@@ -66,6 +66,8 @@ def _load():
     lib.moedec_get_routing.restype = i32
     lib.moedec_get_taps.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp]
     lib.moedec_get_taps.restype = i32
+    lib.moedec_get_scores.argtypes = [vp, vp, i32, vp]
+    lib.moedec_get_scores.restype = i32
     lib.moedec_get_launch_counts.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(i32)]
     lib.moedec_get_launch_counts.restype = i32
     lib.moedec_profile_enable.argtypes = [vp, i32]
@@ -176,6 +178,14 @@ class MoeDecodeLayer:
                                                            _ptr(r["sh"]), _ptr(r.get("up")), batch, _stream_ptr(stream)))
         return r
 
+    def scores(self, batch: int, stream=None):
+        """fp32 router scores [B, E] of the last step, from the same device function the top-k uses."""
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device())
+        s = torch.empty((batch, self.dims.n_experts), dtype=torch.float32, device=dev)
+        self._check("moedec_get_scores", lib.moedec_get_scores(self._h, _ptr(s), batch, _stream_ptr(stream)))
+        return s
+
     def launch_counts(self):
         arr = (ctypes.c_uint64 * 2)()
         n = ctypes.c_int(2)
@@ -222,12 +232,23 @@ class MoeDecodeLayer:
 def router_logits_noalloc(router, x, logits=None, stream=None):
     """fp32 router logits [B, E] without any device allocation by the library (see include/moedec.h).
 
-    For callers that cannot call cudaMalloc; `logits` may be passed in pre-allocated."""
+    For callers that cannot call cudaMalloc; `logits` may be passed in pre-allocated.  router
+    [E, H] and x [B, H] are contiguous 16-bit (bf16 bit patterns) tensors on the current device;
+    logits, if given, is a contiguous fp32 [B, E] tensor there."""
     import torch
+    dev = torch.device("cuda", torch.cuda.current_device())
+    for name, t in (("router", router), ("x", x)):
+        if t.dim() != 2 or t.element_size() != 2 or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous 2-D 16-bit tensor on {dev}")
     E, H = router.shape
     B = x.shape[0]
+    if x.shape[1] != H:
+        raise ValueError(f"x has width {x.shape[1]}, the router {H}")
     if logits is None:
-        logits = torch.empty((B, E), dtype=torch.float32, device=x.device)
+        logits = torch.empty((B, E), dtype=torch.float32, device=dev)
+    elif (logits.dtype != torch.float32 or tuple(logits.shape) != (B, E) or not logits.is_contiguous()
+          or logits.device != dev):
+        raise ValueError(f"logits must be a contiguous float32 [{B}, {E}] tensor on {dev}")
     rc = lib.moedec_router_logits_noalloc(_ptr(router), _ptr(x), E, H, B, _ptr(logits), _stream_ptr(stream))
     if rc != 0:
         raise MoedecError("moedec_router_logits_noalloc", rc)

@@ -410,6 +410,14 @@ MOEDEC_API int moedec_get_taps(moedec_handle *h, float *logits, float *hlat, flo
     return read_device_error(h, s);
 }
 
+MOEDEC_API int moedec_get_scores(moedec_handle *h, float *scores, int batch, void *stream) {
+    if (!h || !scores || batch != h->last_batch || batch <= 0) return MOEDEC_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_scores(h->ws.logits, scores, (size_t)batch * h->d.E, s);
+    if (e != cudaSuccess) return record_cuda(h, e);
+    return read_device_error(h, s);
+}
+
 MOEDEC_API int moedec_get_launch_counts(moedec_handle *h, uint64_t *launches, int *n_variants) {
     if (!h || !launches || !n_variants || *n_variants < 1) return MOEDEC_ERR_INVALID_ARG;
     const int n = *n_variants < 2 ? *n_variants : 2;

@@ -140,6 +140,11 @@ DEVI int prescale_shift(float amax) {
     return t < -100 ? -100 : (t > 100 ? 100 : t);
 }
 
+// Router score of one logit: fp32(1 / (1 + exp(-logit))) evaluated in fp64 (CUDA exp(double)),
+// so that the fp32 result is the correctly rounded sigmoid except in astronomically rare cases.
+// Every kernel that ranks experts, and the score tap, call this one function.
+DEVI float router_score(float logit) { return (float)(1.0 / (1.0 + exp(-(double)logit))); }
+
 DEVI uint16_t f32_to_bf16_rne(float f) {
     uint32_t u = __float_as_uint(f);
     if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u);

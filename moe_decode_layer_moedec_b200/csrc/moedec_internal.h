@@ -155,6 +155,7 @@ cudaError_t launch_up(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_shared_gate_up(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_shared_down(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_scale_check(const uint8_t *s, size_t n, unsigned *bad, cudaStream_t st);
+cudaError_t launch_scores(const float *logits, float *scores, size_t n, cudaStream_t st);
 cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm);
 cudaError_t init_fused_attributes();
 constexpr int kStreamLaunches = 4;  // launches of the streaming small-batch step

@@ -244,7 +244,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float sc = (float)(1.0 / (1.0 + exp(-(double)lg[i])));
+        const float sc = router_score(lg[i]);
         key[i] = valid[i] && sc >= 0.0f ? __float_as_uint(sc) : 0u;  // non-negative fp32 orders like its bits
     }
     stamp(1);

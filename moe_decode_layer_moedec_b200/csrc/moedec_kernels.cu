@@ -16,6 +16,8 @@
 // Split-K partial sums are reduced by the last CTA of each row block (release/acquire ticket)
 // in split order, so every result is deterministic.  Decode is HBM-bound; every kernel streams
 // its weights once with 128-bit loads and keeps the decode tokens on chip.
+#include <algorithm>
+
 #include "moedec_device.cuh"
 #include "moedec_internal.h"
 #include "moedec_items.cuh"
@@ -100,6 +102,14 @@ __global__ void k_scale_check(const uint8_t *s, size_t n, unsigned *bad) {
         found |= (v < 104u || v > 140u) ? 1u : 0u;
     }
     if (__syncthreads_or(found) && threadIdx.x == 0) atomicOr(bad, 1u);
+}
+
+// ---------------------------------------------------------------------------------------------
+// score tap: scores[i] = router_score(logits[i]) for n logits, the same function the top-k ranks by
+
+__global__ void k_scores(const float *logits, float *scores, size_t n) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+        scores[i] = router_score(__ldcg(logits + i));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -198,6 +208,13 @@ cudaError_t launch_shared_down(const StepArgs &a, cudaStream_t s) {
         case 4: return launch_sd_nt<4, false>(a, s);
         default: return launch_sd_nt<8, false>(a, s);
     }
+}
+
+cudaError_t launch_scores(const float *logits, float *scores, size_t n, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    const int grid = (int)std::min<size_t>((n + 255) / 256, 1184);
+    k_scores<<<grid, 256, 0, st>>>(logits, scores, n);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_scale_check(const uint8_t *sc, size_t n, unsigned *bad, cudaStream_t st) {

@@ -540,7 +540,7 @@ DEVI void epi_router(const StepArgs &a, const Geo &g, StSmem &sm, const Item &t,
         const float lg = (float)sum_splits<double, 16>(a.ws.st_rt_part + (size_t)b * g.E + row, (size_t)2 * g.E, p.s_rt);
         a.ws.logits[(size_t)b * g.E + row] = lg;
         // top-k key: fp32 sigmoid score (computed in double) bits + 1; 0 marks "no expert"
-        const float sc = (float)(1.0 / (1.0 + exp(-(double)lg)));
+        const float sc = router_score(lg);
         a.ws.st_key[(size_t)b * g.E + row] = (sc >= 0.0f ? __float_as_uint(sc) : 0u) + 1u;
     }
     if (a.flags & kFlagTestStall) return;  // the routing never completes: its waits must time out

@@ -41,3 +41,24 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Worst float error per (config, tap) of the parity tests that ran, against the bounds."""
+    try:
+        from tests.harness import MARGINS, TOL_MAX_REL, TOL_REL_L2
+    except Exception:
+        return
+    if not MARGINS:
+        return
+    tr = terminalreporter
+    tr.section("parity margins (worst over the tests that ran)")
+    tr.write_line(f"{'config':44s} {'tap':6s} {'rel L2':>10s} {'of bound':>9s} {'max rel':>10s} {'of bound':>9s}")
+    for (cfg, tap), (r, m) in sorted(MARGINS.items()):
+        tr.write_line(f"{cfg:44s} {tap:6s} {r:10.3e} {r / TOL_REL_L2:9.3f} {m:10.3e} {m / TOL_MAX_REL:9.3f}")
+    path = os.environ.get("MOEDEC_PARITY_REPORT")
+    if path:
+        import json
+        with open(path, "w") as f:
+            json.dump([{"config": c, "tap": t, "rel_l2": r, "max_rel": m} for (c, t), (r, m) in sorted(MARGINS.items())],
+                      f, indent=1)

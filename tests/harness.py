@@ -38,8 +38,22 @@ def rel_errors(got: np.ndarray, ref: np.ndarray):
     return rel_l2, max_rel
 
 
+# (config, tap) -> worst (relative L2, max|err|/max|ref|) seen by assert_close in this session;
+# printed at the end of the run (tests/conftest.py), and written as JSON to $MOEDEC_PARITY_REPORT
+MARGINS: dict = {}
+_CONFIG = ["-"]
+
+
+def set_config(name: str):
+    """Label under which the following assert_close calls record their errors."""
+    _CONFIG[0] = name
+
+
 def assert_close(got, ref, name: str):
     rel_l2, max_rel = rel_errors(got, ref)
+    key = (_CONFIG[0], name.split("[")[0])
+    old = MARGINS.get(key, (0.0, 0.0))
+    MARGINS[key] = (max(old[0], rel_l2), max(old[1], max_rel))
     assert rel_l2 <= TOL_REL_L2 and max_rel <= TOL_MAX_REL, \
         f"{name}: relative L2 {rel_l2:.3e} (bound {TOL_REL_L2}), max|err|/max|ref| {max_rel:.3e} (bound {TOL_MAX_REL})"
     return rel_l2, max_rel
@@ -54,7 +68,14 @@ def assert_logits_match(got: np.ndarray, ref: np.ndarray, name: str = "logits"):
     if diff.any():
         ulps = np.abs(got.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
         assert ulps[diff].max() <= 1, f"{name}: logits differ by more than one ulp"
-        assert diff.mean() <= 1e-4, f"{name}: {int(diff.sum())} logits differ"
+        assert diff.sum() <= max(1, 1e-4 * diff.size), f"{name}: {int(diff.sum())} logits differ"
+
+
+def oracle_scores(logits: np.ndarray) -> np.ndarray:
+    """The oracle's fp32 score of every logit (same shape)."""
+    import oracle
+    flat = np.ascontiguousarray(logits, dtype=np.float32).ravel()
+    return np.array([oracle.score(float(v)) for v in flat], dtype=np.float32).reshape(logits.shape)
 
 
 def run_layer(layer, x_np: np.ndarray):
@@ -65,6 +86,7 @@ def run_layer(layer, x_np: np.ndarray):
     B = x_np.shape[0]
     idx, w = layer.routing(B)
     taps = layer.taps(B)
+    taps["scores"] = layer.scores(B)
     torch.cuda.synchronize()
     return (bf16_tensor_to_f32(out), idx.cpu().numpy(), w.cpu().numpy(),
             {k: v.cpu().numpy() for k, v in taps.items()})

@@ -17,6 +17,7 @@ import oracle
 import synth
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 TINY = synth.TINY
 
 
@@ -157,6 +158,38 @@ def test_score_closed_forms():
     xs = np.linspace(-20, 20, 2001).astype(np.float32)
     ss = [oracle.score(float(z)) for z in xs]
     assert all(a <= b for a, b in zip(ss, ss[1:]))  # monotone
+
+
+def test_score_matches_high_precision_sigmoid():
+    # 50-digit decimal sigmoid, rounded to double then fp32, on 4000 fp32 logits across the range
+    # where the score is neither 0 nor saturated: the fp64 evaluation with libm exp must give the
+    # same fp32 bits (it could differ only within ~1e-16 relative of an fp32 rounding boundary)
+    from decimal import Decimal, getcontext
+    getcontext().prec = 50
+    rng = np.random.default_rng(17)
+    lg = np.concatenate([rng.normal(0, 3, 3000), rng.uniform(-60, 30, 1000)]).astype(np.float32)
+    for v in lg:
+        exact = Decimal(1) / (Decimal(1) + (-Decimal(float(v))).exp())
+        assert np.float32(float(exact)) == np.float32(oracle.score(float(v))), float(v)
+
+
+def test_oracle_threads_do_not_change_any_bit(tmp_path):
+    # the OpenMP row loops (the timed CPU baseline uses every core) give the same bits as one thread
+    import subprocess
+    import sys
+    w = synth.WORKLOADS["mid_b2"]
+    W = synth.layer_weights(w, 0)
+    x = synth.tokens(w, batch=5)
+    many = oracle.step(w.dims, W, x)
+    assert oracle.threads() > 1 or os.cpu_count() == 1
+    code = ("import sys, numpy as np; sys.path.insert(0, %r); import oracle, synth; "
+            "w = synth.WORKLOADS['mid_b2']; r = oracle.step(w.dims, synth.layer_weights(w, 0), synth.tokens(w, batch=5)); "
+            "assert oracle.threads() == 1; np.savez(%r, **r)") % (ROOT, str(tmp_path / "one.npz"))
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    subprocess.check_call([sys.executable, "-c", code], env=env)
+    one = np.load(tmp_path / "one.npz")
+    for k in many:
+        assert np.array_equal(many[k], one[k]), k
 
 
 def _brute_topk(scores, k):

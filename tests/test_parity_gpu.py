@@ -11,8 +11,8 @@ import pytest
 
 import oracle
 import synth
-from tests.harness import (assert_close, assert_logits_match, bf16_tensor_to_f32, layer_dims, rel_errors, run_layer,
-                           to_device, upload_weights)
+from tests.harness import (assert_close, assert_logits_match, bf16_tensor_to_f32, layer_dims, oracle_scores, rel_errors,
+                           run_layer, set_config, to_device, upload_weights)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,23 +37,40 @@ def _make_layer(w, W_dev, max_batch, flags=None, schedule="fused"):
     return MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=max_batch, flags=f)
 
 
-def _check_step(w, W, x, layer, tokens=None, check_all_routing=True):
+_ORACLE_CACHE: dict = {}
+
+
+def _oracle_all(w, W, x, layer_idx=0):
+    """oracle.step over every token of x, cached (the oracle does not depend on the schedule)."""
+    key = (w.name, w.dims, layer_idx, x.shape, hash(x.tobytes()), hash(W["router"].tobytes()))
+    if key not in _ORACLE_CACHE:
+        if len(_ORACLE_CACHE) > 8:
+            _ORACLE_CACHE.clear()
+        _ORACLE_CACHE[key] = oracle.step(w.dims, W, x)
+    return _ORACLE_CACHE[key]
+
+
+def _check_step(w, W, x, layer, tokens=None, check_all_routing=True, label=None, layer_idx=0):
     out, idx, wts, taps = run_layer(layer, x)
     B = x.shape[0]
+    set_config(label or f"{w.name} B{B}")
     if check_all_routing:
         lg, ridx, rw = oracle.route(W["router"], x, w.dims.top_k)
         assert np.array_equal(idx, ridx), "routing indices differ from the oracle"
         np.testing.assert_allclose(wts, rw, rtol=2e-6, atol=0)
         assert_logits_match(taps["logits"], lg)
+        # every score the top-k ranked by: CUDA exp(double) against libm exp on the same logits
+        assert np.array_equal(taps["scores"].view(np.uint32), oracle_scores(taps["logits"]).view(np.uint32)), \
+            "fp32 scores differ from the oracle's"
     toks = range(B) if tokens is None else tokens
+    r = _oracle_all(w, W, x, layer_idx)
     for t in toks:
-        r = oracle.step(w.dims, W, x, tokens=range(t, t + 1))
-        assert np.array_equal(idx[t], r["idx"][0])
-        assert_close(taps["h"][t], r["h"][0], f"h[{t}]")
-        assert_close(taps["ylat"][t], r["ylat"][0], f"ylat[{t}]")
-        assert_close(taps["sh"][t], r["sh"][0], f"sh[{t}]")
-        assert_close(taps["up"][t], r["out"][0] - r["sh"][0], f"up[{t}]")
-        assert_close(out[t], r["out"][0], f"out[{t}]")
+        assert np.array_equal(idx[t], r["idx"][t])
+        assert_close(taps["h"][t], r["h"][t], f"h[{t}]")
+        assert_close(taps["ylat"][t], r["ylat"][t], f"ylat[{t}]")
+        assert_close(taps["sh"][t], r["sh"][t], f"sh[{t}]")
+        assert_close(taps["up"][t], r["out"][t] - r["sh"][t], f"up[{t}]")
+        assert_close(out[t], r["out"][t], f"out[{t}]")
     return out, idx
 
 
@@ -72,7 +89,7 @@ def test_mid_parity(mid, B, schedule):
     w, W, W_dev = mid
     x = synth.tokens(w, batch=B)
     layer = _make_layer(w, W_dev, max_batch=B, schedule=schedule)
-    _check_step(w, W, x, layer)
+    _check_step(w, W, x, layer, label=f"mid B{B} {schedule}")
     if schedule == "stream":
         assert layer.kernels_per_step(B) == 4  # the streaming kernel ran (4 launches per step)
 
@@ -135,7 +152,7 @@ def test_tiny_parity(tiny, B, schedule):
     w, W, W_dev = tiny
     layer = _make_layer(w, W_dev, max_batch=64, schedule=schedule)
     x = synth.tokens(w, step=B, batch=B)
-    _check_step(w, W, x, layer)
+    _check_step(w, W, x, layer, label=f"tiny B{B} {schedule}")
 
 
 @pytest.mark.parametrize("schedule", SCHEDULES)
@@ -316,27 +333,63 @@ def test_full_small_batches_all_tokens(full_layers, name, schedule):
     w, W, W_dev = full_layers(name)
     layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
     x = synth.tokens(w)
-    out, idx = _check_step(w, W, x, layer)
+    out, idx = _check_step(w, W, x, layer, label=f"{name} L0 {schedule}")
     if name == "full_b2":
         assert 0 < len(set(idx[0]) & set(idx[1])) < w.dims.top_k
 
 
-@pytest.mark.parametrize("schedule", SCHEDULES)
-def test_full_b16_sampled_tokens(full_layers, schedule):
-    w, W, W_dev = full_layers("full_b16")
+# Above two tokens the streaming schedule is the split-K kernel too, so B >= 16 runs the fused
+# split-K kernel and the multi-kernel schedule; layer 15 and 31 as well as 0 (distinct weights).
+LARGE_CASES = [(l, s) for l in (0, 15, 31) for s in ("fused", "multi")]
+
+
+@pytest.mark.parametrize("layer_idx,schedule", LARGE_CASES)
+def test_full_b16_all_tokens(full_layers, layer_idx, schedule):
+    w, W, W_dev = full_layers("full_b16", layer_idx)
     layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
     x = synth.tokens(w)
-    _check_step(w, W, x, layer, tokens=[0, 7, 15])
+    _check_step(w, W, x, layer, label=f"full_b16 L{layer_idx} {schedule}", layer_idx=layer_idx)
 
 
-@pytest.mark.parametrize("schedule", SCHEDULES)
-@pytest.mark.parametrize("layer_idx", [0, 31])
-def test_full_b64_skewed_sampled_tokens(full_layers, layer_idx, schedule):
+@pytest.mark.parametrize("layer_idx,schedule", LARGE_CASES)
+def test_full_b64_skewed_all_tokens(full_layers, layer_idx, schedule):
     w, W, W_dev = full_layers("full_b64_skewed", layer_idx)
     layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
     x = synth.tokens(w)
-    _, ridx_all = oracle.route(W["router"], x, w.dims.top_k)[0], oracle.route(W["router"], x, w.dims.top_k)[1]
-    # sample the token with the most hot selections, one with none, and the last token
-    hot = np.isin(ridx_all, synth.hot_set(w, layer_idx)).sum(axis=1)
-    sample = sorted({int(np.argmax(hot)), int(np.argmin(hot)), w.batch - 1})
-    _check_step(w, W, x, layer, tokens=sample)
+    _, idx = _check_step(w, W, x, layer, label=f"full_b64_skewed L{layer_idx} {schedule}", layer_idx=layer_idx)
+    # the skew is there: about half of all selections go to the 32 hot experts
+    share = np.isin(idx, synth.hot_set(w, layer_idx)).mean()
+    assert 0.3 < share < 0.7, share
+
+
+# ---- one expert with many tokens: every token group and operand path of the expert items ------
+
+def _tiny_skewed(B, hot, beta, seed):
+    return synth.Workload(f"tiny_hot{hot}_b{B}", synth.TINY, B, seed, hot_experts=hot, hot_beta=beta)
+
+
+@pytest.mark.parametrize("schedule", ["fused", "multi"])
+def test_tiny_hot_experts_token_groups(torch_cuda, schedule):
+    # 8 hot experts of 64 at B = 64 (k = 4, beta = 4): experts take 1..4, 5..8, 9..16 and 17..32
+    # tokens, so an expert item runs one or two 16-token groups on either operand path
+    w = _tiny_skewed(64, 8, 4.0, 3100)
+    W = synth.layer_weights(w, 0)
+    x = synth.tokens(w)
+    _, ridx, _ = oracle.route(W["router"], x, w.dims.top_k)
+    c = np.bincount(ridx.ravel(), minlength=w.dims.n_experts)
+    for lo, hi in ((1, 4), (5, 8), (9, 16), (17, 32)):
+        assert ((c >= lo) & (c <= hi)).any(), (lo, hi, c)
+    layer = _make_layer(w, upload_weights(W), max_batch=64, schedule=schedule)
+    _check_step(w, W, x, layer, label=f"tiny hot8 B64 {schedule}")
+
+
+@pytest.mark.parametrize("B", [17, 64])
+@pytest.mark.parametrize("schedule", ["fused", "multi"])
+def test_tiny_identical_tokens_one_expert_takes_every_token(tiny, B, schedule):
+    # B copies of one token: each of its k experts receives all B tokens (the largest bucket: up
+    # to four 16-token groups of one expert item)
+    w, W, W_dev = tiny
+    x = np.repeat(synth.tokens(w, step=11, batch=1), B, axis=0)
+    layer = _make_layer(w, W_dev, max_batch=64, schedule=schedule)
+    out, idx = _check_step(w, W, x, layer, label=f"tiny identical B{B} {schedule}")
+    assert (idx == idx[0]).all()
