@@ -11,7 +11,8 @@ CUDA graph of exactly K steps that cycles through `--layers` layers of distinct 
 time is the median of `--reps` (5) such regions, each bracketed by a synchronise (and a barrier
 under torchrun); every layer's device error word is read after them, so a step that gave up on
 a bounded wait fails the run instead of being timed.  The headline is `--workload` (full_b1);
-`per_config` repeats the measurement for the metric's other batches (B = 2, 16, 64), each over
+`per_config` repeats the measurement for the metric's other batches (B = 2, 16, 64) and for a
+speculative-decoding batch (B = 256 = 32 sequences x 8 tokens), each over
 32 layers of its own weights.  Rank 0 prints one JSON line.  Under torchrun every rank runs an
 independent replica (the step does not shard; no collective touches the data path); value =
 all ranks' steps / max time.
@@ -39,7 +40,7 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "MoE layer-steps/s & µs/step at B=1..64; achieved HBM GB/s vs B200 peak"
-PER_CONFIG = ("full_b1", "full_b2", "full_b16", "full_b64_skewed")  # the metric's batches
+PER_CONFIG = ("full_b1", "full_b2", "full_b16", "full_b64_skewed", "full_b256")  # the metric's batches, and a speculative-decoding batch
 UNIT = "layer-steps/s"
 
 
@@ -377,8 +378,23 @@ class Timed:
         ms = max_over_ranks(statistics.median(times), self.dist, self.device)
         return ms, times, clk.summary()
 
+    def run_hinted(self, reps, local_rank):
+        """The same measurement with the cross-layer prefetch hint set: layer l's steps prefetch the
+        router of layer l + 1 (the one the graph steps next).  The hints are cleared afterwards."""
+        n = len(self.layers)
+        for l, L_ in enumerate(self.layers):
+            L_.set_next(self.layers[(l + 1) % n])
+        self.g_warm, self.g_main = self.capture(max(self.warmup, 1), 0), self.capture(self.steps, self.warmup)
+        try:
+            return self.run(reps, local_rank)
+        finally:
+            for L_ in self.layers:
+                L_.set_next(None)
+            self.g_warm, self.g_main = self.capture(max(self.warmup, 1), 0), self.capture(self.steps, self.warmup)
+
     def close(self):
         del self.g_main, self.g_warm
+        self.layers = self.x = self.out = None
 
 
 def unique_experts(layers, x, out, stream, B):
@@ -394,15 +410,22 @@ def unique_experts(layers, x, out, stream, B):
     return float(np.mean(uniq))
 
 
-def config_entry(w, ms, times, clocks, steps, world, unique_mean, peak):
-    """One per_config record: time per step, throughput, algorithmic bytes and their HBM fraction."""
+def config_entry(w, ms, times, clocks, steps, world, unique_mean, peak, hinted=None):
+    """One per_config record: time per step, throughput, algorithmic bytes and their HBM fraction;
+    `hinted` = (ms, times, clocks) of the same steps with the cross-layer prefetch hint."""
     ms_per_step = ms / steps
     sb = step_bytes(w.dims, unique_mean, w.batch)
-    return {"workload": w.name, "batch": w.batch, "us_per_step": 1e3 * ms_per_step,
-            "layer_steps_per_s": replica_throughput(world, steps, ms), "unique_experts_per_step": unique_mean,
-            "bytes_per_step": sb, "hbm_gbs": sb / (ms_per_step / 1e3) / 1e9,
-            "hbm_frac": sb / (ms_per_step / 1e3) / 1e9 / peak,
-            "replay_ms": [round(t, 4) for t in times], "clocks": clocks}
+    r = {"workload": w.name, "batch": w.batch, "us_per_step": 1e3 * ms_per_step,
+         "layer_steps_per_s": replica_throughput(world, steps, ms), "unique_experts_per_step": unique_mean,
+         "bytes_per_step": sb, "hbm_gbs": sb / (ms_per_step / 1e3) / 1e9,
+         "hbm_frac": sb / (ms_per_step / 1e3) / 1e9 / peak,
+         "replay_ms": [round(t, 4) for t in times], "clocks": clocks}
+    if hinted:
+        hms = hinted[0] / steps
+        r["next_layer_hint"] = {"us_per_step": 1e3 * hms, "layer_steps_per_s": replica_throughput(world, steps, hinted[0]),
+                                "hbm_frac": sb / (hms / 1e3) / 1e9 / peak, "replay_ms": [round(t, 4) for t in hinted[1]],
+                                "clocks": hinted[2]}
+    return r
 
 
 def main():
@@ -434,6 +457,7 @@ def main():
 
     tm = Timed(layers, x, out, stream, args.steps, args.warmup, dist, device)
     ms, times, clocks = tm.run(args.reps, local_rank)
+    hinted = tm.run_hinted(args.reps, local_rank)
     ms_per_step = ms / args.steps
     value = replica_throughput(world, args.steps, ms)
     kps = layers[0].kernels_per_step(B)
@@ -490,7 +514,7 @@ def main():
     check_device_errors(layers, B, stream)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     e2e_value = replica_throughput(world, args.steps, e2e_ms)
-    per_config = {w.name: config_entry(w, ms, times, clocks, args.steps, world, unique_mean, peak)}
+    per_config = {w.name: config_entry(w, ms, times, clocks, args.steps, world, unique_mean, peak, hinted)}
     tm.close()
     for L_ in layers:
         L_.close()
@@ -509,7 +533,8 @@ def main():
             uc = unique_experts(lc, xc, oc, stream, wc.batch)
             tc = Timed(lc, xc, oc, stream, args.steps, args.warmup, dist, device)
             mc, tsc, cc = tc.run(args.reps, local_rank)
-            per_config[name] = config_entry(wc, mc, tsc, cc, args.steps, world, uc, peak)
+            hc = tc.run_hinted(args.reps, local_rank)
+            per_config[name] = config_entry(wc, mc, tsc, cc, args.steps, world, uc, peak, hc)
             tc.close()
             for L_ in lc:
                 L_.close()

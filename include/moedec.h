@@ -85,7 +85,7 @@ typedef struct moedec_config {
     int32_t expert_inter; /* I: multiple of 128 */
     int32_t shared_inter; /* I_s: multiple of 128 (ignored when n_shared == 0) */
     int32_t n_shared;     /* 0 or 1 shared expert */
-    int32_t max_batch;    /* largest B a step will be called with: 1..64 */
+    int32_t max_batch;    /* largest B a step will be called with: 1..512, and max_batch * top_k <= 8192 */
     uint32_t flags;       /* MOEDEC_FLAG_* */
 } moedec_config;
 
@@ -141,6 +141,21 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
 
 /* Release the workspace, side stream and events (synchronises the side stream). NULL is a no-op. */
 MOEDEC_API int moedec_destroy(moedec_handle *h);
+
+/*
+ * Cross-layer prefetch hint.  Decode runs the layers one after another, and the next layer's
+ * router matrix (E x H bf16) is the first thing its step reads, at the head of its dependency
+ * chain.  With next set, every later fused step of h (the default schedules; the streaming and
+ * multi-kernel schedules ignore the hint) has CTAs that have run out of work issue L2
+ * prefetches of next's router rows (cp.async.bulk.prefetch.L2, no data returned to the SM), so
+ * that the next layer's step starts on L2 hits ("快是可以生成的，可信只能证明（vLLM 重写 Kimi K3
+ * 解码路径…）", section 他们换掉了什么: the next weights are prefetched into cache while the
+ * current step waits).  Results never depend on the hint.
+ *   next  a handle on the same device with the same hidden and n_experts, or NULL to clear the
+ *         hint; only its router pointer is recorded, so it must stay valid while h keeps it.
+ * Errors: INVALID_ARG (NULL h, mismatched next).
+ */
+MOEDEC_API int moedec_set_next(moedec_handle *h, const moedec_handle *next);
 
 /*
  * Routing of the last step, copied on `stream` into caller device buffers:

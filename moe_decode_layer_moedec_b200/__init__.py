@@ -66,6 +66,8 @@ def _load():
     lib.moedec_get_routing.restype = i32
     lib.moedec_get_taps.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp]
     lib.moedec_get_taps.restype = i32
+    lib.moedec_set_next.argtypes = [vp, vp]
+    lib.moedec_set_next.restype = i32
     lib.moedec_get_scores.argtypes = [vp, vp, i32, vp]
     lib.moedec_get_scores.restype = i32
     lib.moedec_get_launch_counts.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(i32)]
@@ -178,6 +180,11 @@ class MoeDecodeLayer:
                                                            _ptr(r["sh"]), _ptr(r.get("up")), batch, _stream_ptr(stream)))
         return r
 
+    def set_next(self, nxt: "MoeDecodeLayer | None"):
+        """Prefetch hint: steps of this layer pull `nxt`'s router rows into L2 (None clears it)."""
+        self._next = nxt  # keep the next layer's handle (and its router tensor) alive
+        self._check("moedec_set_next", lib.moedec_set_next(self._h, nxt._h if nxt is not None else None))
+
     def scores(self, batch: int, stream=None):
         """fp32 router scores [B, E] of the last step, from the same device function the top-k uses."""
         import torch
@@ -218,9 +225,12 @@ class MoeDecodeLayer:
         return int(lib.moedec_kernels_per_step(self._h, batch))
 
     def close(self):
+        """Destroy the handle and drop the references to the weight tensors and the hinted layer."""
         if getattr(self, "_h", None):
             lib.moedec_destroy(self._h)
             self._h = None
+        self._weights = None
+        self._next = None
 
     def __del__(self):
         try:

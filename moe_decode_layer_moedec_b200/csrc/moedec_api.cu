@@ -25,6 +25,7 @@ struct moedec_handle {
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     int device = 0, n_sm = 0;
     int last_batch = 0;
+    const uint16_t *next_router = nullptr;  // moedec_set_next
     uint64_t launches[2] = {0, 0};
     char cuda_error[256] = {0};
     // per-kernel event timing (moedec_profile_enable)
@@ -229,7 +230,8 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
         (c.n_shared != 0 && c.n_shared != 1) || (c.n_shared && c.shared_inter <= 0))
         return MOEDEC_ERR_INVALID_ARG;
     if (c.hidden % 128 || c.latent % 128 || c.expert_inter % 128 || (c.n_shared && c.shared_inter % 128) ||
-        c.n_experts > kMaxExperts || c.top_k > c.n_experts || c.top_k > kMaxTopK || c.max_batch > kMaxBatch)
+        c.n_experts > kMaxExperts || c.top_k > c.n_experts || c.top_k > kMaxTopK || c.max_batch > kMaxBatch ||
+        c.max_batch * c.top_k > kMaxEntries)
         return MOEDEC_ERR_UNSUPPORTED;
     const void *ptrs[] = {w->router, w->w_down_lat, w->w_up_lat, w->gate_q, w->gate_s, w->up_q, w->up_s, w->down_q, w->down_s};
     for (const void *p : ptrs)
@@ -337,6 +339,7 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     a.w = h->w;
     a.ws = h->ws;
     a.p = h->p;
+    a.next_router = h->next_router;
     a.x = x;
     a.out = out;
     a.B = batch;
@@ -372,6 +375,13 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     if (e != cudaSuccess) return record_cuda(h, e);
     h->launches[variant] += (uint64_t)kernels_per_step(h->d);
     h->last_batch = batch;
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_set_next(moedec_handle *h, const moedec_handle *next) {
+    if (!h) return MOEDEC_ERR_INVALID_ARG;
+    if (next && (next->d.H != h->d.H || next->d.E != h->d.E || next->device != h->device)) return MOEDEC_ERR_INVALID_ARG;
+    h->next_router = next ? next->w.router : nullptr;
     return MOEDEC_OK;
 }
 

@@ -8,9 +8,9 @@
 //   1 top-k, one per token     waits: all router blocks            CTA items; last builds buckets
 //   2 W_dn row blocks          (h)                                 CTA items
 //   3 shared gate/up blocks    (sh_a)                              CTA items
-//   4 expert gate/up, 16 rows  waits: buckets, all of h            warp items
+//   4 expert gate/up           waits: buckets, all of h            static per-CTA segments
 //   5 shared down blocks       waits: all of sh_a                  CTA items
-//   6 expert down, 16 rows     waits: that expert's gate/up items  warp items; w * y added into ylat
+//   6 expert down              waits: that expert's gate/up tiles  static per-CTA segments; w * y added into ylat
 //   7 W_up row blocks          waits: their ylat rows, all of sh   CTA items; writes out
 //
 // An item only ever waits on items of earlier queues (all of which were claimed by resident CTAs
@@ -21,7 +21,7 @@
 // Routing is known only after queue 1, but nothing waits for a kernel boundary: while one CTA
 // ranks the experts the others already stream W_dn and the shared expert, and an expert's down
 // rows start as soon as its own gate/up rows are done.
-#include "moedec_items.cuh"
+#include "moedec_experts.cuh"
 
 namespace moedec {
 
@@ -39,8 +39,11 @@ template <> struct Tier<4> { static constexpr int NTX = 8, NTS = 8, NTU = 16; st
 
 __host__ __device__ inline int tier_for_batch(int B) { return B <= 4 ? 0 : B <= 8 ? 1 : B <= 16 ? 2 : B <= 32 ? 3 : 4; }
 
+// Dynamic shared memory: the phases' staging buffers from offset 0 (fused_stage_smem bytes), then
+// the routing tables of the step (they must survive the shared-down staging between the two
+// expert phases).
 template <int TIER>
-__host__ __device__ inline size_t fused_smem(const StepArgs &a) {
+__host__ __device__ inline size_t fused_stage_smem(const StepArgs &a) {
     using T = Tier<TIER>;
     size_t m = (size_t)8 * (a.p.rt.krange + 4) * sizeof(double);
     auto mx = [&](size_t v) { m = v > m ? v : m; };
@@ -48,8 +51,14 @@ __host__ __device__ inline size_t fused_smem(const StepArgs &a) {
     mx((size_t)8 * T::NTX * f16_pitch(a.p.sgu.krange) * 2);
     mx((size_t)8 * T::NTS * f16_pitch(a.p.sd.krange) * 2);
     mx((size_t)8 * T::NTU * bf16_pitch(up_chunk(T::NTU, a.p.up.krange)) * 2);
-    mx((size_t)8 * expert_warp_smem(a.B));
-    return m;
+    mx(seg_smem(a.d));
+    mx((size_t)a.d.E * ((a.B + 63) / 64) * 8);  // the bucket builder's token masks (B > 64)
+    return (m + 15) & ~(size_t)15;
+}
+
+template <int TIER>
+__host__ __device__ inline size_t fused_smem(const StepArgs &a) {
+    return fused_stage_smem<TIER>(a) + sizeof(SplitKRoute);
 }
 
 template <int TIER>
@@ -59,13 +68,12 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
     __shared__ TopkSmem topk;
     __shared__ unsigned s_flag;
     __shared__ int s_ok;
-    __shared__ int s_ent[8][kExpertTokGroup];
-    __shared__ int s_shift[8][kExpertTokGroup];
-    __shared__ float s_w[8][kExpertTokGroup];
-    __shared__ SplitKRoute route;
+    SplitKRoute &route = *reinterpret_cast<SplitKRoute *>(smem + fused_stage_smem<TIER>(a));
+    __shared__ SegPlan segp;
+    __shared__ SegSmem segs;
+    __shared__ int s_scan[32];
     __shared__ int s_next;
     unsigned *ctl = a.ws.ctl;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     bool alive = true;
     const int n_rt = a.p.rt.blocks * a.p.rt.splits, n_dn = a.p.dn.blocks * a.p.dn.splits;
     const int n_sgu = a.d.n_shared ? a.p.sgu.blocks * a.p.sgu.splits : 0;
@@ -96,30 +104,16 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
             it = nxt;
         }
     };
-    auto warp_queue = [&](int q, int n, bool down, auto body) {
-        int it = 0;
-        if (lane == 0) it = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
-        it = __shfl_sync(0xffffffffu, it, 0);
-        if (it < n) warp_prefetch_expert(a, it, down);
-        int ok = 1;
-        while (ok && it < n) {
-            int nxt = 0;
-            if (lane == 0) nxt = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
-            nxt = __shfl_sync(0xffffffffu, nxt, 0);
-            if (nxt < n) warp_prefetch_expert(a, nxt, down);
-            ok = body(it) ? 1 : 0;
-            it = nxt;
-        }
-        return ok;
-    };
-
     // 0: router
     cta_queue(Q_ROUTER, n_rt, [&](int it) { prefetch_router(a, it); },
               [&](int it) { item_router<true>(a, it, smem, &s_flag); return true; });
     stamp(1);
     // 1: top-k
     cta_queue(Q_TOPK, a.B, [](int) {},
-              [&](int it) { return item_topk<true>(a, it, topk, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat); });
+              [&](int it) {
+                  return item_topk<true>(a, it, topk, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat, nullptr,
+                                         reinterpret_cast<unsigned long long *>(smem));
+              });
     stamp(2);
     // 2: W_dn
     cta_queue(Q_DN, n_dn, [&](int it) { prefetch_dn(a, it); },
@@ -129,34 +123,48 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
     cta_queue(Q_SGU, n_sgu, [&](int it) { prefetch_sgu(a, it); },
               [&](int it) { item_sgu<true, T::NTX>(a, it, smem, &s_flag); return true; });
     stamp(4);
-    // 4: expert gate/up (warp items): routing and all of h must be final
+    // 4: expert gate/up: routing and all of h must be final; the CTA's static range of the
+    // (slot, token group, 128-row block) items, one activation staging per segment
     if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
     if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)a.p.dn.blocks, &s_ok);
     stamp(5);
+    auto range = [&](int n, int &lo, int &hi) {
+        lo = (int)((long long)n * blockIdx.x / gridDim.x);
+        hi = (int)((long long)n * (blockIdx.x + 1) / gridDim.x);
+    };
+    uint16_t *xs_e = reinterpret_cast<uint16_t *>(smem);
     if (alive) {
         cta_load_routing(a, route);
         __syncthreads();
-        const int n = route.n_active * (a.d.I / 16);
-        uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)warp * expert_warp_smem(a.B));
-        warp_queue(Q_EGU, n, false,
-                   [&](int it) { return warp_expert_item<true, false>(a, xs, it, s_ent[warp], s_shift[warp], &route); });
+        seg_plan(segp, route, s_scan);
+        __syncthreads();
+        const int nb = a.d.I / 128;
+        int lo, hi;
+        range(nb * segp.ngroups, lo, hi);
+        for_each_segment(segp, route, nb, lo, hi, [&](int j, int g, int b0, int b1) {
+            seg_gate_up_any(a, route, segs, xs_e, j, g, b0, b1);
+            return true;
+        });
     }
     stamp(6);
     // 5: shared down
     cta_queue(Q_SD, n_sd, [&](int it) { prefetch_sd(a, it); },
               [&](int it) { return item_sd<true, T::NTS, T::SPLITS>(a, it, smem, &s_flag, &s_ok); });
     stamp(7);
-    // 6: expert down (warp items), each waits on its expert's gate/up rows
+    // 6: expert down: the same plan over L / 128 blocks per expert; each segment waits for its
+    // expert's gate/up tiles
     if (alive) {
         __syncthreads();
-        const int n = route.n_active * (a.d.L / 16);
-        uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)warp * expert_warp_smem(a.B));
-        const int ok = warp_queue(Q_EDOWN, n, true, [&](int it) {
-            return warp_expert_item<true, true>(a, xs, it, s_ent[warp], s_shift[warp], &route, s_w[warp]);
+        const int nb = a.d.L / 128;
+        int lo, hi;
+        range(nb * segp.ngroups, lo, hi);
+        const bool ok = for_each_segment(segp, route, nb, lo, hi, [&](int j, int g, int b0, int b1) {
+            return seg_down_any(a, route, segs, xs_e, j, g, b0, b1);
         });
-        alive = __syncthreads_and(ok) != 0;
+        alive = __syncthreads_and(ok ? 1 : 0) != 0;
     }
     stamp(8);
+    if (alive) prefetch_next_router(a, blockIdx.x, gridDim.x);
     // 7: W_up and the output
     cta_queue(Q_UP, n_up, [&](int it) { prefetch_up(a, it); },
               [&](int it) { return item_up<true, T::NTU>(a, it, smem, &s_flag, &s_ok); });

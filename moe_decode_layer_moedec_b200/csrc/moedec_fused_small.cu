@@ -19,7 +19,7 @@
 //   expert g/u   16 rows of one expert   waits: buckets, all of h     -> a rows, max |a|
 //   expert down  16 rows of one expert   waits: its g/u rows          -> w * y rows added into ylat
 //                                                                        (fp32 reductions)
-//   W_up         16 rows x K/4           waits: ylat, sh              -> out rows
+//   W_up         16 rows x K/4           waits: ylat (sh: a tile's last split) -> out rows
 // and the shared expert (an eighth of the grid) runs beside it:
 //   shared g/u   16 rows x K/8, g and u  MXFP4, x staged as fp16      -> sh_a rows, max |sh_a|
 //   shared down  16 rows x K             waits: all of sh_a           -> sh rows
@@ -452,8 +452,9 @@ DEVI bool w_edown(const StepArgs &a, const RouteSmem &rt, int item, uint16_t *ws
     return true;
 }
 
-// W_up: 16 rows x K/s_up; ylat staged as bf16 hi/lo columns (2b, 2b+1); out = bf16(. + sh)
-DEVI void w_up(const StepArgs &a, int item, const uint16_t *ys) {
+// W_up: 16 rows x K/s_up; ylat staged as bf16 hi/lo columns (2b, 2b+1); out = bf16(. + sh).
+// Returns false if the step was aborted while the tile's last split waited for sh.
+DEVI bool w_up(const StepArgs &a, int item, const uint16_t *ys) {
     const int H = a.d.H, L = a.d.L, B = a.B, maxB = a.d.max_batch;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int tile = item / a.p.s_up, ks = item % a.p.s_up, row0 = tile * 16;
@@ -466,7 +467,10 @@ DEVI void w_up(const StepArgs &a, int item, const uint16_t *ys) {
         part[(size_t)q * H + row0 + g + 8] = acc[2] + acc[3];
     }
     const int tk = a.p.ctl_tk + (a.d.E + 7) / 8 + a.d.L / 16 + a.d.Is / 16 + a.d.H / 16 + tile;
-    if (!warp_ticket_last(a.ws.ctl + tk, a.p.s_up)) return;
+    if (!warp_ticket_last(a.ws.ctl + tk, a.p.s_up)) return true;
+    // only the warp that completes the tile adds the shared expert's rows: the rest of W_up
+    // streams while the shared expert finishes
+    if (a.d.n_shared && !warp_wait_geq(a, a.ws.ctl + CTL_SD_DONE, (unsigned)(H / 16))) return false;
     if (q < B)
         for (int h2 = 0; h2 < 2; ++h2) {
             const int r = row0 + g + 8 * h2;
@@ -475,6 +479,34 @@ DEVI void w_up(const StepArgs &a, int item, const uint16_t *ys) {
             const float shv = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)q * H + r) : 0.0f;
             a.out[(size_t)q * H + r] = f32_to_bf16_rne(s + shv);
         }
+    return true;
+}
+
+// ---------------------------------------------------------------------------------------------
+// L2 prefetch of a CTA's own later weights while it waits.  Item ranges are static ([n c / G,
+// n (c+1) / G) of each queue), so a CTA knows which W_up rows it will read before its chain gets
+// there, and which expert down rows as soon as the routing is out.  The bytes move while the SM
+// would otherwise idle in a wait; the later phase then reads them from L2.
+
+// W_up items of CTA c of the G chain CTAs: 16 rows x L / s_up, one row segment per thread
+DEVI void prefetch_up_range(const StepArgs &a, int c, int G) {
+    const int n = a.d.H / 16 * a.p.s_up, lo = (int)((long long)n * c / G), hi = (int)((long long)n * (c + 1) / G);
+    const int KW = a.d.L / a.p.s_up;
+    for (int i = threadIdx.x; i < (hi - lo) * 16; i += blockDim.x) {
+        const int it = lo + i / 16, r = i % 16, tile = it / a.p.s_up, ks = it % a.p.s_up;
+        prefetch_l2(a.w.w_up + (size_t)(tile * 16 + r) * a.d.L + (size_t)ks * KW, (uint32_t)KW * 2);
+    }
+}
+
+// expert down items of CTA c: 16 contiguous rows (whole K) of one active expert, codes and scales
+DEVI void prefetch_edown_range(const StepArgs &a, const RouteSmem &rt, int c, int G) {
+    const int L = a.d.L, I = a.d.I, tiles = L / 16;
+    const int n = rt.n_active * tiles, lo = (int)((long long)n * c / G), hi = (int)((long long)n * (c + 1) / G);
+    for (int i = threadIdx.x; i < 2 * (hi - lo); i += blockDim.x) {
+        const int it = lo + i / 2, e = rt.e[it / tiles], tile = it % tiles;
+        if (i & 1) prefetch_l2(a.w.down_s + ((size_t)e * L + (size_t)tile * 16) * (I / 32), 16 * (I / 32));
+        else prefetch_l2(a.w.down_q + ((size_t)e * L + (size_t)tile * 16) * (I / 2), 16 * (I / 2));
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -495,8 +527,8 @@ __host__ __device__ inline size_t fused_small_smem(const StepArgs &a) {
 __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ TopkSmem topk;
-    __shared__ int s_shift[kMaxBatch], s_ok;
-    __shared__ unsigned s_amax[kMaxBatch];
+    __shared__ int s_shift[kSmallMaxBatch], s_ok;
+    __shared__ unsigned s_amax[kSmallMaxBatch];
     __shared__ CtaTake claim;
     __shared__ RouteSmem route;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
@@ -575,6 +607,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
             warp_queue(QS_SD, n_sd, c_sh, G_sh, [&](int it) { w_sd(a, it, xs, s_shift); return true; });
         }
         stamp(7);
+        prefetch_next_router(a, c_sh, G_sh);  // nothing left to do here: pull the next layer's router
     } else {
         // ---- routed chain CTAs ----
         // router and W_dn read x as bf16
@@ -590,6 +623,8 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         if (alive && c_m >= n_tk)
             warp_queue(QS_DN, n_dn, c_m - n_tk, G_m - n_tk, [&](int it) { w_dn(a, it, xs); return true; });
         stamp(3);
+        // W_up rows of this CTA into L2 while the routing is computed
+        if (alive) prefetch_up_range(a, c_m, G_m);
         // expert gate/up: routing and all of h final; stage h of every token (fp16 hi/lo)
         if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
         stamp(11);
@@ -599,6 +634,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
             if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
             cta_load_routing(a, route);
             __syncthreads();
+            prefetch_edown_range(a, route, c_m, G_m);  // this CTA's expert down rows, during gate/up
             stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, B, [](int t) { return t; }, s_shift, 0, L);
             __syncthreads();
             const int n = route.n_active * (I / 16) * a.p.s_egu;
@@ -614,19 +650,18 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
             alive = __syncthreads_and(ok) != 0;
         }
         stamp(8);
-        // W_up: every ylat block complete (all B*k entries added), and all of sh; stage ylat
-        // (bf16 hi/lo)
+        // W_up: every ylat block complete (all B*k entries added); stage ylat (bf16 hi/lo).  The
+        // shared expert's sh is awaited only by the warp that completes each tile
         if (alive) {
             int ok = 1;
             for (int blk = threadIdx.x; blk < L / 16; blk += blockDim.x)
                 ok &= wait_geq(a, ctl + a.p.ctl_ylat + blk, (unsigned)(B * a.d.k)) ? 1 : 0;
-            if (threadIdx.x == 0 && a.d.n_shared) ok &= wait_geq(a, ctl + CTL_SD_DONE, (unsigned)(H / 16)) ? 1 : 0;
             __threadfence();
             alive = __syncthreads_and(ok) != 0;
             if (alive) {
                 stage_bf16split_from_f32(xs, bf16_pitch(L), a.ws.ylat, L, B, 0, L);
                 __syncthreads();
-                warp_queue(QS_UP, n_up, c_m, G_m, [&](int it) { w_up(a, it, xs); return true; });
+                warp_queue(QS_UP, n_up, c_m, G_m, [&](int it) { return w_up(a, it, xs); });
             }
         }
     }

@@ -6,8 +6,9 @@
 
 namespace moedec {
 
-constexpr int kMaxBatch = 64;      // token masks of the routing buckets are one 64-bit word
+constexpr int kMaxBatch = 512;     // tokens per step (speculative decoding: batch x (drafts + 1))
 constexpr int kMaxTopK = 32;
+constexpr int kMaxEntries = 8192;  // tokens x top_k per step (routing tables of a fused step in shared memory)
 constexpr int kMaxExperts = 1024;  // one top-k thread per expert
 constexpr int kDenseWarps = 8;     // dense split-K kernels: 8 warps x 16 rows = 128 rows per CTA
 constexpr int kDenseRows = 128;
@@ -133,6 +134,7 @@ struct Work {
 struct StepArgs {
     Dims d;
     Weights w;
+    const uint16_t *next_router;  // [E][H] router of the layer that steps next (L2 prefetch hint), or nullptr
     Work ws;
     Plan p;
     const uint16_t *x;  // [B][H]

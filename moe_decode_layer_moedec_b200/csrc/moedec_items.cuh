@@ -135,16 +135,20 @@ DEVI void item_dn(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
     const int KR = a.p.dn.krange, k0 = ks * KR;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     const int pitch = bf16_pitch(KR);
-    __syncthreads();
-    stage_bf16(xs, pitch, a.x, H, B, 8 * NT, k0, KR);
-    __syncthreads();
     const int warp = threadIdx.x >> 5;
     const int row0 = rb * kDenseRows + warp * 16;
-    if (row0 < L) {
-        float acc[NT][4] = {};
-        tile_bf16<NT>(a.w.w_dn, H, row0, k0, KR / 32, xs, pitch, 0, B, acc);
-        float *part = a.ws.dn_part + (size_t)ks * maxB * L;
-        tile_foreach<NT, false>(acc, B, [&](int t, int r, float v) { part[(size_t)t * L + row0 + r] = v; });
+    float *part = a.ws.dn_part + (size_t)ks * maxB * L;
+    // token groups of 8 NT columns (one group up to 64 tokens; larger batches re-read the rows)
+    for (int tg = 0; tg < B; tg += 8 * NT) {
+        const int nb = min(8 * NT, B - tg);
+        __syncthreads();
+        stage_bf16(xs, pitch, a.x + (size_t)tg * H, H, nb, 8 * NT, k0, KR);
+        __syncthreads();
+        if (row0 < L) {
+            float acc[NT][4] = {};
+            tile_bf16<NT>(a.w.w_dn, H, row0, k0, KR / 32, xs, pitch, 0, nb, acc);
+            tile_foreach<NT, false>(acc, nb, [&](int t, int r, float v) { part[(size_t)(tg + t) * L + row0 + r] = v; });
+        }
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_dn + rb, a.p.dn.splits, s_flag)) {
         for (int t = threadIdx.x; t < B; t += blockDim.x) s_amax[t] = 0u;
@@ -203,9 +207,11 @@ DEVI unsigned long long warp_take_best(unsigned long long (&w)[N]) {
 // published (the small-batch step adds the expert outputs into ylat).
 // acc64: when given, the logits are the fp64 sums there ([B][E]): they are rounded to fp32 into
 // ws.logits and the accumulator is cleared; otherwise ws.logits already holds them.
+// masks: shared memory for the bucket builder's token masks when B > 64 (E * ceil(B / 64) words);
+// up to 64 tokens the masks are one word per expert in TopkSmem.
 template <bool FUSED>
 DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u, unsigned long long *stamps = nullptr,
-                    float *zero_rows = nullptr, double *acc64 = nullptr) {
+                    float *zero_rows = nullptr, double *acc64 = nullptr, unsigned long long *masks = nullptr) {
     const int E = a.d.E, K = a.d.k, B = a.B;
     if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, rt_done, &t.ok)) return false;
     // optional trace (global ns): logits complete, keys, warp candidates, ranked, routing
@@ -311,14 +317,18 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
         stamp(7);
         return true;
     }
-    // the last token's CTA groups the B*K selections by expert
+    // the last token's CTA groups the B*K selections by expert: one bit per (expert, token) in W
+    // words per expert, so that an expert's entries come out token-ascending (the position of a
+    // selection is the number of lower tokens of its expert)
     if (!cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
+    const int W = (B + 63) / 64;
+    unsigned long long *mk = W == 1 ? t.mask : masks;  // [E][W]
     auto sel_e = [&](int i) { return __ldcg(a.ws.idx + i); };
-    for (int i = tid; i < E; i += blockDim.x) t.mask[i] = 0ull;
+    for (int i = tid; i < E * W; i += blockDim.x) mk[i] = 0ull;
     __syncthreads();
     for (int i = tid; i < B * K; i += blockDim.x) {
-        const int ex = sel_e(i);
-        if (ex >= 0 && ex < E) atomicOr(&t.mask[ex], 1ull << (i / K));
+        const int ex = sel_e(i), tb = i / K;
+        if (ex >= 0 && ex < E) atomicOr(&mk[ex * W + tb / 64], 1ull << (tb % 64));
         else atomicOr(a.ws.err, kErrBucket);
         a.ws.a_amax[i] = 0u;
     }
@@ -328,7 +338,9 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int e = 4 * tid + i;
-        cnt[i] = e < E ? __popcll(t.mask[e]) : 0;
+        cnt[i] = 0;
+        if (e < E)
+            for (int w = 0; w < W; ++w) cnt[i] += __popcll(mk[e * W + w]);
         n_act_t += cnt[i] > 0 ? 1 : 0;
         n_ent_t += cnt[i];
     }
@@ -352,7 +364,10 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
     for (int i = tid; i < B * K; i += blockDim.x) {
         const int ex = sel_e(i), tb = i / K;
         if (ex < 0 || ex >= E) continue;
-        a.ws.entries[t.off[ex] + __popcll(t.mask[ex] & ((1ull << tb) - 1ull))] = i;
+        const unsigned long long *m = mk + ex * W;
+        int pos = t.off[ex] + __popcll(m[tb / 64] & ((1ull << (tb % 64)) - 1ull));
+        for (int w = 0; w < tb / 64; ++w) pos += __popcll(m[w]);
+        a.ws.entries[pos] = i;
     }
     stamp(6);
     if (FUSED) cta_signal_add(a.ws.ctl + CTL_ROUTE_READY, 1u);
@@ -413,7 +428,7 @@ DEVI void cta_load_routing(const StepArgs &a, RouteTables<NEXP, NENT> &r) {
     if (threadIdx.x == 0) r.n_active = __ldcg(a.ws.n_active);
 }
 
-using SplitKRoute = RouteTables<kMaxExperts, kMaxBatch * kMaxTopK>;
+using SplitKRoute = RouteTables<kMaxExperts, kMaxEntries>;
 
 // ---------------------------------------------------------------------------------------------
 // routed experts: one warp = 16 rows of one active expert for up to 16 of its tokens
@@ -604,20 +619,24 @@ DEVI bool item_up(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
         }
         if (!__syncthreads_and(ok)) return false;
     }
-    float acc[NT][4] = {};
-    for (int c0 = k0; c0 < k0 + KR; c0 += kc) {
-        __syncthreads();
-        stage_bf16split_from_f32(xs, pitch, a.ws.ylat, L, B, c0, kc);
-        for (int i = threadIdx.x; i < (8 * NT - 2 * B) * (kc / 8); i += blockDim.x) {  // unused columns
-            const int col = 2 * B + i / (kc / 8), u = i % (kc / 8);
-            *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
+    // token groups of 4 NT tokens (hi/lo column pairs fill the 8 NT columns)
+    for (int tg = 0; tg < B; tg += 4 * NT) {
+        const int nb = min(4 * NT, B - tg);
+        float acc[NT][4] = {};
+        for (int c0 = k0; c0 < k0 + KR; c0 += kc) {
+            __syncthreads();
+            stage_bf16split_from_f32(xs, pitch, a.ws.ylat + (size_t)tg * L, L, nb, c0, kc);
+            for (int i = threadIdx.x; i < (8 * NT - 2 * nb) * (kc / 8); i += blockDim.x) {  // unused columns
+                const int col = 2 * nb + i / (kc / 8), u = i % (kc / 8);
+                *reinterpret_cast<uint4 *>(xs + (size_t)col * pitch + 8 * u) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            __syncthreads();
+            if (row0 < H) tile_bf16<NT>(a.w.w_up, L, row0, c0, kc / 32, xs, pitch, 0, 2 * nb, acc);
         }
-        __syncthreads();
-        if (row0 < H) tile_bf16<NT>(a.w.w_up, L, row0, c0, kc / 32, xs, pitch, 0, 2 * B, acc);
-    }
-    if (row0 < H) {
-        float *part = a.ws.up_part + (size_t)ks * maxB * H;
-        tile_foreach<NT, true>(acc, B, [&](int t, int r, float v) { part[(size_t)t * H + row0 + r] = v; });
+        if (row0 < H) {
+            float *part = a.ws.up_part + (size_t)ks * maxB * H;
+            tile_foreach<NT, true>(acc, nb, [&](int t, int r, float v) { part[(size_t)(tg + t) * H + row0 + r] = v; });
+        }
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_up + rb, a.p.up.splits, s_flag)) {
         if (FUSED && a.d.n_shared && !cta_wait_geq(a, a.ws.ctl + CTL_SD_DONE, (unsigned)a.p.sd.blocks, s_ok)) return false;
@@ -660,21 +679,24 @@ DEVI void item_sgu(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_
     }
     __syncthreads();
     for (int t = threadIdx.x; t < B; t += blockDim.x) s_shift[t] = prescale_shift(__uint_as_float(s_amax[t]));
-    __syncthreads();
-    stage_f16_from_bf16(xs, pitch, a.x, H, B, s_shift, k0, KR);
-    __syncthreads();
     const int warp = threadIdx.x >> 5;
     const int row0 = rb * kDenseRows + warp * 16;
-    if (row0 < Is) {
-        float *part = a.ws.sgu_part + (size_t)ks * maxB * 2 * Is;
+    float *part = a.ws.sgu_part + (size_t)ks * maxB * 2 * Is;
+    for (int tg = 0; tg < B; tg += 8 * NT) {
+        const int nb = min(8 * NT, B - tg);
+        __syncthreads();
+        stage_f16_from_bf16(xs, pitch, a.x + (size_t)tg * H, H, nb, s_shift + tg, k0, KR);
+        __syncthreads();
+        if (row0 < Is) {
 #pragma unroll 1
-        for (int m = 0; m < 2; ++m) {
-            float acc[NT][4] = {};
-            tile_fp4<NT, false>(m ? a.w.sh_up_q : a.w.sh_gate_q, m ? a.w.sh_up_s : a.w.sh_gate_s, nullptr, nullptr, H / 2,
-                                H / 32, row0, k0, KR / 128, xs, pitch, 0, B, acc, acc);
-            tile_foreach<NT, false>(acc, B, [&](int t, int r, float v) {
-                part[(size_t)t * 2 * Is + m * Is + row0 + r] = v * exp2i(s_shift[t]);
-            });
+            for (int m = 0; m < 2; ++m) {
+                float acc[NT][4] = {};
+                tile_fp4<NT, false>(m ? a.w.sh_up_q : a.w.sh_gate_q, m ? a.w.sh_up_s : a.w.sh_gate_s, nullptr, nullptr,
+                                    H / 2, H / 32, row0, k0, KR / 128, xs, pitch, 0, nb, acc, acc);
+                tile_foreach<NT, false>(acc, nb, [&](int t, int r, float v) {
+                    part[(size_t)(tg + t) * 2 * Is + m * Is + row0 + r] = v * exp2i(s_shift[tg + t]);
+                });
+            }
         }
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_sgu + rb, a.p.sgu.splits, s_flag)) {
@@ -710,20 +732,24 @@ DEVI bool item_sd(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
     }
     __syncthreads();
     for (int t = threadIdx.x; t < B; t += blockDim.x) s_shift[t] = prescale_shift(__uint_as_float(s_amax[t]));
-    __syncthreads();
-    stage_f16_from_f32<SPLIT>(xs, pitch, a.ws.sh_a, Is, B, [](int t) { return t; }, s_shift, k0, KR);
-    __syncthreads();
     const int warp = threadIdx.x >> 5;
     const int row0 = rb * kDenseRows + warp * 16;
-    const int ncols = SPLIT ? 2 * B : B;
-    if (row0 < H) {
-        float acc[NT][4] = {};
-        tile_fp4<NT, false>(a.w.sh_down_q, a.w.sh_down_s, nullptr, nullptr, Is / 2, Is / 32, row0, k0, KR / 128, xs,
-                            pitch, 0, ncols, acc, acc);
-        float *part = a.ws.sd_part + (size_t)ks * maxB * H;
-        tile_foreach<NT, SPLIT>(acc, B, [&](int t, int r, float v) {
-            part[(size_t)t * H + row0 + r] = v * exp2i(s_shift[t]);
-        });
+    float *part = a.ws.sd_part + (size_t)ks * maxB * H;
+    constexpr int GT = SPLIT ? 4 * NT : 8 * NT;  // tokens per group
+    for (int tg = 0; tg < B; tg += GT) {
+        const int nb = min(GT, B - tg);
+        __syncthreads();
+        stage_f16_from_f32<SPLIT>(xs, pitch, a.ws.sh_a + (size_t)tg * Is, Is, nb, [](int t) { return t; }, s_shift + tg, k0,
+                                  KR);
+        __syncthreads();
+        if (row0 < H) {
+            float acc[NT][4] = {};
+            tile_fp4<NT, false>(a.w.sh_down_q, a.w.sh_down_s, nullptr, nullptr, Is / 2, Is / 32, row0, k0, KR / 128, xs,
+                                pitch, 0, SPLIT ? 2 * nb : nb, acc, acc);
+            tile_foreach<NT, SPLIT>(acc, nb, [&](int t, int r, float v) {
+                part[(size_t)(tg + t) * H + row0 + r] = v * exp2i(s_shift[tg + t]);
+            });
+        }
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_sd + rb, a.p.sd.splits, s_flag)) {
         for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
@@ -784,6 +810,15 @@ DEVI void prefetch_sd(const StepArgs &a, int bid) {
     const int rb = bid / a.p.sd.splits, ks = bid % a.p.sd.splits, Is = a.d.Is;
     const int rows = min(kDenseRows, a.d.H - rb * kDenseRows), kr = a.p.sd.krange;
     prefetch_fp4_rows(a.w.sh_down_q, a.w.sh_down_s, Is, rb * kDenseRows, rows, ks * kr, kr);
+}
+
+// Router rows [E c / G, E (c+1) / G) of the layer that steps next (a.next_router), one row per
+// thread: the cross-layer hint, issued by CTAs that have no work left in this step.
+DEVI void prefetch_next_router(const StepArgs &a, int c, int G) {
+    if (!a.next_router) return;
+    const int E = a.d.E, lo = (int)((long long)E * c / G), hi = (int)((long long)E * (c + 1) / G);
+    for (int r = lo + (int)threadIdx.x; r < hi; r += blockDim.x)
+        prefetch_l2(a.next_router + (size_t)r * a.d.H, (uint32_t)a.d.H * 2);
 }
 
 // 16 rows of an active expert, whole K: contiguous in the row-major layout (lane 0 issues them)

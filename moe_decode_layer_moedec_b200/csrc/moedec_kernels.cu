@@ -42,8 +42,9 @@ __global__ void __launch_bounds__(256) k_router_dn(StepArgs a) {
 
 // top-k: one CTA of 256 threads per token; the last one builds the expert buckets
 __global__ void __launch_bounds__(256) k_topk(StepArgs a) {
+    extern __shared__ __align__(16) unsigned char smem[];  // token masks of the bucket builder above 64 tokens
     __shared__ TopkSmem t;
-    item_topk<false>(a, blockIdx.x, t);
+    item_topk<false>(a, blockIdx.x, t, 0u, nullptr, nullptr, nullptr, reinterpret_cast<unsigned long long *>(smem));
 }
 
 // routed experts: every warp takes a contiguous range of (expert, 16-row) warp items
@@ -136,7 +137,8 @@ cudaError_t launch_router_dn(const StepArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_topk(const StepArgs &a, cudaStream_t s) {
-    k_topk<<<a.B, 256, 0, s>>>(a);
+    const size_t sm = a.B > 64 ? (size_t)a.d.E * ((a.B + 63) / 64) * 8 : 0;
+    k_topk<<<a.B, 256, sm, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -230,7 +232,7 @@ int kernels_per_step(const Dims &d) { return d.n_shared ? 8 : 6; }
 cudaError_t init_kernel_attributes() {
     const int lim = 160 * 1024;
     const void *fns[] = {
-        (const void *)k_router_dn<1>, (const void *)k_router_dn<2>, (const void *)k_router_dn<4>,
+        (const void *)k_topk, (const void *)k_router_dn<1>, (const void *)k_router_dn<2>, (const void *)k_router_dn<4>,
         (const void *)k_router_dn<8>, (const void *)k_expert<true>, (const void *)k_expert<false>,
         (const void *)k_up<1>, (const void *)k_up<2>, (const void *)k_up<4>, (const void *)k_up<8>,
         (const void *)k_up<16>, (const void *)k_shared_gu<1>, (const void *)k_shared_gu<2>,

@@ -16,6 +16,8 @@ full_b2            full size, B=2; token 1 = bf16(token 0 + 0.1 N(0,1))
 full_b16           full size, B=16, independent N(0,1) tokens
 full_b64_skewed    full size, B=64; 32 hot router rows get beta * u added (u ~ N(0,1/H)),
                    timed over 32 layers of distinct weights
+full_b256          full size, B=256 independent tokens (speculative decoding: 32 sequences x
+                   (7 drafts + 1) verified per step)
 =================  ====================================================================
 
 Value recipe: tokens bf16 ~ N(0,1); router, W_dn, W_up bf16 ~ N(0, 1/fan_in); MXFP4 codes
@@ -142,6 +144,9 @@ WORKLOADS = {
     "full_b16": Workload("full_b16", FULL, 16, 1003, description="full-size layer, B=16, independent tokens"),
     "full_b64_skewed": Workload("full_b64_skewed", FULL, 64, 1004, hot_experts=32, hot_beta=HOT_BETA_B64,
                                 layers=32, description="full-size layer, B=64, 32 hot experts, 32 layers"),
+    # speculative decoding verifies batch x (drafts + 1) tokens per step: 32 sequences x 8 (7 drafts)
+    "full_b256": Workload("full_b256", FULL, 256, 1006,
+                          description="full-size layer, B=256 (speculative decode: 32 x (7 drafts + 1)), independent"),
 }
 
 
