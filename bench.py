@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--reps", type=int, default=5, help="timed replays of the K-step graph (median)")
     p.add_argument("--no-per-config", action="store_true", help="skip the B=2/16/64 entries of per_config")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--ncu", action="store_true",
+                   help="profiling case for ncu: --steps eager steps over --layers resident layers, no timing")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
     return p.parse_args()
 
@@ -178,8 +180,8 @@ KERNEL_SOURCES = {
                           "moedec_router.cuh", "moedec_internal.h"],
     "fused_step_small": ["moedec_fused_small.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
                          "moedec_router.cuh", "moedec_internal.h"],
-    "fused_step_splitk": ["moedec_fused.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
-                          "moedec_router.cuh", "moedec_internal.h"],
+    "fused_step_splitk": ["moedec_fused.cu", "moedec_experts.cuh", "moedec_items.cuh", "moedec_tiles.cuh",
+                          "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h"],
 }
 
 
@@ -428,6 +430,22 @@ def config_entry(w, ms, times, clocks, steps, world, unique_mean, peak, hinted=N
     return r
 
 
+def profile_case(args, w, n_layers, local_rank, rank):
+    """The small case an ncu capture runs: step i on layer i mod n_layers, eagerly, then every
+    layer's device error word is read (the run exits non-zero on a device-side error)."""
+    import torch
+    layers, dev_weights = load_layers(w, n_layers, args.schedule, local_rank, rank)
+    x = torch.from_numpy(synth.tokens(w).view(np.int16)).to(f"cuda:{local_rank}")
+    out = torch.empty_like(x)
+    for i in range(args.steps):
+        layers[i % n_layers].step(x, out=out)
+    torch.cuda.synchronize()
+    for L_ in layers:
+        L_.routing(w.batch)
+        L_.close()
+    log(f"[bench] profiling case done: {args.steps} steps of {w.name} over {n_layers} layers")
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -447,6 +465,8 @@ def main():
     d = w.dims
     B = w.batch
     n_layers = default_layers(w, args.layers)
+    if args.ncu:
+        return profile_case(args, w, n_layers, local_rank, rank)
     peak, peak_src = measured_peak_hbm()
     layers, dev_weights = load_layers(w, n_layers, args.schedule, local_rank, rank)
     x_host = torch.from_numpy(synth.tokens(w).view(np.int16)).pin_memory()

@@ -24,7 +24,9 @@
 
 namespace moedec {
 
-constexpr int kSegTok = 16;  // tokens of one expert per group (at most two 8-column MMA tiles)
+// Tokens of one expert per group: 16 (two 8-column MMA tiles) in the one-CTA-per-SM layout, 8 (one
+// tile, one code path, fewer registers) in the two-CTAs-per-SM layout.
+constexpr int kSegTok = 16;
 
 // One MXFP4 weight stream of a warp: `ntiles` 16-row tiles (tile t starts at row row0 + t *
 // tstride), each over the whole K (rpt = K / 128 rounds of 16 code bytes and one scale byte per
@@ -147,12 +149,13 @@ struct SegPlan {
 };
 
 // all threads (blockDim.x == 256: four slots per thread, 1024 at most); a barrier must follow
-DEVI void seg_plan(SegPlan &sp, const SplitKRoute &rt, int *s_warp) {
+template <int SEGTOK, class RT>
+DEVI void seg_plan(SegPlan &sp, const RT &rt, int *s_warp) {
     int c[4], tot = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int j = 4 * threadIdx.x + i;
-        c[i] = j < rt.n_active ? (rt.cnt[j] + kSegTok - 1) / kSegTok : 0;
+        c[i] = j < rt.n_active ? (rt.cnt[j] + SEGTOK - 1) / SEGTOK : 0;
         tot += c[i];
     }
     int n;
@@ -187,8 +190,8 @@ struct SegSmem {
 // The CTA's segments in order: body(j, g, b0, b1) for each maximal run of items of one token
 // group (slot j, group g) inside [lo, hi) of an expert phase with nb blocks per expert.  Uniform
 // over the CTA.  Returns false as soon as a body does.
-template <class Body>
-DEVI bool for_each_segment(const SegPlan &sp, const SplitKRoute &rt, int nb, int lo, int hi, Body body) {
+template <class RT, class Body>
+DEVI bool for_each_segment(const SegPlan &sp, const RT &rt, int nb, int lo, int hi, Body body) {
     int i = lo;
     while (i < hi) {
         const int gi = i / nb, b0 = i % nb, b1 = min(nb, b0 + (hi - i));
@@ -205,11 +208,11 @@ DEVI bool for_each_segment(const SegPlan &sp, const SplitKRoute &rt, int nb, int
 // fp16 hi/lo column pairs for at most 4 tokens, one fp16 column each otherwise (per-token
 // power-of-two prescale).  Every tile's warp adds 1 to ctl_gu[j] when its a rows are written.
 
-template <int NT>
-DEVI void seg_gate_up(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
+template <int NT, int SEGTOK, int D, class RT>
+DEVI void seg_gate_up(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
     const int L = a.d.L, I = a.d.I, K = a.d.k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2, q = lane & 3;
-    const int e = rt.e[j], ntok = min(kSegTok, rt.cnt[j] - g * kSegTok), off = rt.off[j] + g * kSegTok;
+    const int e = rt.e[j], ntok = min(SEGTOK, rt.cnt[j] - g * SEGTOK), off = rt.off[j] + g * SEGTOK;
     const size_t eq = (size_t)e * I * (L / 2), es = (size_t)e * I * (L / 32);
     const int pitch = f16_pitch(L);
     const bool split = ntok <= 4;  // hi/lo column pairs (only with NT == 1)
@@ -269,15 +272,20 @@ DEVI void seg_gate_up(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss, uin
         }
         warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, 1u);
     };
-    ring_fp4_tiles<NT, true, (NT == 1 ? 4 : 2)>(a.w.gate_q + eq, a.w.gate_s + es, a.w.up_q + eq, a.w.up_s + es, L, b0 * 128 + warp * 16,
+    ring_fp4_tiles<NT, true, D>(a.w.gate_q + eq, a.w.gate_s + es, a.w.up_q + eq, a.w.up_s + es, L, b0 * 128 + warp * 16,
                                 128, b1 - b0, xs, pitch, split ? 2 * ntok : ntok, pre, epi);
 }
 
-DEVI void seg_gate_up_any(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0,
-                          int b1) {
+// MINB: CTAs per SM of the calling kernel (2: 8-token groups, a shallower ring, one code path)
+template <int MINB, class RT>
+DEVI void seg_gate_up_any(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
+    if (MINB > 1) {
+        seg_gate_up<1, 8, 2>(a, rt, ss, xs, j, g, b0, b1);
+        return;
+    }
     const int ntok = min(kSegTok, rt.cnt[j] - g * kSegTok);
-    if (ntok <= 8) seg_gate_up<1>(a, rt, ss, xs, j, g, b0, b1);
-    else seg_gate_up<2>(a, rt, ss, xs, j, g, b0, b1);
+    if (ntok <= 8) seg_gate_up<1, kSegTok, 4>(a, rt, ss, xs, j, g, b0, b1);
+    else seg_gate_up<2, kSegTok, 2>(a, rt, ss, xs, j, g, b0, b1);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -286,12 +294,12 @@ DEVI void seg_gate_up_any(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss,
 // tokens into ctl_ylat).  Waits for every gate/up tile of expert slot j (all its groups) first,
 // with the segment's first weight rounds already in flight.  Returns false after an abort.
 
-template <int NT>
-DEVI bool seg_down(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
+template <int NT, int SEGTOK, int D, class RT>
+DEVI bool seg_down(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
     const int L = a.d.L, I = a.d.I, K = a.d.k;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gq = lane >> 2, q = lane & 3;
-    const int e = rt.e[j], ntok = min(kSegTok, rt.cnt[j] - g * kSegTok), off = rt.off[j] + g * kSegTok;
-    const unsigned gu_tiles = (unsigned)((rt.cnt[j] + kSegTok - 1) / kSegTok * (I / 16));
+    const int e = rt.e[j], ntok = min(SEGTOK, rt.cnt[j] - g * SEGTOK), off = rt.off[j] + g * SEGTOK;
+    const unsigned gu_tiles = (unsigned)((rt.cnt[j] + SEGTOK - 1) / SEGTOK * (I / 16));
     const size_t eq = (size_t)e * L * (I / 2), es = (size_t)e * L * (I / 32);
     const int pitch = f16_pitch(I);
     const bool split = NT == 1 && ntok <= 4;  // hi/lo column pairs
@@ -323,22 +331,26 @@ DEVI bool seg_down(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss, uint16
     };
     (void)gq;
     (void)q;
-    ring_fp4_tiles<NT, false, (NT == 1 ? 8 : 4)>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I, b0 * 128 + warp * 16, 128,
+    ring_fp4_tiles<NT, false, D>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I, b0 * 128 + warp * 16, 128,
                                  b1 - b0, xs, pitch, split ? 2 * ntok : ntok, pre, epi);
     return ok;
 }
 
-DEVI bool seg_down_any(const StepArgs &a, const SplitKRoute &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0,
-                       int b1) {
+template <int MINB, class RT>
+DEVI bool seg_down_any(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
+    if (MINB > 1) return seg_down<1, 8, 4>(a, rt, ss, xs, j, g, b0, b1);
     const int ntok = min(kSegTok, rt.cnt[j] - g * kSegTok);
-    if (ntok <= 8) return seg_down<1>(a, rt, ss, xs, j, g, b0, b1);
-    return seg_down<2>(a, rt, ss, xs, j, g, b0, b1);
+    if (ntok <= 8) return seg_down<1, kSegTok, 8>(a, rt, ss, xs, j, g, b0, b1);
+    return seg_down<2, kSegTok, 4>(a, rt, ss, xs, j, g, b0, b1);
 }
 
-// shared memory of the staged activations of one segment (halfs)
-__host__ __device__ inline size_t seg_smem(const Dims &d) {
+// tokens per group of the layout with MINB CTAs per SM
+__host__ __device__ constexpr int seg_tok(int minb) { return minb > 1 ? 8 : kSegTok; }
+
+// shared memory of the staged activations of one segment (bytes)
+__host__ __device__ inline size_t seg_smem(const Dims &d, int segtok) {
     const int K = d.L > d.I ? d.L : d.I;
-    return (size_t)kSegTok * f16_pitch(K) * 2;
+    return (size_t)segtok * f16_pitch(K) * 2;
 }
 
 }  // namespace moedec

@@ -28,16 +28,40 @@ namespace moedec {
 enum Queue { Q_ROUTER = 0, Q_TOPK, Q_DN, Q_SGU, Q_EGU, Q_SD, Q_EDOWN, Q_UP, Q_COUNT };
 
 // Batch tiers: token-column tiles of the x consumers (NTX), the shared down (NTS, hi/lo split at
-// B <= 4) and the up-projection (NTU, always hi/lo).
+// B <= 4) and the up-projection (NTU, always hi/lo); larger batches run the dense parts in token
+// groups of that width.  Up to 64 tokens the kernel runs two CTAs per SM (128 registers per
+// thread: 16 warps per SM hide the latency of the MXFP4 decode and MMA chains that 8 warps at
+// 255 registers cannot), with 8-token expert groups and routing tables for 64 x 32 selections;
+// above 64 tokens one CTA per SM, 16-token expert groups and tables for 8192 selections.
 template <int TIER>
 struct Tier;
-template <> struct Tier<0> { static constexpr int NTX = 1, NTS = 1, NTU = 1; static constexpr bool SPLITS = true; };
-template <> struct Tier<1> { static constexpr int NTX = 1, NTS = 1, NTU = 2; static constexpr bool SPLITS = false; };
-template <> struct Tier<2> { static constexpr int NTX = 2, NTS = 2, NTU = 4; static constexpr bool SPLITS = false; };
-template <> struct Tier<3> { static constexpr int NTX = 4, NTS = 4, NTU = 8; static constexpr bool SPLITS = false; };
-template <> struct Tier<4> { static constexpr int NTX = 8, NTS = 8, NTU = 16; static constexpr bool SPLITS = false; };
+template <> struct Tier<0> {
+    static constexpr int NTX = 1, NTS = 1, NTU = 1, MINB = 2;
+    static constexpr bool SPLITS = true;
+    using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
+};
+template <> struct Tier<1> {
+    static constexpr int NTX = 1, NTS = 1, NTU = 2, MINB = 2;
+    static constexpr bool SPLITS = false;
+    using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
+};
+template <> struct Tier<2> {
+    static constexpr int NTX = 2, NTS = 2, NTU = 4, MINB = 2;
+    static constexpr bool SPLITS = false;
+    using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
+};
+template <> struct Tier<3> {
+    static constexpr int NTX = 4, NTS = 4, NTU = 4, MINB = 2;
+    static constexpr bool SPLITS = false;
+    using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
+};
+template <> struct Tier<4> {
+    static constexpr int NTX = 8, NTS = 8, NTU = 16, MINB = 1;
+    static constexpr bool SPLITS = false;
+    using RT = SplitKRoute;
+};
 
-__host__ __device__ inline int tier_for_batch(int B) { return B <= 4 ? 0 : B <= 8 ? 1 : B <= 16 ? 2 : B <= 32 ? 3 : 4; }
+__host__ __device__ inline int tier_for_batch(int B) { return B <= 4 ? 0 : B <= 8 ? 1 : B <= 16 ? 2 : B <= 64 ? 3 : 4; }
 
 // Dynamic shared memory: the phases' staging buffers from offset 0 (fused_stage_smem bytes), then
 // the routing tables of the step (they must survive the shared-down staging between the two
@@ -51,24 +75,25 @@ __host__ __device__ inline size_t fused_stage_smem(const StepArgs &a) {
     mx((size_t)8 * T::NTX * f16_pitch(a.p.sgu.krange) * 2);
     mx((size_t)8 * T::NTS * f16_pitch(a.p.sd.krange) * 2);
     mx((size_t)8 * T::NTU * bf16_pitch(up_chunk(T::NTU, a.p.up.krange)) * 2);
-    mx(seg_smem(a.d));
+    mx(seg_smem(a.d, seg_tok(T::MINB)));
     mx((size_t)a.d.E * ((a.B + 63) / 64) * 8);  // the bucket builder's token masks (B > 64)
     return (m + 15) & ~(size_t)15;
 }
 
 template <int TIER>
 __host__ __device__ inline size_t fused_smem(const StepArgs &a) {
-    return fused_stage_smem<TIER>(a) + sizeof(SplitKRoute);
+    return fused_stage_smem<TIER>(a) + sizeof(typename Tier<TIER>::RT);
 }
 
 template <int TIER>
-__global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
+__global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
     using T = Tier<TIER>;
+    using RT = typename T::RT;
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ TopkSmem topk;
     __shared__ unsigned s_flag;
     __shared__ int s_ok;
-    SplitKRoute &route = *reinterpret_cast<SplitKRoute *>(smem + fused_stage_smem<TIER>(a));
+    RT &route = *reinterpret_cast<RT *>(smem + fused_stage_smem<TIER>(a));
     __shared__ SegPlan segp;
     __shared__ SegSmem segs;
     __shared__ int s_scan[32];
@@ -136,13 +161,13 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
     if (alive) {
         cta_load_routing(a, route);
         __syncthreads();
-        seg_plan(segp, route, s_scan);
+        seg_plan<seg_tok(T::MINB)>(segp, route, s_scan);
         __syncthreads();
         const int nb = a.d.I / 128;
         int lo, hi;
         range(nb * segp.ngroups, lo, hi);
         for_each_segment(segp, route, nb, lo, hi, [&](int j, int g, int b0, int b1) {
-            seg_gate_up_any(a, route, segs, xs_e, j, g, b0, b1);
+            seg_gate_up_any<T::MINB>(a, route, segs, xs_e, j, g, b0, b1);
             return true;
         });
     }
@@ -159,7 +184,7 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
         int lo, hi;
         range(nb * segp.ngroups, lo, hi);
         const bool ok = for_each_segment(segp, route, nb, lo, hi, [&](int j, int g, int b0, int b1) {
-            return seg_down_any(a, route, segs, xs_e, j, g, b0, b1);
+            return seg_down_any<T::MINB>(a, route, segs, xs_e, j, g, b0, b1);
         });
         alive = __syncthreads_and(ok ? 1 : 0) != 0;
     }
@@ -191,8 +216,13 @@ __global__ void __launch_bounds__(256, 1) k_fused(StepArgs a) {
 template <int TIER>
 static cudaError_t launch_fused_tier(const StepArgs &a, cudaStream_t s, int n_sm) {
     const size_t sm = fused_smem<TIER>(a);
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_fused<TIER>, 256, sm);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (per_sm > Tier<TIER>::MINB) per_sm = Tier<TIER>::MINB;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(n_sm);
+    cfg.gridDim = dim3(n_sm * per_sm);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = sm;
     cfg.stream = s;

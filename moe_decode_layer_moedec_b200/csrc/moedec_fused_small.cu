@@ -179,8 +179,10 @@ DEVI bool warp_ticket_last(unsigned *counter, unsigned expected) {
 // ---------------------------------------------------------------------------------------------
 // warp items
 
-// router: 8 rows x K/s_rt (fp64 m8n8k4; slot q of step s of chunk c holds k = 32c + 8q + s)
-DEVI void w_router(const StepArgs &a, int item, const uint16_t *xs) {
+// router: 8 rows x K/s_rt (fp64 m8n8k4; slot q of step s of chunk c holds k = 32c + 8q + s).
+// pre() runs once the ring's first D chunks are requested (the first item stages x there).
+template <class Pre = NoPre>
+DEVI void w_router(const StepArgs &a, int item, const uint16_t *xs, Pre pre = Pre()) {
     const int E = a.d.E, H = a.d.H, B = a.B;
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int rg = item / a.p.s_rt, ks = item % a.p.s_rt;
@@ -194,6 +196,7 @@ DEVI void w_router(const StepArgs &a, int item, const uint16_t *xs) {
     uint4 A[D];
 #pragma unroll
     for (int s = 0; s < D; ++s) A[s] = (row_ok && s < nch) ? ldg_weights(rrow + 32 * s) : make_uint4(0u, 0u, 0u, 0u);
+    pre();
     for (int c0i = 0; c0i < nch; c0i += D) {
 #pragma unroll
         for (int s = 0; s < D; ++s) {
@@ -483,33 +486,6 @@ DEVI bool w_up(const StepArgs &a, int item, const uint16_t *ys) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// L2 prefetch of a CTA's own later weights while it waits.  Item ranges are static ([n c / G,
-// n (c+1) / G) of each queue), so a CTA knows which W_up rows it will read before its chain gets
-// there, and which expert down rows as soon as the routing is out.  The bytes move while the SM
-// would otherwise idle in a wait; the later phase then reads them from L2.
-
-// W_up items of CTA c of the G chain CTAs: 16 rows x L / s_up, one row segment per thread
-DEVI void prefetch_up_range(const StepArgs &a, int c, int G) {
-    const int n = a.d.H / 16 * a.p.s_up, lo = (int)((long long)n * c / G), hi = (int)((long long)n * (c + 1) / G);
-    const int KW = a.d.L / a.p.s_up;
-    for (int i = threadIdx.x; i < (hi - lo) * 16; i += blockDim.x) {
-        const int it = lo + i / 16, r = i % 16, tile = it / a.p.s_up, ks = it % a.p.s_up;
-        prefetch_l2(a.w.w_up + (size_t)(tile * 16 + r) * a.d.L + (size_t)ks * KW, (uint32_t)KW * 2);
-    }
-}
-
-// expert down items of CTA c: 16 contiguous rows (whole K) of one active expert, codes and scales
-DEVI void prefetch_edown_range(const StepArgs &a, const RouteSmem &rt, int c, int G) {
-    const int L = a.d.L, I = a.d.I, tiles = L / 16;
-    const int n = rt.n_active * tiles, lo = (int)((long long)n * c / G), hi = (int)((long long)n * (c + 1) / G);
-    for (int i = threadIdx.x; i < 2 * (hi - lo); i += blockDim.x) {
-        const int it = lo + i / 2, e = rt.e[it / tiles], tile = it % tiles;
-        if (i & 1) prefetch_l2(a.w.down_s + ((size_t)e * L + (size_t)tile * 16) * (I / 32), 16 * (I / 32));
-        else prefetch_l2(a.w.down_q + ((size_t)e * L + (size_t)tile * 16) * (I / 2), 16 * (I / 2));
-    }
-}
-
-// ---------------------------------------------------------------------------------------------
 // the kernel
 
 __host__ __device__ inline size_t fused_small_smem(const StepArgs &a) {
@@ -610,9 +586,18 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         prefetch_next_router(a, c_sh, G_sh);  // nothing left to do here: pull the next layer's router
     } else {
         // ---- routed chain CTAs ----
-        // router and W_dn read x as bf16
-        stage_x_bf16();
-        warp_queue(QS_ROUTER, n_rt, c_m, G_m, [&](int it) { w_router(a, it, xs); return true; });
+        // router and W_dn read x as bf16: each warp requests its first router item's rows, then
+        // the CTA stages x (every warp takes part in the staging once, item or not)
+        __syncthreads();  // the claim counters are initialised
+        int it0 = -1;
+        if (lane == 0) it0 = cta_take(claim, QS_ROUTER, n_rt, c_m, G_m);
+        it0 = __shfl_sync(0xffffffffu, it0, 0);
+        if (it0 >= 0) {
+            w_router(a, it0, xs, [&]() { stage_x_bf16(); });
+            warp_queue(QS_ROUTER, n_rt, c_m, G_m, [&](int it) { w_router(a, it, xs); return true; });
+        } else {
+            stage_x_bf16();
+        }
         stamp(1);
         __syncthreads();
         for (int it = c_m; alive && it < B; it += G_m)
@@ -623,8 +608,6 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         if (alive && c_m >= n_tk)
             warp_queue(QS_DN, n_dn, c_m - n_tk, G_m - n_tk, [&](int it) { w_dn(a, it, xs); return true; });
         stamp(3);
-        // W_up rows of this CTA into L2 while the routing is computed
-        if (alive) prefetch_up_range(a, c_m, G_m);
         // expert gate/up: routing and all of h final; stage h of every token (fp16 hi/lo)
         if (alive) alive = cta_wait_geq(a, ctl + CTL_ROUTE_READY, 1u, &s_ok);
         stamp(11);
@@ -634,7 +617,6 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
             if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
             cta_load_routing(a, route);
             __syncthreads();
-            prefetch_edown_range(a, route, c_m, G_m);  // this CTA's expert down rows, during gate/up
             stage_f16_from_f32<true>(xs, f16_pitch(L), a.ws.h, L, B, [](int t) { return t; }, s_shift, 0, L);
             __syncthreads();
             const int n = route.n_active * (I / 16) * a.p.s_egu;
