@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--reps", type=int, default=5, help="timed replays of the K-step graph (median)")
     p.add_argument("--no-per-config", action="store_true", help="skip the B=2/16/64 entries of per_config")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--fp4-stream", action="store_true",
+                   help="build and run bench_fp4_stream.cu (streaming rate of the MXFP4 tile path, piece by piece)")
     p.add_argument("--ncu", action="store_true",
                    help="profiling case for ncu: --steps eager steps over --layers resident layers, no timing")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
@@ -446,8 +448,20 @@ def profile_case(args, w, n_layers, local_rank, rank):
     log(f"[bench] profiling case done: {args.steps} steps of {w.name} over {n_layers} layers")
 
 
+def fp4_stream():
+    """Compile bench_fp4_stream.cu for sm_100a (under _build/) and run it; prints its table."""
+    exe = os.path.join(ROOT, "_build", "bench_fp4_stream")
+    os.makedirs(os.path.dirname(exe), exist_ok=True)
+    subprocess.check_call(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
+                           "--expt-relaxed-constexpr", "-I", ROOT, "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "bench_fp4_stream.cu"), "-o", exe])
+    subprocess.check_call([exe])
+
+
 def main():
     args = parse()
+    if args.fp4_stream:
+        return fp4_stream()
     if args.impl == "reference":
         return run_reference(args)
     rank, local_rank, world = dist_env()

@@ -206,7 +206,8 @@ DEVI bool for_each_segment(const SegPlan &sp, const RT &rt, int nb, int lo, int 
 // expert gate/up: a = silu(G_e h) * (U_e h) for the entries of one token group, 128-row blocks
 // [b0, b1) of expert slot j (warp w: rows 128 b + 16 w).  Activations: h of the group's tokens,
 // fp16 hi/lo column pairs for at most 4 tokens, one fp16 column each otherwise (per-token
-// power-of-two prescale).  Every tile's warp adds 1 to ctl_gu[j] when its a rows are written.
+// power-of-two prescale).  Each warp adds its number of tiles to ctl_gu[j] once its a rows of the
+// segment are written.
 
 template <int NT, int SEGTOK, int D, class RT>
 DEVI void seg_gate_up(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs, int j, int g, int b0, int b1) {
@@ -270,10 +271,11 @@ DEVI void seg_gate_up(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs
                 if (ok && gq == 0) atomicMax(a.ws.a_amax + ss.ent[tk], __float_as_uint(m));
             }
         }
-        warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, 1u);
     };
     ring_fp4_tiles<NT, true, D>(a.w.gate_q + eq, a.w.gate_s + es, a.w.up_q + eq, a.w.up_s + es, L, b0 * 128 + warp * 16,
                                 128, b1 - b0, xs, pitch, split ? 2 * ntok : ntok, pre, epi);
+    // the warp's a rows of this segment are written: count its tiles (one fence per segment)
+    warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, (unsigned)(b1 - b0));
 }
 
 // MINB: CTAs per SM of the calling kernel (2: 8-token groups, a shallower ring, one code path)
@@ -290,8 +292,8 @@ DEVI void seg_gate_up_any(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t
 
 // ---------------------------------------------------------------------------------------------
 // expert down: y = D_e a for the entries of one token group, 128-row blocks [b0, b1) of L; the
-// combine is folded in (w * y added into ylat with fp32 reductions; each 16-row tile counts its
-// tokens into ctl_ylat).  Waits for every gate/up tile of expert slot j (all its groups) first,
+// combine is folded in (w * y added into ylat with fp32 reductions; after the segment each of the
+// warp's 16-row tiles counts its tokens into ctl_ylat).  Waits for every gate/up tile of expert slot j (all its groups) first,
 // with the segment's first weight rounds already in flight.  Returns false after an abort.
 
 template <int NT, int SEGTOK, int D, class RT>
@@ -327,12 +329,18 @@ DEVI bool seg_down(const StepArgs &a, const RT &rt, SegSmem &ss, uint16_t *xs, i
         };
         if (split) tile_foreach<NT, true>(acc, ntok, add);
         else tile_foreach<NT, false>(acc, ntok, add);
-        warp_signal_add(a.ws.ctl + a.p.ctl_ylat + row0 / 16, (unsigned)ntok);
     };
     (void)gq;
     (void)q;
     ring_fp4_tiles<NT, false, D>(a.w.down_q + eq, a.w.down_s + es, nullptr, nullptr, I, b0 * 128 + warp * 16, 128,
                                  b1 - b0, xs, pitch, split ? 2 * ntok : ntok, pre, epi);
+    // the warp's ylat additions of this segment are done: one fence, then each tile's count
+    if (ok) {
+        __threadfence();
+        __syncwarp();
+        if (lane == 0)
+            for (int b = b0; b < b1; ++b) atomicAdd(a.ws.ctl + a.p.ctl_ylat + (b * 128 + warp * 16) / 16, (unsigned)ntok);
+    }
     return ok;
 }
 

@@ -1,11 +1,11 @@
 // moedec_fused.cu -- the whole decode layer step as one persistent kernel.
 //
-// One CTA per SM (cooperative launch, so every CTA is resident).  The step's work items sit in
-// eight queues that every CTA drains in the same order, claiming each next item one item ahead
-// and prefetching that item's weights into L2 while the current one runs:
+// One or two CTAs per SM (cooperative launch, so every CTA is resident).  The step's work items
+// sit in queues that every CTA drains in the same order (the routed experts in static per-CTA
+// segments, the top-k one token per CTA):
 //
 //   0 router row blocks        (fp64 logits)                       CTA items
-//   1 top-k, one per token     waits: all router blocks            CTA items; last builds buckets
+//   1 top-k, one per token     waits: all router blocks            token t on CTA t; last builds buckets
 //   2 W_dn row blocks          (h)                                 CTA items
 //   3 shared gate/up blocks    (sh_a)                              CTA items
 //   4 expert gate/up           waits: buckets, all of h            static per-CTA segments
@@ -69,7 +69,7 @@ __host__ __device__ inline int tier_for_batch(int B) { return B <= 4 ? 0 : B <= 
 template <int TIER>
 __host__ __device__ inline size_t fused_stage_smem(const StepArgs &a) {
     using T = Tier<TIER>;
-    size_t m = (size_t)8 * (a.p.rt.krange + 4) * sizeof(double);
+    size_t m = router_smem(a.p.rt.krange);
     auto mx = [&](size_t v) { m = v > m ? v : m; };
     mx((size_t)8 * T::NTX * bf16_pitch(a.p.dn.krange) * 2);
     mx((size_t)8 * T::NTX * f16_pitch(a.p.sgu.krange) * 2);
@@ -110,43 +110,37 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
     };
     stamp(0);
 
-    // Items are taken dynamically (one atomic per item on the queue head) but one item ahead: the
-    // index of the next item is claimed when the current one starts, and that item's weights are
-    // prefetched into L2 while the current one runs.
-    auto cta_queue = [&](int q, int n, auto prefetch, auto body) {
-        __syncthreads();
-        if (threadIdx.x == 0) s_next = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
-        __syncthreads();
-        int it = s_next;
-        if (it < n) prefetch(it);
-        while (alive && it < n) {
+    // Items are taken dynamically, one atomic per item on the queue head, each when the CTA is
+    // ready for it.  (Claiming one item ahead, to prefetch its weights into L2, let the first CTAs
+    // into a queue hold two items each while later ones got none: the dense queues have fewer
+    // items than two per CTA.)
+    auto cta_queue = [&](int q, int n, auto body) {
+        while (alive) {
             __syncthreads();
             if (threadIdx.x == 0) s_next = (int)atomicAdd(ctl + CTL_QHEAD + q, 1u);
             __syncthreads();
-            const int nxt = s_next;
-            if (nxt < n) prefetch(nxt);
+            const int it = s_next;
+            if (it >= n) break;
             alive = body(it);
-            it = nxt;
         }
     };
     // 0: router
-    cta_queue(Q_ROUTER, n_rt, [&](int it) { prefetch_router(a, it); },
-              [&](int it) { item_router<true>(a, it, smem, &s_flag); return true; });
+    cta_queue(Q_ROUTER, n_rt, [&](int it) { item_router<true>(a, it, smem, &s_flag); return true; });
     stamp(1);
-    // 1: top-k
-    cta_queue(Q_TOPK, a.B, [](int) {},
-              [&](int it) {
-                  return item_topk<true>(a, it, topk, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat, nullptr,
-                                         reinterpret_cast<unsigned long long *>(smem));
-              });
+    // 1: top-k, token t on CTA t (and t + G, ...).  While fewer tokens than CTAs, the top-k CTAs
+    // take no W_dn or shared gate/up items: a CTA that ranked a token would claim them late and
+    // enter its static range of the expert phase after the others
+    for (int t = blockIdx.x; alive && t < a.B; t += gridDim.x)
+        alive = item_topk<true>(a, t, topk, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat, nullptr,
+                                reinterpret_cast<unsigned long long *>(smem));
     stamp(2);
-    // 2: W_dn
-    cta_queue(Q_DN, n_dn, [&](int it) { prefetch_dn(a, it); },
-              [&](int it) { item_dn<true, T::NTX>(a, it, smem, &s_flag); return true; });
-    stamp(3);
-    // 3: shared gate/up
-    cta_queue(Q_SGU, n_sgu, [&](int it) { prefetch_sgu(a, it); },
-              [&](int it) { item_sgu<true, T::NTX>(a, it, smem, &s_flag); return true; });
+    if ((int)blockIdx.x >= a.B || a.B >= (int)gridDim.x) {
+        // 2: W_dn
+        cta_queue(Q_DN, n_dn, [&](int it) { item_dn<true, T::NTX>(a, it, smem, &s_flag); return true; });
+        stamp(3);
+        // 3: shared gate/up
+        cta_queue(Q_SGU, n_sgu, [&](int it) { item_sgu<true, T::NTX>(a, it, smem, &s_flag); return true; });
+    }
     stamp(4);
     // 4: expert gate/up: routing and all of h must be final; the CTA's static range of the
     // (slot, token group, 128-row block) items, one activation staging per segment
@@ -173,8 +167,7 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
     }
     stamp(6);
     // 5: shared down
-    cta_queue(Q_SD, n_sd, [&](int it) { prefetch_sd(a, it); },
-              [&](int it) { return item_sd<true, T::NTS, T::SPLITS>(a, it, smem, &s_flag, &s_ok); });
+    cta_queue(Q_SD, n_sd, [&](int it) { return item_sd<true, T::NTS, T::SPLITS>(a, it, smem, &s_flag, &s_ok); });
     stamp(7);
     // 6: expert down: the same plan over L / 128 blocks per expert; each segment waits for its
     // expert's gate/up tiles
@@ -191,8 +184,7 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
     stamp(8);
     if (alive) prefetch_next_router(a, blockIdx.x, gridDim.x);
     // 7: W_up and the output
-    cta_queue(Q_UP, n_up, [&](int it) { prefetch_up(a, it); },
-              [&](int it) { return item_up<true, T::NTU>(a, it, smem, &s_flag, &s_ok); });
+    cta_queue(Q_UP, n_up, [&](int it) { return item_up<true, T::NTU>(a, it, smem, &s_flag, &s_ok); });
     stamp(9);
     // leave; the last CTA out clears the control block for the next step
     __syncthreads();

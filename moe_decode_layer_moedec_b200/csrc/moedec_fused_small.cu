@@ -244,13 +244,24 @@ DEVI void w_dn(const StepArgs &a, int item, const uint16_t *xs) {
             part[(size_t)(2 * q + j) * L + row0 + g + 8] = acc[2 + j];
         }
     if (!warp_ticket_last(a.ws.ctl + a.p.ctl_tk + (a.d.E + 7) / 8 + tile, a.p.s_dn)) return;
+    // the lane's (token, row) sums: tokens 2q, 2q+1 x rows g, g+8, their loads in flight together
+    const float *pp[4];
+    bool okv[4];
+    float sv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int b = 2 * q + (i >> 1), r = row0 + g + 8 * (i & 1);
+        okv[i] = b < B;
+        pp[i] = a.ws.dn_part + (okv[i] ? (size_t)b * L + r : 0);
+    }
+    sum_splits_batch<4, 8>(pp, okv, (size_t)maxB * L, a.p.s_dn, sv);
     for (int j = 0; j < 2; ++j) {
         const int b = 2 * q + j;
         float m = 0.0f;
         if (b < B)
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int r = row0 + g + 8 * h2;
-                const float v = sum_splits(a.ws.dn_part + (size_t)b * L + r, (size_t)maxB * L, a.p.s_dn);
+                const float v = sv[2 * j + h2];
                 a.ws.h[(size_t)b * L + r] = v;
                 m = fmaxf(m, fabsf(v));
             }
@@ -288,10 +299,15 @@ DEVI void w_sgu(const StepArgs &a, int item, const uint16_t *xs16, const int *xs
         if (b < B) {
             const float sc = exp2i(xshift[b]);
             const float *p = a.ws.sgu_part + (size_t)b * 2 * Is;
+            // gate and up sums of rows g, g+8, their loads in flight together
+            const float *pp[4] = {p + row0 + g, p + Is + row0 + g, p + row0 + g + 8, p + Is + row0 + g + 8};
+            const bool okv[4] = {true, true, true, true};
+            float sv[4];
+            sum_splits_batch<4, 8>(pp, okv, (size_t)maxB * 2 * Is, a.p.s_sgu, sv);
             for (int h2 = 0; h2 < 2; ++h2) {
                 const int r = row0 + g + 8 * h2;
-                const float gs = sum_splits(p + r, (size_t)maxB * 2 * Is, a.p.s_sgu) * sc;
-                const float us = sum_splits(p + Is + r, (size_t)maxB * 2 * Is, a.p.s_sgu) * sc;
+                const float gs = sv[2 * h2] * sc;
+                const float us = sv[2 * h2 + 1] * sc;
                 const float v = gs / (1.0f + expf(-gs)) * us;
                 a.ws.sh_a[(size_t)b * Is + r] = v;
                 m = fmaxf(m, fabsf(v));
@@ -355,10 +371,15 @@ DEVI void w_egu(const StepArgs &a, const RouteSmem &rt, int item, const uint16_t
         const float *p = a.ws.egu_part + (size_t)ent_q * 2 * I + row0;
         const size_t st = nent * 2 * I;
         float *dst = a.ws.a + (size_t)ent_q * I + row0;
+        // gate and up sums of rows g, g+8, their loads in flight together
+        const float *pp[4] = {p + g, p + I + g, p + g + 8, p + I + g + 8};
+        const bool okv[4] = {true, true, true, true};
+        float sv[4];
+        sum_splits_batch<4, 2>(pp, okv, st, S, sv);
         for (int h2 = 0; h2 < 2; ++h2) {
             const int r = g + 8 * h2;
-            const float gs = (S > 1 ? sum_splits(p + r, st, S) : __ldcg(p + r)) * sc;
-            const float us = (S > 1 ? sum_splits(p + I + r, st, S) : __ldcg(p + I + r)) * sc;
+            const float gs = sv[2 * h2] * sc;
+            const float us = sv[2 * h2 + 1] * sc;
             const float v = gs / (1.0f + expf(-gs)) * us;
             dst[r] = v;
             m = fmaxf(m, fabsf(v));
@@ -474,14 +495,18 @@ DEVI bool w_up(const StepArgs &a, int item, const uint16_t *ys) {
     // only the warp that completes the tile adds the shared expert's rows: the rest of W_up
     // streams while the shared expert finishes
     if (a.d.n_shared && !warp_wait_geq(a, a.ws.ctl + CTL_SD_DONE, (unsigned)(H / 16))) return false;
-    if (q < B)
+    if (q < B) {
+        const float *pp[2] = {a.ws.up_part + (size_t)q * H + row0 + g, a.ws.up_part + (size_t)q * H + row0 + g + 8};
+        const bool okv[2] = {true, true};
+        float sv[2], shv[2];
+        for (int h2 = 0; h2 < 2; ++h2) shv[h2] = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)q * H + row0 + g + 8 * h2) : 0.0f;
+        sum_splits_batch<2, 4>(pp, okv, (size_t)maxB * H, a.p.s_up, sv);
         for (int h2 = 0; h2 < 2; ++h2) {
             const int r = row0 + g + 8 * h2;
-            const float s = sum_splits(a.ws.up_part + (size_t)q * H + r, (size_t)maxB * H, a.p.s_up);
-            if (a.ws.up_tap) a.ws.up_tap[(size_t)q * H + r] = s;
-            const float shv = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)q * H + r) : 0.0f;
-            a.out[(size_t)q * H + r] = f32_to_bf16_rne(s + shv);
+            if (a.ws.up_tap) a.ws.up_tap[(size_t)q * H + r] = sv[h2];
+            a.out[(size_t)q * H + r] = f32_to_bf16_rne(sv[h2] + shv[h2]);
         }
+    }
     return true;
 }
 

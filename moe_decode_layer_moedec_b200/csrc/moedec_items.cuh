@@ -153,12 +153,28 @@ DEVI void item_dn(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_dn + rb, a.p.dn.splits, s_flag)) {
         for (int t = threadIdx.x; t < B; t += blockDim.x) s_amax[t] = 0u;
         __syncthreads();
-        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
-            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
-            if (r >= L) continue;
-            const float s = sum_splits(a.ws.dn_part + (size_t)b * L + r, (size_t)maxB * L, a.p.dn.splits);
-            a.ws.h[(size_t)b * L + r] = s;
-            atomicMax(s_amax + b, __float_as_uint(fabsf(s)));
+        constexpr int NP = 4;  // (row, token) sums per thread and pass, their loads in flight together
+        for (int i0 = threadIdx.x; i0 < kDenseRows * B; i0 += NP * blockDim.x) {
+            const float *pp[NP];
+            bool ok[NP];
+            size_t o[NP];
+            float sum[NP];
+            int bb[NP];
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const int i = i0 + j * blockDim.x, r = rb * kDenseRows + (i % kDenseRows);
+                bb[j] = i / kDenseRows;
+                ok[j] = i < kDenseRows * B && r < L;
+                o[j] = ok[j] ? (size_t)bb[j] * L + r : 0;
+                pp[j] = a.ws.dn_part + o[j];
+            }
+            sum_splits_batch<NP, 8>(pp, ok, (size_t)maxB * L, a.p.dn.splits, sum);
+#pragma unroll
+            for (int j = 0; j < NP; ++j)
+                if (ok[j]) {
+                    a.ws.h[o[j]] = sum[j];
+                    atomicMax(s_amax + bb[j], __float_as_uint(fabsf(sum[j])));
+                }
         }
         __syncthreads();
         for (int t = threadIdx.x; t < B; t += blockDim.x) atomicMax(a.ws.ctl + a.p.ctl_hamax + t, s_amax[t]);
@@ -640,13 +656,27 @@ DEVI bool item_up(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_up + rb, a.p.up.splits, s_flag)) {
         if (FUSED && a.d.n_shared && !cta_wait_geq(a, a.ws.ctl + CTL_SD_DONE, (unsigned)a.p.sd.blocks, s_ok)) return false;
-        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
-            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
-            if (r >= H) continue;
-            const float s = sum_splits(a.ws.up_part + (size_t)b * H + r, (size_t)maxB * H, a.p.up.splits);
-            if (a.ws.up_tap) a.ws.up_tap[(size_t)b * H + r] = s;
-            const float shv = a.d.n_shared ? __ldcg(a.ws.sh + (size_t)b * H + r) : 0.0f;
-            a.out[(size_t)b * H + r] = f32_to_bf16_rne(s + shv);
+        constexpr int NP = 4;
+        for (int i0 = threadIdx.x; i0 < kDenseRows * B; i0 += NP * blockDim.x) {
+            const float *pp[NP];
+            bool ok[NP];
+            size_t o[NP];
+            float sum[NP], shv[NP];
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const int i = i0 + j * blockDim.x, r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+                ok[j] = i < kDenseRows * B && r < H;
+                o[j] = ok[j] ? (size_t)b * H + r : 0;
+                pp[j] = a.ws.up_part + o[j];
+                shv[j] = (ok[j] && a.d.n_shared) ? __ldcg(a.ws.sh + o[j]) : 0.0f;
+            }
+            sum_splits_batch<NP, 8>(pp, ok, (size_t)maxB * H, a.p.up.splits, sum);
+#pragma unroll
+            for (int j = 0; j < NP; ++j)
+                if (ok[j]) {
+                    if (a.ws.up_tap) a.ws.up_tap[o[j]] = sum[j];
+                    a.out[o[j]] = f32_to_bf16_rne(sum[j] + shv[j]);
+                }
         }
     }
     return true;
@@ -700,13 +730,27 @@ DEVI void item_sgu(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_
         }
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_sgu + rb, a.p.sgu.splits, s_flag)) {
-        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
-            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
-            if (r >= Is) continue;
-            const float *p = a.ws.sgu_part + (size_t)b * 2 * Is + r;
-            const float gs = sum_splits(p, (size_t)maxB * 2 * Is, a.p.sgu.splits);
-            const float us = sum_splits(p + Is, (size_t)maxB * 2 * Is, a.p.sgu.splits);
-            a.ws.sh_a[(size_t)b * Is + r] = gs / (1.0f + expf(-gs)) * us;
+        constexpr int NR = 2;  // (row, token) pairs per thread and pass: gate and up sums of each
+        for (int i0 = threadIdx.x; i0 < kDenseRows * B; i0 += NR * blockDim.x) {
+            const float *pp[2 * NR];
+            bool ok[2 * NR];
+            size_t o[NR];
+            float sum[2 * NR];
+#pragma unroll
+            for (int j = 0; j < NR; ++j) {
+                const int i = i0 + j * blockDim.x, r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+                ok[2 * j] = ok[2 * j + 1] = i < kDenseRows * B && r < Is;
+                o[j] = ok[2 * j] ? (size_t)b * Is + r : 0;
+                pp[2 * j] = a.ws.sgu_part + (ok[2 * j] ? (size_t)b * 2 * Is + r : 0);
+                pp[2 * j + 1] = pp[2 * j] + Is;
+            }
+            sum_splits_batch<2 * NR, 8>(pp, ok, (size_t)maxB * 2 * Is, a.p.sgu.splits, sum);
+#pragma unroll
+            for (int j = 0; j < NR; ++j)
+                if (ok[2 * j]) {
+                    const float gs = sum[2 * j], us = sum[2 * j + 1];
+                    a.ws.sh_a[o[j]] = gs / (1.0f + expf(-gs)) * us;
+                }
         }
         if (FUSED) cta_signal_add(a.ws.ctl + CTL_SGU_DONE, 1u);
     }
@@ -752,11 +796,23 @@ DEVI bool item_sd(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
         }
     }
     if (cta_ticket_last(a.ws.tickets + a.p.ticket_sd + rb, a.p.sd.splits, s_flag)) {
-        for (int i = threadIdx.x; i < kDenseRows * B; i += blockDim.x) {
-            const int r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
-            if (r >= H) continue;
-            const float s = sum_splits(a.ws.sd_part + (size_t)b * H + r, (size_t)maxB * H, a.p.sd.splits);
-            a.ws.sh[(size_t)b * H + r] = s;
+        constexpr int NP = 4;
+        for (int i0 = threadIdx.x; i0 < kDenseRows * B; i0 += NP * blockDim.x) {
+            const float *pp[NP];
+            bool ok[NP];
+            size_t o[NP];
+            float sum[NP];
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const int i = i0 + j * blockDim.x, r = rb * kDenseRows + (i % kDenseRows), b = i / kDenseRows;
+                ok[j] = i < kDenseRows * B && r < H;
+                o[j] = ok[j] ? (size_t)b * H + r : 0;
+                pp[j] = a.ws.sd_part + o[j];
+            }
+            sum_splits_batch<NP, 8>(pp, ok, (size_t)maxB * H, a.p.sd.splits, sum);
+#pragma unroll
+            for (int j = 0; j < NP; ++j)
+                if (ok[j]) a.ws.sh[o[j]] = sum[j];
         }
         if (FUSED) cta_signal_add(a.ws.ctl + CTL_SD_DONE, 1u);
     }
@@ -764,53 +820,7 @@ DEVI bool item_sd(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
 }
 
 // ---------------------------------------------------------------------------------------------
-// L2 prefetch of an item's weights (issued one item ahead by the fused schedule).  CTA items
-// spread their row segments over the CTA's threads; warp items issue a few whole-tile ranges.
-
-DEVI void prefetch_rows(const void *base, size_t row_bytes, int rows, size_t off, uint32_t seg) {
-    for (int r = threadIdx.x; r < rows; r += blockDim.x)
-        prefetch_l2(static_cast<const uint8_t *>(base) + (size_t)r * row_bytes + off, seg);
-}
-
-DEVI void prefetch_router(const StepArgs &a, int bid) {
-    const int rb = bid / a.p.rt.splits, ks = bid % a.p.rt.splits, H = a.d.H;
-    const int rows = min(kRouterRows, a.d.E - rb * kRouterRows);
-    prefetch_rows(a.w.router + (size_t)rb * kRouterRows * H, (size_t)H * 2, rows, (size_t)ks * a.p.rt.krange * 2,
-                  a.p.rt.krange * 2);
-}
-
-DEVI void prefetch_dn(const StepArgs &a, int bid) {
-    const int rb = bid / a.p.dn.splits, ks = bid % a.p.dn.splits, H = a.d.H;
-    const int rows = min(kDenseRows, a.d.L - rb * kDenseRows);
-    prefetch_rows(a.w.w_dn + (size_t)rb * kDenseRows * H, (size_t)H * 2, rows, (size_t)ks * a.p.dn.krange * 2,
-                  a.p.dn.krange * 2);
-}
-
-DEVI void prefetch_up(const StepArgs &a, int bid) {
-    const int rb = bid / a.p.up.splits, ks = bid % a.p.up.splits, L = a.d.L;
-    const int rows = min(kDenseRows, a.d.H - rb * kDenseRows);
-    prefetch_rows(a.w.w_up + (size_t)rb * kDenseRows * L, (size_t)L * 2, rows, (size_t)ks * a.p.up.krange * 2,
-                  a.p.up.krange * 2);
-}
-
-// MXFP4 row block: codes (K/2 bytes per row) and scales (K/32 bytes per row) of a K range
-DEVI void prefetch_fp4_rows(const uint8_t *q, const uint8_t *s, int K, int row0, int rows, int k0, int kr) {
-    prefetch_rows(q + (size_t)row0 * (K / 2), (size_t)K / 2, rows, (size_t)k0 / 2, kr / 2);
-    prefetch_rows(s + (size_t)row0 * (K / 32), (size_t)K / 32, rows, (size_t)k0 / 32, kr / 32);
-}
-
-DEVI void prefetch_sgu(const StepArgs &a, int bid) {
-    const int rb = bid / a.p.sgu.splits, ks = bid % a.p.sgu.splits, H = a.d.H;
-    const int rows = min(kDenseRows, a.d.Is - rb * kDenseRows), kr = a.p.sgu.krange;
-    prefetch_fp4_rows(a.w.sh_gate_q, a.w.sh_gate_s, H, rb * kDenseRows, rows, ks * kr, kr);
-    prefetch_fp4_rows(a.w.sh_up_q, a.w.sh_up_s, H, rb * kDenseRows, rows, ks * kr, kr);
-}
-
-DEVI void prefetch_sd(const StepArgs &a, int bid) {
-    const int rb = bid / a.p.sd.splits, ks = bid % a.p.sd.splits, Is = a.d.Is;
-    const int rows = min(kDenseRows, a.d.H - rb * kDenseRows), kr = a.p.sd.krange;
-    prefetch_fp4_rows(a.w.sh_down_q, a.w.sh_down_s, Is, rb * kDenseRows, rows, ks * kr, kr);
-}
+// L2 prefetch for the cross-layer hint
 
 // Router rows [E c / G, E (c+1) / G) of the layer that steps next (a.next_router), one row per
 // thread: the cross-layer hint, issued by CTAs that have no work left in this step.
@@ -819,25 +829,6 @@ DEVI void prefetch_next_router(const StepArgs &a, int c, int G) {
     const int E = a.d.E, lo = (int)((long long)E * c / G), hi = (int)((long long)E * (c + 1) / G);
     for (int r = lo + (int)threadIdx.x; r < hi; r += blockDim.x)
         prefetch_l2(a.next_router + (size_t)r * a.d.H, (uint32_t)a.d.H * 2);
-}
-
-// 16 rows of an active expert, whole K: contiguous in the row-major layout (lane 0 issues them)
-DEVI void warp_prefetch_expert(const StepArgs &a, int item, bool down) {
-    if ((threadIdx.x & 31) != 0) return;
-    const int L = a.d.L, I = a.d.I;
-    const int tiles = (down ? L : I) / 16, j = item / tiles, tile = item % tiles;
-    const int e = __ldcg(a.ws.active_e + j);
-    if (down) {
-        const size_t q0 = (size_t)e * L * (I / 2) + (size_t)tile * 16 * (I / 2), s0 = (size_t)e * L * (I / 32) + (size_t)tile * 16 * (I / 32);
-        prefetch_l2(a.w.down_q + q0, 16 * (I / 2));
-        prefetch_l2(a.w.down_s + s0, 16 * (I / 32));
-    } else {
-        const size_t q0 = (size_t)e * I * (L / 2) + (size_t)tile * 16 * (L / 2), s0 = (size_t)e * I * (L / 32) + (size_t)tile * 16 * (L / 32);
-        prefetch_l2(a.w.gate_q + q0, 16 * (L / 2));
-        prefetch_l2(a.w.up_q + q0, 16 * (L / 2));
-        prefetch_l2(a.w.gate_s + s0, 16 * (L / 32));
-        prefetch_l2(a.w.up_s + s0, 16 * (L / 32));
-    }
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -116,12 +116,11 @@ __global__ void k_scores(const float *logits, float *scores, size_t n) {
 // ---------------------------------------------------------------------------------------------
 // host launchers
 
-static size_t router_smem(const StepArgs &a) { return (size_t)8 * (a.p.rt.krange + 4) * sizeof(double); }
 
 template <int NT>
 static cudaError_t launch_router_dn_nt(const StepArgs &a, cudaStream_t s) {
     const size_t dn_smem = (size_t)8 * NT * bf16_pitch(a.p.dn.krange) * 2;
-    const size_t sm = router_smem(a) > dn_smem ? router_smem(a) : dn_smem;
+    const size_t sm = router_smem(a.p.rt.krange) > dn_smem ? router_smem(a.p.rt.krange) : dn_smem;
     const int grid = a.p.rt.blocks * a.p.rt.splits + a.p.dn.blocks * a.p.dn.splits;
     k_router_dn<NT><<<grid, 256, sm, s>>>(a);
     return cudaGetLastError();

@@ -69,8 +69,8 @@ extern "C" MOEDEC_API int moedec_router_logits_noalloc(const uint16_t *router, c
     void *scratch = nullptr;
     cudaError_t e = scratch_for_current_device(&scratch);
     if (e != cudaSuccess) return MOEDEC_ERR_CUDA;
-    // at most 8 tokens x (512 + 4) doubles = 33 KB: within the default dynamic shared-memory limit
-    const size_t smem = (size_t)8 * (a.p.rt.krange + 4) * sizeof(double);
+    // 32 tokens x (512 + 8) bf16 = 33 KB: within the default dynamic shared-memory limit
+    const size_t smem = router_smem(a.p.rt.krange);
     a.d.E = n_experts;
     a.d.H = hidden;
     a.d.max_batch = batch;

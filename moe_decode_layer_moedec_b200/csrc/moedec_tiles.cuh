@@ -37,6 +37,28 @@ DEVI T sum_splits(const T *p, size_t stride, int n) {
     return s;
 }
 
+// NP such sums at once: out[i] = sum over k < n of p[i][k * stride], each in split order (the
+// same additions as sum_splits, so the same bits).  The loads of all NP sums for W splits are
+// issued before the first add: a thread that reduces several rows pays one L2 round trip per 16
+// W splits for all of them instead of one per row.  valid[i] false gives out[i] = 0, no loads.
+template <int NP, int W = 16, class T>
+DEVI void sum_splits_batch(const T *const (&p)[NP], const bool (&valid)[NP], size_t stride, int n, T (&out)[NP]) {
+#pragma unroll
+    for (int i = 0; i < NP; ++i) out[i] = T(0);
+    for (int k0 = 0; k0 < n; k0 += W) {
+        T v[NP][W];
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k) v[i][k] = (valid[i] && k0 + k < n) ? __ldcg(p[i] + (size_t)(k0 + k) * stride) : T(0);
+#pragma unroll
+        for (int i = 0; i < NP; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k)
+                if (k0 + k < n) out[i] += v[i][k];
+    }
+}
+
 DEVI float exp2i(int t) { return __int_as_float((127 + t) << 23); }  // 2^t, |t| < 127
 
 // block-wide max of non-negative floats (every thread gets the result); s_red has >= 32 slots
