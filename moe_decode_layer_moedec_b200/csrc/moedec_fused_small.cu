@@ -22,8 +22,7 @@
 //   W_up         16 rows x K/4           waits: ylat (sh: a tile's last split) -> out rows
 // and the shared expert (an eighth of the grid) runs beside it:
 //   shared g/u   16 rows x K/8, g and u  MXFP4, x staged as fp16      -> sh_a rows, max |sh_a|
-//   shared down  16 rows x K             waits: all of sh_a           -> sh rows (tiles also taken by
-//                                                                        chain CTAs done with expert down)
+//   shared down  16 rows x K             waits: all of sh_a           -> sh rows
 // Every phase entry is a CTA-wide barrier (the phase's activations are staged once per CTA), so
 // the shared parts, which nothing on the chain needs before W_up, must not sit between the
 // chain's phases: a CTA there would hold the chain until its slowest shared item ends.
@@ -577,23 +576,6 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         __syncthreads();
     };
 
-    // Shared-expert down tiles go out through one global counter (claimed per warp): the shared
-    // CTAs start on them once sh_a is final, and routed-chain CTAs that are done with the expert
-    // down projection join in before W_up, whose last splits wait for sh.  Stages sh_a first.
-    auto shared_down_tiles = [&]() {
-        if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_shamax + threadIdx.x)));
-        __syncthreads();
-        stage_f16_from_f32<true>(xs, f16_pitch(Is), a.ws.sh_a, Is, B, [](int t) { return t; }, s_shift, 0, Is);
-        __syncthreads();
-        for (;;) {
-            int it = 0;
-            if (lane == 0) it = (int)atomicAdd(ctl + CTL_QHEAD + QS_SD, 1u);
-            it = __shfl_sync(0xffffffffu, it, 0);
-            if (it >= n_sd) break;
-            w_sd(a, it, xs, s_shift);
-        }
-    };
-
     cta_take_init(claim);
     if (sh_cta) {
         // ---- shared expert CTAs: gate/up on x, then down on sh_a (off the routed chain) ----
@@ -616,9 +598,15 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         __syncthreads();
         warp_queue(QS_SGU, n_sgu, c_sh, G_sh, [&](int it) { w_sgu(a, it, xs, s_shift); return true; });
         stamp(4);
-        // shared down: all of sh_a final; stage it (fp16 hi/lo); tiles from the shared queue
+        // shared down: all of sh_a final; stage it (fp16 hi/lo)
         alive = cta_wait_geq(a, ctl + CTL_SGU_DONE, (unsigned)(Is / 16), &s_ok);
-        if (alive) shared_down_tiles();
+        if (alive) {
+            if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_shamax + threadIdx.x)));
+            __syncthreads();
+            stage_f16_from_f32<true>(xs, f16_pitch(Is), a.ws.sh_a, Is, B, [](int t) { return t; }, s_shift, 0, Is);
+            __syncthreads();
+            warp_queue(QS_SD, n_sd, c_sh, G_sh, [&](int it) { w_sd(a, it, xs, s_shift); return true; });
+        }
         stamp(7);
         prefetch_next_router(a, c_sh, G_sh);  // nothing left to do here: pull the next layer's router
     } else {
@@ -669,16 +657,6 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
             alive = __syncthreads_and(ok) != 0;
         }
         stamp(8);
-        // shared down tiles still unclaimed: take some before W_up (sh_a is final by now in
-        // practice; the wait is bounded like every other)
-        if (alive && a.d.n_shared) {
-            if (threadIdx.x == 0) s_ok = ld_acquire(ctl + CTL_QHEAD + QS_SD) < (unsigned)n_sd ? 1 : 0;
-            __syncthreads();
-            if (s_ok) {
-                alive = cta_wait_geq(a, ctl + CTL_SGU_DONE, (unsigned)(Is / 16), &s_ok);
-                if (alive) shared_down_tiles();
-            }
-        }
         // W_up: every ylat block complete (all B*k entries added); stage ylat (bf16 hi/lo).  The
         // shared expert's sh is awaited only by the warp that completes each tile
         if (alive) {
