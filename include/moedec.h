@@ -74,6 +74,10 @@ typedef enum moedec_status {
                                           streaming kernel (each warp streams its work items through
                                           a shared-memory ring of cp.async stages) instead of the
                                           small-batch persistent kernel */
+#define MOEDEC_FLAG_NO_TMA_RING 64u    /* batches above 4 tokens: stage each expert segment's activations
+                                          in shared memory and stream its weights through registers,
+                                          instead of the per-warp TMA weight rings (the default when
+                                          latent/256 and expert_inter/256 are 1, 2, 4 or 8) */
 #define MOEDEC_TRACE_STAMPS 16         /* stamps per CTA */
 
 typedef struct moedec_config {
@@ -156,6 +160,15 @@ MOEDEC_API int moedec_destroy(moedec_handle *h);
  * Errors: INVALID_ARG (NULL h, mismatched next).
  */
 MOEDEC_API int moedec_set_next(moedec_handle *h, const moedec_handle *next);
+
+/*
+ * Which path the routed experts of the split-K step (batches above 4 tokens) take on this handle:
+ * 1 = per-warp TMA weight rings (tensor maps over gate_q, up_q and down_q were made at create),
+ * 0 = activation staging per segment with register-fed weight loads (MOEDEC_FLAG_NO_TMA_RING, or
+ * latent/256 or expert_inter/256 not in {1, 2, 4, 8}).  Both give results within the float
+ * tolerance of each other (the order of fp32 sums differs).  Returns MOEDEC_ERR_INVALID_ARG for NULL h.
+ */
+MOEDEC_API int moedec_tma_ring(const moedec_handle *h);
 
 /*
  * Routing of the last step, copied on `stream` into caller device buffers:

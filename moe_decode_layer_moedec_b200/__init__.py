@@ -23,6 +23,7 @@ FLAG_TEST_STALL = 4
 FLAG_MULTI_KERNEL = 8
 FLAG_TRACE = 16
 FLAG_STREAM = 32
+FLAG_NO_TMA_RING = 64
 TRACE_STAMPS = 16
 STATUS = {0: "MOEDEC_OK", -1: "MOEDEC_ERR_INVALID_ARG", -2: "MOEDEC_ERR_UNSUPPORTED", -3: "MOEDEC_ERR_CUDA",
           -4: "MOEDEC_ERR_OOM", -5: "MOEDEC_ERR_TIMEOUT", -6: "MOEDEC_ERR_DEVICE"}
@@ -68,6 +69,8 @@ def _load():
     lib.moedec_get_taps.restype = i32
     lib.moedec_set_next.argtypes = [vp, vp]
     lib.moedec_set_next.restype = i32
+    lib.moedec_tma_ring.argtypes = [vp]
+    lib.moedec_tma_ring.restype = i32
     lib.moedec_get_scores.argtypes = [vp, vp, i32, vp]
     lib.moedec_get_scores.restype = i32
     lib.moedec_get_launch_counts.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(i32)]
@@ -184,6 +187,13 @@ class MoeDecodeLayer:
         """Prefetch hint: steps of this layer pull `nxt`'s router rows into L2 (None clears it)."""
         self._next = nxt  # keep the next layer's handle (and its router tensor) alive
         self._check("moedec_set_next", lib.moedec_set_next(self._h, nxt._h if nxt is not None else None))
+
+    def tma_ring(self) -> bool:
+        """True when the split-K step streams the routed experts through per-warp TMA rings."""
+        r = lib.moedec_tma_ring(self._h)
+        if r < 0:
+            self._check("moedec_tma_ring", r)
+        return r == 1
 
     def scores(self, batch: int, stream=None):
         """fp32 router scores [B, E] of the last step, from the same device function the top-k uses."""

@@ -19,6 +19,7 @@ struct moedec_handle {
     Weights w;
     Plan p;
     Work ws;
+    ExpertMaps maps;  // TMA maps of the expert codes (maps.ok == 0: none)
     void *buf = nullptr;
     size_t buf_bytes = 0;
     cudaStream_t side = nullptr;
@@ -65,6 +66,42 @@ SplitPlan split(int rows, int rows_per_block, int K) {
     s.krange = krange_for(K);
     s.splits = K / s.krange;
     return s;
+}
+
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                      const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                      CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 2D uint8 map over `rows` rows of `row_bytes` bytes: boxes of 8 rows x 128 bytes, 128-byte swizzle.
+bool encode_rows(TensorMapEncodeFn fn, CUtensorMap *m, const void *base, uint64_t row_bytes, uint64_t rows) {
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {128, 8}, elem[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, elem,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The expert code maps of the split-K step's ring phases; left with ok == 0 (the step then stages
+// activations per segment and streams weights through registers) when the dims do not fit, the
+// driver has no tensor-map encoder, or MOEDEC_FLAG_NO_TMA_RING is set.
+void make_expert_maps(moedec_handle *h) {
+    ExpertMaps &m = h->maps;
+    memset(&m, 0, sizeof(m));
+    const Dims &d = h->d;
+    if ((h->cfg.flags & MOEDEC_FLAG_NO_TMA_RING) || !ring_dims_ok(d)) return;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return;
+    }
+    const TensorMapEncodeFn enc = reinterpret_cast<TensorMapEncodeFn>(fn);
+    const bool ok = encode_rows(enc, &m.gate, h->w.gate_q, (uint64_t)d.L / 2, (uint64_t)d.E * d.I) &&
+                    encode_rows(enc, &m.up, h->w.up_q, (uint64_t)d.L / 2, (uint64_t)d.E * d.I) &&
+                    encode_rows(enc, &m.down, h->w.down_q, (uint64_t)d.I / 2, (uint64_t)d.E * d.L);
+    m.ok = ok ? 1 : 0;
 }
 
 // carve aligned sub-buffers from one allocation
@@ -300,6 +337,7 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     }
     if (e != cudaSuccess) rc = record_cuda(h, e);
     if (rc == MOEDEC_OK && !(c.flags & MOEDEC_FLAG_SKIP_SCALE_CHECK)) rc = check_scales(h);
+    if (rc == MOEDEC_OK) make_expert_maps(h);
     if (rc != MOEDEC_OK) {
         moedec_destroy(h);
         return rc;
@@ -352,7 +390,7 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
         else if (fused_small_supports(h->d, batch))
             e = timed(h, K_FUSED_SMALL, s, [&] { return launch_fused_small(a, s, h->n_sm); });
         else
-            e = timed(h, K_FUSED, s, [&] { return launch_fused(a, s, h->n_sm); });
+            e = timed(h, K_FUSED, s, [&] { return launch_fused(a, h->maps, s, h->n_sm); });
         if (e != cudaSuccess) return record_cuda(h, e);
         h->launches[variant] += (uint64_t)moedec_kernels_per_step(h, batch);
         h->last_batch = batch;
@@ -383,6 +421,11 @@ MOEDEC_API int moedec_set_next(moedec_handle *h, const moedec_handle *next) {
     if (next && (next->d.H != h->d.H || next->d.E != h->d.E || next->device != h->device)) return MOEDEC_ERR_INVALID_ARG;
     h->next_router = next ? next->w.router : nullptr;
     return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_tma_ring(const moedec_handle *h) {
+    if (!h) return MOEDEC_ERR_INVALID_ARG;
+    return h->maps.ok ? 1 : 0;
 }
 
 MOEDEC_API int moedec_get_routing(moedec_handle *h, int32_t *idx, float *w, int batch, void *stream) {

@@ -21,7 +21,7 @@
 // Routing is known only after queue 1, but nothing waits for a kernel boundary: while one CTA
 // ranks the experts the others already stream W_dn and the shared expert, and an expert's down
 // rows start as soon as its own gate/up rows are done.
-#include "moedec_experts.cuh"
+#include "moedec_ring.cuh"
 
 namespace moedec {
 
@@ -80,13 +80,16 @@ __host__ __device__ inline size_t fused_stage_smem(const StepArgs &a) {
     return (m + 15) & ~(size_t)15;
 }
 
+// Dynamic shared memory of a launch: with the TMA rings the expert phases read the routing from
+// global memory and the route tables are not kept (ring and staging buffers share offset 0).
 template <int TIER>
-__host__ __device__ inline size_t fused_smem(const StepArgs &a) {
-    return fused_stage_smem<TIER>(a) + sizeof(typename Tier<TIER>::RT);
+__host__ __device__ inline size_t fused_smem(const StepArgs &a, bool ring) {
+    const size_t st = fused_stage_smem<TIER>(a), r = ring_smem(ring_stages(Tier<TIER>::MINB));
+    return ring ? (st > r ? st : r) : st + sizeof(typename Tier<TIER>::RT);
 }
 
 template <int TIER>
-__global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
+__global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, const __grid_constant__ ExpertMaps maps) {
     using T = Tier<TIER>;
     using RT = typename T::RT;
     extern __shared__ __align__(16) unsigned char smem[];
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
     __shared__ SegSmem segs;
     __shared__ int s_scan[32];
     __shared__ int s_next;
+    __shared__ RingSync rs;
     unsigned *ctl = a.ws.ctl;
     bool alive = true;
     const int n_rt = a.p.rt.blocks * a.p.rt.splits, n_dn = a.p.dn.blocks * a.p.dn.splits;
@@ -109,6 +113,12 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
         if (trace && threadIdx.x == 0) trace[i] = global_ns();
     };
     stamp(0);
+    constexpr int NSW = ring_stages(T::MINB);
+    const bool use_ring = maps.ok != 0;
+    uint8_t *ring = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);  // 1 KB aligned (128-byte swizzle)
+    float4 *ring_part = reinterpret_cast<float4 *>(ring + 8 * NSW * kRingBytes);
+    unsigned ring_pos = 0;
+    if (use_ring) ring_init(rs);
 
     // Items are taken dynamically, one atomic per item on the queue head, each when the CTA is
     // ready for it.  (Claiming one item ahead, to prefetch its weights into L2, let the first CTAs
@@ -152,7 +162,20 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
         hi = (int)((long long)n * (blockIdx.x + 1) / gridDim.x);
     };
     uint16_t *xs_e = reinterpret_cast<uint16_t *>(smem);
-    if (alive) {
+    int n_act = 0;
+    if (alive && use_ring) {
+        n_act = __ldcg(a.ws.n_active);
+        ring_plan(a, segp, s_scan, n_act);
+        if (threadIdx.x < 8 * kRingSlots) {
+            rs.cnt[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
+            rs.gen[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
+        }
+        __syncthreads();
+        int lo, hi;
+        range((a.d.I / 8) * segp.ngroups, lo, hi);
+        const bool ok = ring_phase<true, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+        alive = __syncthreads_and(ok ? 1 : 0) != 0;
+    } else if (alive) {
         cta_load_routing(a, route);
         __syncthreads();
         seg_plan<seg_tok(T::MINB)>(segp, route, s_scan);
@@ -173,12 +196,26 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
     // expert's gate/up tiles
     if (alive) {
         __syncthreads();
-        const int nb = a.d.L / 128;
-        int lo, hi;
-        range(nb * segp.ngroups, lo, hi);
-        const bool ok = for_each_segment(segp, route, nb, lo, hi, [&](int j, int g, int b0, int b1) {
-            return seg_down_any<T::MINB>(a, route, segs, xs_e, j, g, b0, b1);
-        });
+        bool ok;
+        if (use_ring) {
+            if (threadIdx.x < 8 * kRingSlots) {
+                rs.cnt[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
+                rs.gen[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
+            }
+            for (int i = threadIdx.x; i < kRingMaxBlocks; i += blockDim.x) rs.blk[i] = 0u;
+            __syncthreads();
+            int lo, hi;
+            range((a.d.L / 16) * segp.ngroups, lo, hi);
+            ok = ring_phase<false, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+            ring_publish_down(a, rs);
+        } else {
+            const int nb = a.d.L / 128;
+            int lo, hi;
+            range(nb * segp.ngroups, lo, hi);
+            ok = for_each_segment(segp, route, nb, lo, hi, [&](int j, int g, int b0, int b1) {
+                return seg_down_any<T::MINB>(a, route, segs, xs_e, j, g, b0, b1);
+            });
+        }
         alive = __syncthreads_and(ok ? 1 : 0) != 0;
     }
     stamp(8);
@@ -206,8 +243,8 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a) {
 }
 
 template <int TIER>
-static cudaError_t launch_fused_tier(const StepArgs &a, cudaStream_t s, int n_sm) {
-    const size_t sm = fused_smem<TIER>(a);
+static cudaError_t launch_fused_tier(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm) {
+    const size_t sm = fused_smem<TIER>(a, maps.ok != 0);
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_fused<TIER>, 256, sm);
     if (e != cudaSuccess) return e;
@@ -223,16 +260,16 @@ static cudaError_t launch_fused_tier(const StepArgs &a, cudaStream_t s, int n_sm
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fused<TIER>, a);
+    return cudaLaunchKernelEx(&cfg, k_fused<TIER>, a, maps);
 }
 
-cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm) {
+cudaError_t launch_fused(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm) {
     switch (tier_for_batch(a.B)) {
-        case 0: return launch_fused_tier<0>(a, s, n_sm);
-        case 1: return launch_fused_tier<1>(a, s, n_sm);
-        case 2: return launch_fused_tier<2>(a, s, n_sm);
-        case 3: return launch_fused_tier<3>(a, s, n_sm);
-        default: return launch_fused_tier<4>(a, s, n_sm);
+        case 0: return launch_fused_tier<0>(a, maps, s, n_sm);
+        case 1: return launch_fused_tier<1>(a, maps, s, n_sm);
+        case 2: return launch_fused_tier<2>(a, maps, s, n_sm);
+        case 3: return launch_fused_tier<3>(a, maps, s, n_sm);
+        default: return launch_fused_tier<4>(a, maps, s, n_sm);
     }
 }
 

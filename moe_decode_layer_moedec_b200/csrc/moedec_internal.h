@@ -1,6 +1,7 @@
 // moedec_internal.h -- parameter blocks shared by the host orchestration and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -143,6 +144,21 @@ struct StepArgs {
     unsigned flags;     // MOEDEC_FLAG_* of the handle
 };
 
+// TMA tensor maps of the routed experts' MXFP4 codes (2D uint8 [rows][K/2 bytes]: gate and up
+// E*I rows of L/2 bytes, down E*L rows of I/2 bytes), boxes of 8 rows x 128 bytes with the
+// 128-byte swizzle.  Made at create when L/256 and I/256 are 1, 2, 4 or 8; `ok` is 0 otherwise
+// (the split-K step then stages the experts' activations per segment instead).
+struct alignas(64) ExpertMaps {
+    CUtensorMap gate, up, down;
+    int ok;
+};
+
+// K dimensions the ring phases cover: L/256 and I/256 in {1, 2, 4, 8} (one 128-byte line of a row per warp)
+__host__ __device__ inline bool ring_dims_ok(const Dims &d) {
+    auto ok = [](int k) { return k % 256 == 0 && (k / 256 == 1 || k / 256 == 2 || k / 256 == 4 || k / 256 == 8); };
+    return ok(d.L) && ok(d.I);
+}
+
 // error word bits
 constexpr unsigned kErrBucket = 1u;    // routing bucket overflow (internal invariant)
 constexpr unsigned kErrTimeout = 2u;   // a bounded device wait gave up
@@ -158,7 +174,7 @@ cudaError_t launch_shared_gate_up(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_shared_down(const StepArgs &a, cudaStream_t s);
 cudaError_t launch_scale_check(const uint8_t *s, size_t n, unsigned *bad, cudaStream_t st);
 cudaError_t launch_scores(const float *logits, float *scores, size_t n, cudaStream_t st);
-cudaError_t launch_fused(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t launch_fused(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm);
 cudaError_t init_fused_attributes();
 constexpr int kStreamLaunches = 4;  // launches of the streaming small-batch step
 bool stream_supports(const Dims &d, int B);

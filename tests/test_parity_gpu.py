@@ -28,12 +28,18 @@ SCHEDULES = ["fused", "multi", "stream"]
 
 
 def _make_layer(w, W_dev, max_batch, flags=None, schedule="fused"):
-    from moe_decode_layer_moedec_b200 import FLAG_MULTI_KERNEL, FLAG_STREAM, FLAG_TAPS, MoeDecodeLayer
+    # schedules: "fused" (the default), "multi" (eight stream-ordered kernels), "stream" (the
+    # streaming small-batch kernel at 1-2 tokens), "noring" (fused, with the split-K step's
+    # routed experts on register-fed loads instead of the per-warp TMA rings)
+    from moe_decode_layer_moedec_b200 import (FLAG_MULTI_KERNEL, FLAG_NO_TMA_RING, FLAG_STREAM, FLAG_TAPS,
+                                              MoeDecodeLayer)
     f = FLAG_TAPS if flags is None else flags
     if schedule == "multi":
         f |= FLAG_MULTI_KERNEL
     if schedule == "stream":
         f |= FLAG_STREAM
+    if schedule == "noring":
+        f |= FLAG_NO_TMA_RING
     return MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=max_batch, flags=f)
 
 
@@ -105,6 +111,18 @@ def test_mid_parity(mid, B, schedule):
         assert layer.kernels_per_step(B) == 4  # the streaming kernel ran (4 launches per step)
 
 
+@pytest.mark.parametrize("B", [5, 13, 64])
+@pytest.mark.parametrize("schedule", ["fused", "noring"])
+def test_mid_split_k_parity(mid, B, schedule):
+    # L = I = 512: two 128-byte lines per row, so the ring phases run four row groups of two
+    # warps that add their K halves in shared memory
+    w, W, W_dev = mid
+    x = synth.tokens(w, step=B, batch=B)
+    layer = _make_layer(w, W_dev, max_batch=B, schedule=schedule)
+    assert layer.tma_ring() == (schedule == "fused")
+    _check_step(w, W, x, layer, label=f"mid B{B} {schedule}")
+
+
 @pytest.mark.parametrize("schedule", ["fused", "stream"])
 def test_mid_back_to_back_and_graph(mid, torch_cuda, schedule):
     # consecutive steps of different tokens, eager and replayed from a CUDA graph, agree with a
@@ -166,6 +184,16 @@ def test_tiny_parity(tiny, B, schedule):
     layer = _make_layer(w, W_dev, max_batch=max(64, B), schedule=schedule)
     x = synth.tokens(w, step=B, batch=B)
     _check_step(w, W, x, layer, label=f"tiny B{B} {schedule}")
+
+
+@pytest.mark.parametrize("B", [5, 9, 17, 64, 65, 200, 512])
+def test_tiny_parity_register_path(tiny, B):
+    # the split-K step's routed experts on register-fed loads (MOEDEC_FLAG_NO_TMA_RING)
+    w, W, W_dev = tiny
+    layer = _make_layer(w, W_dev, max_batch=max(64, B), schedule="noring")
+    assert not layer.tma_ring()
+    x = synth.tokens(w, step=B, batch=B)
+    _check_step(w, W, x, layer, label=f"tiny B{B} noring")
 
 
 @pytest.mark.parametrize("schedule", SCHEDULES)
@@ -356,13 +384,14 @@ def test_full_small_batches_all_tokens(full_layers, name, schedule):
 
 # Above two tokens the streaming schedule is the split-K kernel too, so B >= 16 runs the fused
 # split-K kernel and the multi-kernel schedule; layer 15 and 31 as well as 0 (distinct weights).
-LARGE_CASES = [(l, s) for l in (0, 15, 31) for s in ("fused", "multi")]
+LARGE_CASES = [(l, s) for l in (0, 15, 31) for s in ("fused", "multi")] + [(0, "noring")]
 
 
 @pytest.mark.parametrize("layer_idx,schedule", LARGE_CASES)
 def test_full_b16_all_tokens(full_layers, layer_idx, schedule):
     w, W, W_dev = full_layers("full_b16", layer_idx)
     layer = _make_layer(w, W_dev, max_batch=w.batch, schedule=schedule)
+    assert layer.tma_ring() == (schedule != "noring")
     x = synth.tokens(w)
     _check_step(w, W, x, layer, label=f"full_b16 L{layer_idx} {schedule}", layer_idx=layer_idx)
 
@@ -393,7 +422,7 @@ def _tiny_skewed(B, hot, beta, seed):
     return synth.Workload(f"tiny_hot{hot}_b{B}", synth.TINY, B, seed, hot_experts=hot, hot_beta=beta)
 
 
-@pytest.mark.parametrize("schedule", ["fused", "multi"])
+@pytest.mark.parametrize("schedule", ["fused", "multi", "noring"])
 def test_tiny_hot_experts_token_groups(torch_cuda, schedule):
     # 8 hot experts of 64 at B = 64 (k = 4, beta = 4): experts take 1..4, 5..8, 9..16 and 17..32
     # tokens, so an expert item runs one or two 16-token groups on either operand path
@@ -409,7 +438,7 @@ def test_tiny_hot_experts_token_groups(torch_cuda, schedule):
 
 
 @pytest.mark.parametrize("B", [17, 64])
-@pytest.mark.parametrize("schedule", ["fused", "multi"])
+@pytest.mark.parametrize("schedule", ["fused", "multi", "noring"])
 def test_tiny_identical_tokens_one_expert_takes_every_token(tiny, B, schedule):
     # B copies of one token: each of its k experts receives all B tokens (the largest bucket: up
     # to four 16-token groups of one expert item)
