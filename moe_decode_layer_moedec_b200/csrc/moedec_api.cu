@@ -388,7 +388,7 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
         if ((h->cfg.flags & MOEDEC_FLAG_STREAM) && stream_supports(h->d, batch))
             e = timed(h, K_FUSED_STREAM, s, [&] { return launch_stream(a, s, h->n_sm); });
         else if (fused_small_supports(h->d, batch))
-            e = timed(h, K_FUSED_SMALL, s, [&] { return launch_fused_small(a, s, h->n_sm); });
+            e = timed(h, K_FUSED_SMALL, s, [&] { return launch_fused_small(a, h->maps, s, h->n_sm); });
         else
             e = timed(h, K_FUSED, s, [&] { return launch_fused(a, h->maps, s, h->n_sm); });
         if (e != cudaSuccess) return record_cuda(h, e);

@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
     uint8_t *ring = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);  // 1 KB aligned (128-byte swizzle)
     float4 *ring_part = reinterpret_cast<float4 *>(ring + 8 * NSW * kRingBytes);
     unsigned ring_pos = 0;
-    if (use_ring) ring_init(rs);
+    if (use_ring) ring_init(rs, maps);
 
     // Items are taken dynamically, one atomic per item on the queue head, each when the CTA is
     // ready for it.  (Claiming one item ahead, to prefetch its weights into L2, let the first CTAs
@@ -263,7 +263,11 @@ static cudaError_t launch_fused_tier(const StepArgs &a, const ExpertMaps &maps, 
     return cudaLaunchKernelEx(&cfg, k_fused<TIER>, a, maps);
 }
 
-cudaError_t launch_fused(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm) {
+cudaError_t launch_fused(const StepArgs &a, const ExpertMaps &maps_in, cudaStream_t s, int n_sm) {
+    // above 64 tokens (one CTA of 8 warps per SM) the register path with 16-token expert groups
+    // is faster than the rings (B = 256: 2,517 against 2,926 us): too few consumer warps per SM
+    ExpertMaps maps = maps_in;
+    if (tier_for_batch(a.B) == 4) maps.ok = 0;
     switch (tier_for_batch(a.B)) {
         case 0: return launch_fused_tier<0>(a, maps, s, n_sm);
         case 1: return launch_fused_tier<1>(a, maps, s, n_sm);

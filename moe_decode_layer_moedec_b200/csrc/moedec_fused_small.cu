@@ -28,7 +28,7 @@
 // chain's phases: a CTA there would hold the chain until its slowest shared item ends.
 #include <algorithm>
 
-#include "moedec_items.cuh"
+#include "moedec_ring.cuh"
 
 namespace moedec {
 
@@ -513,7 +513,7 @@ DEVI bool w_up(const StepArgs &a, int item, const uint16_t *ys) {
 // ---------------------------------------------------------------------------------------------
 // the kernel
 
-__host__ __device__ inline size_t fused_small_smem(const StepArgs &a) {
+__host__ __device__ inline size_t fused_small_smem(const StepArgs &a, bool ring) {
     const int B = a.B;
     size_t m = (size_t)B * bf16_pitch(a.d.H) * 2;                        // x, bf16
     auto mx = [&](size_t v) { m = v > m ? v : m; };
@@ -522,17 +522,28 @@ __host__ __device__ inline size_t fused_small_smem(const StepArgs &a) {
     mx((size_t)2 * B * f16_pitch(a.d.Is) * 2);                            // sh_a, fp16 hi/lo
     mx((size_t)kWarps * 2 * B * f16_pitch(edown_kc(a.d.I, B)) * 2);  // a, per warp
     mx((size_t)2 * B * bf16_pitch(a.d.L) * 2);                            // ylat, bf16 hi/lo
+    if (ring) mx(ring_smem(kRingStagesSmall));                              // expert TMA rings
     return m;
 }
 
-__global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
+__global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a, const __grid_constant__ ExpertMaps maps) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ TopkSmem topk;
     __shared__ int s_shift[kSmallMaxBatch], s_ok;
     __shared__ unsigned s_amax[kSmallMaxBatch];
     __shared__ CtaTake claim;
     __shared__ RouteSmem route;
+    __shared__ RingSync rs;
+    __shared__ SegPlan segp;
+    __shared__ int s_scan[32];
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
+    // routed experts through the per-warp TMA rings (as in the split-K step), when the maps exist
+    constexpr int NSW = kRingStagesSmall;
+    const bool use_ring = maps.ok != 0;
+    uint8_t *ring = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+    float4 *ring_part = reinterpret_cast<float4 *>(ring + 8 * NSW * kRingBytes);
+    unsigned ring_pos = 0;
+    if (use_ring) ring_init(rs, maps);
     unsigned *ctl = a.ws.ctl;
     const int H = a.d.H, L = a.d.L, I = a.d.I, Is = a.d.Is, B = a.B, E = a.d.E;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -638,7 +649,28 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
         stamp(11);
         if (alive) alive = cta_wait_geq(a, ctl + CTL_DN_DONE, (unsigned)(L / 16), &s_ok);
         stamp(5);
-        if (alive) {
+        auto range = [&](int n, int &lo, int &hi) {  // the chain CTAs' static split of a ring phase
+            lo = (int)((long long)n * c_m / G_m);
+            hi = (int)((long long)n * (c_m + 1) / G_m);
+        };
+        auto ring_counters = [&]() {
+            if (threadIdx.x < 8 * kRingSlots) {
+                rs.cnt[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
+                rs.gen[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
+            }
+            for (int i = threadIdx.x; i < kRingMaxBlocks; i += blockDim.x) rs.blk[i] = 0u;
+        };
+        int n_act = 0;
+        if (alive && use_ring) {
+            n_act = __ldcg(a.ws.n_active);
+            ring_plan(a, segp, s_scan, n_act);
+            ring_counters();
+            __syncthreads();
+            int lo, hi;
+            range((I / 8) * segp.ngroups, lo, hi);
+            const bool ok = ring_phase<true, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+            alive = __syncthreads_and(ok ? 1 : 0) != 0;
+        } else if (alive) {
             if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
             cta_load_routing(a, route);
             __syncthreads();
@@ -648,8 +680,17 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a) {
             warp_queue(QS_EGU, n, c_m, G_m, [&](int it) { w_egu(a, route, it, xs, s_shift); return true; });
         }
         stamp(6);
-        // expert down (per-warp staging of the expert's entries)
-        if (alive) {
+        // expert down (ring phase, or per-warp staging of the expert's entries)
+        if (alive && use_ring) {
+            __syncthreads();
+            ring_counters();
+            __syncthreads();
+            int lo, hi;
+            range((L / 16) * segp.ngroups, lo, hi);
+            const bool ok = ring_phase<false, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+            ring_publish_down(a, rs);
+            alive = __syncthreads_and(ok ? 1 : 0) != 0;
+        } else if (alive) {
             __syncthreads();
             const int n = route.n_active * (L / 16);
             uint16_t *ws = xs + (size_t)warp * 2 * B * f16_pitch(edown_kc(I, B));
@@ -709,9 +750,13 @@ bool fused_small_supports(const Dims &d, int B) {
            (d.n_shared == 0 || d.Is % 128 == 0) && d.k <= kMaxTopK && smem <= kSmallSmemLimit;
 }
 
-cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm) {
+cudaError_t launch_fused_small(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm) {
     int per_sm = 0;
-    const size_t sm = fused_small_smem(a);
+    // one token: the register path (the ring's shared memory costs the register-fed phases more L1
+    // than its few units per warp gain); two to four tokens: the TMA rings
+    ExpertMaps m = maps;
+    if (a.B < 2) m.ok = 0;
+    const size_t sm = fused_small_smem(a, m.ok != 0);
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_fused_small, 256, sm);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
@@ -726,7 +771,7 @@ cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_fused_small, a);
+    return cudaLaunchKernelEx(&cfg, k_fused_small, a, m);
 }
 
 cudaError_t init_fused_small_attributes() {

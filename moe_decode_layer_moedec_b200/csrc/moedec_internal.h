@@ -182,7 +182,7 @@ void stream_plan(const Dims &d, StreamPlan &sp, int ctl_base);
 cudaError_t launch_stream(const StepArgs &a, cudaStream_t s, int n_sm);
 cudaError_t init_stream_attributes();
 bool fused_small_supports(const Dims &d, int B);
-cudaError_t launch_fused_small(const StepArgs &a, cudaStream_t s, int n_sm);
+cudaError_t launch_fused_small(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm);
 cudaError_t init_fused_small_attributes();
 int kernels_per_step(const Dims &d);
 cudaError_t init_kernel_attributes();

@@ -30,12 +30,13 @@
 namespace moedec {
 
 constexpr int kRingBytes = 2048;  // one stage: two boxes of 8 rows x 128 bytes
-constexpr int kRingSlots = 4;     // partial-sum slots per row group
+constexpr int kRingSlots = 2;     // partial-sum slots per row group
 constexpr int kRingMaxStages = 6;
 constexpr int kRingTok = 8;       // tokens per group (one 8-column MMA tile)
 constexpr int kRingMaxBlocks = 128;  // 16-row blocks of L (L <= 2048 on the ring path)
 
-__host__ __device__ constexpr int ring_stages(int minb) { return minb > 1 ? 4 : 6; }
+__host__ __device__ constexpr int ring_stages(int minb) { return minb > 1 ? 3 : 6; }
+constexpr int kRingStagesSmall = 2;  // small-batch step: a few units per warp, keep the L1 share
 
 // dynamic shared memory of the ring phases (1 KB of alignment slack, the rings, the partials)
 __host__ __device__ inline size_t ring_smem(int nsw) {
@@ -180,11 +181,17 @@ DEVI void ring_plan(const StepArgs &a, SegPlan &sp, int *s_warp, int n_active) {
     if (threadIdx.x == 0) sp.ngroups = n;
 }
 
-// all threads, once per kernel before the first barrier: every warp's stage barriers
-DEVI void ring_init(RingSync &rs) {
+// all threads, once per kernel before the first barrier: every warp's stage barriers, and the
+// three tensor maps fetched ahead into the TMA unit's descriptor cache
+DEVI void ring_init(RingSync &rs, const ExpertMaps &maps) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane < kRingMaxStages) mbar_init(smem_u32(&rs.full[warp][lane]), 1u);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (threadIdx.x == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.gate) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.up) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.down) : "memory");
+    }
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -186,9 +186,9 @@ def test_tiny_parity(tiny, B, schedule):
     _check_step(w, W, x, layer, label=f"tiny B{B} {schedule}")
 
 
-@pytest.mark.parametrize("B", [5, 9, 17, 64, 65, 200, 512])
+@pytest.mark.parametrize("B", [1, 2, 3, 5, 9, 17, 64, 65, 200, 512])
 def test_tiny_parity_register_path(tiny, B):
-    # the split-K step's routed experts on register-fed loads (MOEDEC_FLAG_NO_TMA_RING)
+    # the fused steps' routed experts on register-fed loads (MOEDEC_FLAG_NO_TMA_RING)
     w, W, W_dev = tiny
     layer = _make_layer(w, W_dev, max_batch=max(64, B), schedule="noring")
     assert not layer.tma_ring()
