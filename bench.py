@@ -180,10 +180,10 @@ class ClockSampler:
 KERNEL_SOURCES = {
     "fused_step_stream": ["moedec_stream.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
                           "moedec_router.cuh", "moedec_internal.h"],
-    "fused_step_small": ["moedec_fused_small.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
-                         "moedec_router.cuh", "moedec_internal.h"],
-    "fused_step_splitk": ["moedec_fused.cu", "moedec_experts.cuh", "moedec_items.cuh", "moedec_tiles.cuh",
-                          "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h"],
+    "fused_step_small": ["moedec_fused_small.cu", "moedec_ring.cuh", "moedec_experts.cuh", "moedec_items.cuh",
+                         "moedec_tiles.cuh", "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h"],
+    "fused_step_splitk": ["moedec_fused.cu", "moedec_ring.cuh", "moedec_experts.cuh", "moedec_items.cuh",
+                          "moedec_tiles.cuh", "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h"],
 }
 
 
