@@ -165,9 +165,9 @@ MOEDEC_API int moedec_set_next(moedec_handle *h, const moedec_handle *next);
  * Whether this handle can stream the routed experts of the fused steps through per-warp TMA
  * weight rings: 1 when create made tensor maps over gate_q, up_q and down_q, 0 with
  * MOEDEC_FLAG_NO_TMA_RING or when latent/256 or expert_inter/256 is not in {1, 2, 4, 8}.  With 1,
- * steps of 2 to 64 tokens use the rings; 1 token and more than 64 tokens keep the register-fed
- * expert path, which is faster there.  Both paths agree within the float tolerance (the order of
- * fp32 sums differs).  Returns MOEDEC_ERR_INVALID_ARG for NULL h.
+ * steps of 2 or more tokens use the rings; a step of 1 token keeps the register-fed expert path,
+ * which is faster there.  Both paths agree within the float tolerance (the order of fp32 sums
+ * differs).  Returns MOEDEC_ERR_INVALID_ARG for NULL h.
  */
 MOEDEC_API int moedec_tma_ring(const moedec_handle *h);
 

@@ -189,7 +189,7 @@ class MoeDecodeLayer:
         self._check("moedec_set_next", lib.moedec_set_next(self._h, nxt._h if nxt is not None else None))
 
     def tma_ring(self) -> bool:
-        """True when steps of 2-64 tokens stream the routed experts through per-warp TMA rings."""
+        """True when steps of 2 or more tokens stream the routed experts through per-warp TMA rings."""
         r = lib.moedec_tma_ring(self._h)
         if r < 0:
             self._check("moedec_tma_ring", r)

@@ -84,7 +84,7 @@ __host__ __device__ inline size_t fused_stage_smem(const StepArgs &a) {
 // global memory and the route tables are not kept (ring and staging buffers share offset 0).
 template <int TIER>
 __host__ __device__ inline size_t fused_smem(const StepArgs &a, bool ring) {
-    const size_t st = fused_stage_smem<TIER>(a), r = ring_smem(ring_stages(Tier<TIER>::MINB));
+    const size_t st = fused_stage_smem<TIER>(a), r = ring_rows_smem(ring_stages(Tier<TIER>::MINB), a.d);
     return ring ? (st > r ? st : r) : st + sizeof(typename Tier<TIER>::RT);
 }
 
@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
     constexpr int NSW = ring_stages(T::MINB);
     const bool use_ring = maps.ok != 0;
     uint8_t *ring = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);  // 1 KB aligned (128-byte swizzle)
-    float4 *ring_part = reinterpret_cast<float4 *>(ring + 8 * NSW * kRingBytes);
+    uint16_t *ring_xs = reinterpret_cast<uint16_t *>(ring + 8 * NSW * kRingBytes);
+    __shared__ RingGroup ring_gr;
     unsigned ring_pos = 0;
     if (use_ring) ring_init(rs, maps);
 
@@ -166,14 +167,10 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
     if (alive && use_ring) {
         n_act = __ldcg(a.ws.n_active);
         ring_plan(a, segp, s_scan, n_act);
-        if (threadIdx.x < 8 * kRingSlots) {
-            rs.cnt[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
-            rs.gen[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
-        }
         __syncthreads();
         int lo, hi;
         range((a.d.I / 8) * segp.ngroups, lo, hi);
-        const bool ok = ring_phase<true, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+        const bool ok = ring_rows<true, NSW>(a, maps, n_act, segp, rs, ring_gr, ring, ring_xs, lo, hi, ring_pos);
         alive = __syncthreads_and(ok ? 1 : 0) != 0;
     } else if (alive) {
         cta_load_routing(a, route);
@@ -198,15 +195,11 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
         __syncthreads();
         bool ok;
         if (use_ring) {
-            if (threadIdx.x < 8 * kRingSlots) {
-                rs.cnt[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
-                rs.gen[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
-            }
             for (int i = threadIdx.x; i < kRingMaxBlocks; i += blockDim.x) rs.blk[i] = 0u;
             __syncthreads();
             int lo, hi;
             range((a.d.L / 16) * segp.ngroups, lo, hi);
-            ok = ring_phase<false, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+            ok = ring_rows<false, NSW>(a, maps, n_act, segp, rs, ring_gr, ring, ring_xs, lo, hi, ring_pos);
             ring_publish_down(a, rs);
         } else {
             const int nb = a.d.L / 128;
@@ -263,11 +256,7 @@ static cudaError_t launch_fused_tier(const StepArgs &a, const ExpertMaps &maps, 
     return cudaLaunchKernelEx(&cfg, k_fused<TIER>, a, maps);
 }
 
-cudaError_t launch_fused(const StepArgs &a, const ExpertMaps &maps_in, cudaStream_t s, int n_sm) {
-    // above 64 tokens (one CTA of 8 warps per SM) the register path with 16-token expert groups
-    // is faster than the rings (B = 256: 2,517 against 2,926 us): too few consumer warps per SM
-    ExpertMaps maps = maps_in;
-    if (tier_for_batch(a.B) == 4) maps.ok = 0;
+cudaError_t launch_fused(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm) {
     switch (tier_for_batch(a.B)) {
         case 0: return launch_fused_tier<0>(a, maps, s, n_sm);
         case 1: return launch_fused_tier<1>(a, maps, s, n_sm);

@@ -522,7 +522,7 @@ __host__ __device__ inline size_t fused_small_smem(const StepArgs &a, bool ring)
     mx((size_t)2 * B * f16_pitch(a.d.Is) * 2);                            // sh_a, fp16 hi/lo
     mx((size_t)kWarps * 2 * B * f16_pitch(edown_kc(a.d.I, B)) * 2);  // a, per warp
     mx((size_t)2 * B * bf16_pitch(a.d.L) * 2);                            // ylat, bf16 hi/lo
-    if (ring) mx(ring_smem(kRingStagesSmall));                              // expert TMA rings
+    if (ring) mx(ring_rows_smem(kRingStagesSmall, a.d));                    // expert TMA rings
     return m;
 }
 
@@ -541,7 +541,8 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a, const __grid
     constexpr int NSW = kRingStagesSmall;
     const bool use_ring = maps.ok != 0;
     uint8_t *ring = smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
-    float4 *ring_part = reinterpret_cast<float4 *>(ring + 8 * NSW * kRingBytes);
+    uint16_t *ring_xs = reinterpret_cast<uint16_t *>(ring + 8 * NSW * kRingBytes);
+    __shared__ RingGroup ring_gr;
     unsigned ring_pos = 0;
     if (use_ring) ring_init(rs, maps);
     unsigned *ctl = a.ws.ctl;
@@ -654,10 +655,6 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a, const __grid
             hi = (int)((long long)n * (c_m + 1) / G_m);
         };
         auto ring_counters = [&]() {
-            if (threadIdx.x < 8 * kRingSlots) {
-                rs.cnt[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
-                rs.gen[threadIdx.x / kRingSlots][threadIdx.x % kRingSlots] = 0u;
-            }
             for (int i = threadIdx.x; i < kRingMaxBlocks; i += blockDim.x) rs.blk[i] = 0u;
         };
         int n_act = 0;
@@ -668,7 +665,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a, const __grid
             __syncthreads();
             int lo, hi;
             range((I / 8) * segp.ngroups, lo, hi);
-            const bool ok = ring_phase<true, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+            const bool ok = ring_rows<true, NSW>(a, maps, n_act, segp, rs, ring_gr, ring, ring_xs, lo, hi, ring_pos);
             alive = __syncthreads_and(ok ? 1 : 0) != 0;
         } else if (alive) {
             if (threadIdx.x < B) s_shift[threadIdx.x] = prescale_shift(__uint_as_float(__ldcg(ctl + a.p.ctl_hamax + threadIdx.x)));
@@ -687,7 +684,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a, const __grid
             __syncthreads();
             int lo, hi;
             range((L / 16) * segp.ngroups, lo, hi);
-            const bool ok = ring_phase<false, NSW>(a, maps, n_act, segp, rs, ring, ring_part, lo, hi, ring_pos);
+            const bool ok = ring_rows<false, NSW>(a, maps, n_act, segp, rs, ring_gr, ring, ring_xs, lo, hi, ring_pos);
             ring_publish_down(a, rs);
             alive = __syncthreads_and(ok ? 1 : 0) != 0;
         } else if (alive) {
