@@ -37,26 +37,31 @@ template <int TIER>
 struct Tier;
 template <> struct Tier<0> {
     static constexpr int NTX = 1, NTS = 1, NTU = 1, MINB = 2;
+    static constexpr int MAXB = 64;
     static constexpr bool SPLITS = true;
     using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
 };
 template <> struct Tier<1> {
     static constexpr int NTX = 1, NTS = 1, NTU = 2, MINB = 2;
+    static constexpr int MAXB = 64;
     static constexpr bool SPLITS = false;
     using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
 };
 template <> struct Tier<2> {
     static constexpr int NTX = 2, NTS = 2, NTU = 4, MINB = 2;
+    static constexpr int MAXB = 64;
     static constexpr bool SPLITS = false;
     using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
 };
 template <> struct Tier<3> {
     static constexpr int NTX = 4, NTS = 4, NTU = 4, MINB = 2;
+    static constexpr int MAXB = 64;
     static constexpr bool SPLITS = false;
     using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
 };
 template <> struct Tier<4> {
     static constexpr int NTX = 8, NTS = 8, NTU = 16, MINB = 1;
+    static constexpr int MAXB = kMaxBatch;
     static constexpr bool SPLITS = false;
     using RT = SplitKRoute;
 };
@@ -76,7 +81,7 @@ __host__ __device__ inline size_t fused_stage_smem(const StepArgs &a) {
     mx((size_t)8 * T::NTS * f16_pitch(a.p.sd.krange) * 2);
     mx((size_t)8 * T::NTU * bf16_pitch(up_chunk(T::NTU, a.p.up.krange)) * 2);
     mx(seg_smem(a.d, seg_tok(T::MINB)));
-    mx((size_t)a.d.E * ((a.B + 63) / 64) * 8);  // the bucket builder's token masks (B > 64)
+    mx(topk_lists_smem(a.d.E, a.B));  // the top-k's candidates, token masks and offsets
     return (m + 15) & ~(size_t)15;
 }
 
@@ -142,15 +147,14 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
     // take no W_dn or shared gate/up items: a CTA that ranked a token would claim them late and
     // enter its static range of the expert phase after the others
     for (int t = blockIdx.x; alive && t < a.B; t += gridDim.x)
-        alive = item_topk<true>(a, t, topk, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat, nullptr,
-                                reinterpret_cast<unsigned long long *>(smem));
+        alive = item_topk<true>(a, t, topk, smem, (unsigned)a.p.rt.blocks, nullptr, a.ws.ylat, nullptr);
     stamp(2);
     if ((int)blockIdx.x >= a.B || a.B >= (int)gridDim.x) {
         // 2: W_dn
-        cta_queue(Q_DN, n_dn, [&](int it) { item_dn<true, T::NTX>(a, it, smem, &s_flag); return true; });
+        cta_queue(Q_DN, n_dn, [&](int it) { item_dn<true, T::NTX, T::MAXB>(a, it, smem, &s_flag); return true; });
         stamp(3);
         // 3: shared gate/up
-        cta_queue(Q_SGU, n_sgu, [&](int it) { item_sgu<true, T::NTX>(a, it, smem, &s_flag); return true; });
+        cta_queue(Q_SGU, n_sgu, [&](int it) { item_sgu<true, T::NTX, T::MAXB>(a, it, smem, &s_flag); return true; });
     }
     stamp(4);
     // 4: expert gate/up: routing and all of h must be final; the CTA's static range of the
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
     }
     stamp(6);
     // 5: shared down
-    cta_queue(Q_SD, n_sd, [&](int it) { return item_sd<true, T::NTS, T::SPLITS>(a, it, smem, &s_flag, &s_ok); });
+    cta_queue(Q_SD, n_sd, [&](int it) { return item_sd<true, T::NTS, T::SPLITS, T::MAXB>(a, it, smem, &s_flag, &s_ok); });
     stamp(7);
     // 6: expert down: the same plan over L / 128 blocks per expert; each segment waits for its
     // expert's gate/up tiles

@@ -522,6 +522,7 @@ __host__ __device__ inline size_t fused_small_smem(const StepArgs &a, bool ring)
     mx((size_t)2 * B * f16_pitch(a.d.Is) * 2);                            // sh_a, fp16 hi/lo
     mx((size_t)kWarps * 2 * B * f16_pitch(edown_kc(a.d.I, B)) * 2);  // a, per warp
     mx((size_t)2 * B * bf16_pitch(a.d.L) * 2);                            // ylat, bf16 hi/lo
+    mx(topk_lists_smem(a.d.E, B));                                        // top-k lists
     if (ring) mx(ring_rows_smem(kRingStagesSmall, a.d));                    // expert TMA rings
     return m;
 }
@@ -638,7 +639,7 @@ __global__ void __launch_bounds__(256, 2) k_fused_small(StepArgs a, const __grid
         stamp(1);
         __syncthreads();
         for (int it = c_m; alive && it < B; it += G_m)
-            alive = item_topk<true>(a, it, topk, (unsigned)n_rt,
+            alive = item_topk<true>(a, it, topk, smem, (unsigned)n_rt,  // the top-k CTAs take no W_dn item: xs is free
                                     trace ? a.ws.trace + (size_t)(G + blockIdx.x) * kTraceStamps : nullptr, a.ws.ylat,
                                     a.ws.rt_acc);
         stamp(2);

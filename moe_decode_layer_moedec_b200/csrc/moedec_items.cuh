@@ -127,9 +127,10 @@ DEVI void item_router(const StepArgs &a, int bid, unsigned char *smem, unsigned 
 // h = W_dn x: one 128-row block x K range (bf16 MMAs); the block's last CTA publishes h rows and
 // folds their per-token max |h| into the token's staging exponent
 
-template <bool FUSED, int NT>
+// MAXB: tokens per step at most (sizes the per-token shared arrays of the dense items)
+template <bool FUSED, int NT, int MAXB = kMaxBatch>
 DEVI void item_dn(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
-    __shared__ unsigned s_amax[kMaxBatch];
+    __shared__ unsigned s_amax[MAXB];
     const int L = a.d.L, H = a.d.H, B = a.B, maxB = a.d.max_batch;
     const int rb = bid / a.p.dn.splits, ks = bid % a.p.dn.splits;
     const int KR = a.p.dn.krange, k0 = ks * KR;
@@ -196,9 +197,15 @@ struct TopkSmem {
     unsigned digit, want;
     int ok;
     unsigned flag;
-    unsigned long long mask[kMaxExperts];
-    int off[kMaxExperts];
 };
+
+// Shared memory of item_topk's candidate and bucket lists (bytes): max(E ceil(B / 64), 256) words
+// of selection masks (the warps' candidates first), then E offsets.  Callers place it in dynamic
+// shared memory that is free while the top-k runs.
+__host__ __device__ inline size_t topk_lists_smem(int E, int B) {
+    const size_t w = (size_t)E * ((B + 63) / 64);
+    return (w > 256 ? w : 256) * 8 + (size_t)E * 4;
+}
 
 // Warp maximum of the lanes' N packed words; the lane holding it clears it (words are unique
 // apart from 0, which only ever ties with another 0).  Returns the maximum to every lane.  Two
@@ -223,12 +230,14 @@ DEVI unsigned long long warp_take_best(unsigned long long (&w)[N]) {
 // published (the small-batch step adds the expert outputs into ylat).
 // acc64: when given, the logits are the fp64 sums there ([B][E]): they are rounded to fp32 into
 // ws.logits and the accumulator is cleared; otherwise ws.logits already holds them.
-// masks: shared memory for the bucket builder's token masks when B > 64 (E * ceil(B / 64) words);
-// up to 64 tokens the masks are one word per expert in TopkSmem.
+// lists: topk_lists_smem(E, B) bytes of shared memory (16-byte aligned) for the warps' candidates,
+// the bucket builder's token masks (ceil(B / 64) words per expert) and the experts' offsets.
 template <bool FUSED>
-DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u, unsigned long long *stamps = nullptr,
-                    float *zero_rows = nullptr, double *acc64 = nullptr, unsigned long long *masks = nullptr) {
+DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists, unsigned rt_done = 0u,
+                    unsigned long long *stamps = nullptr, float *zero_rows = nullptr, double *acc64 = nullptr) {
     const int E = a.d.E, K = a.d.k, B = a.B;
+    unsigned long long *masks = reinterpret_cast<unsigned long long *>(lists);
+    int *offs = reinterpret_cast<int *>(lists + topk_lists_smem(E, B) - (size_t)E * 4);
     if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_RT_DONE, rt_done, &t.ok)) return false;
     // optional trace (global ns): logits complete, keys, warp candidates, ranked, routing
     // written, expert masks, buckets written, buckets published
@@ -279,7 +288,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
 #pragma unroll
     for (int i = 0; i < 4; ++i)
         P[i] = valid[i] ? ((unsigned long long)key[i] << 32) | (0xffffffffu - (unsigned)(4 * tid + i)) : 0ull;
-    unsigned long long *cand = t.mask;  // nw * K candidates; the expert masks are built after
+    unsigned long long *cand = masks;  // nw * K candidates; the expert masks are built after
     for (int r = 0; r < K; ++r) {
         const unsigned long long m = warp_take_best(P);
         if (lane == 0) cand[warp * K + r] = m;
@@ -338,7 +347,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
     // selection is the number of lower tokens of its expert)
     if (!cta_ticket_last(a.ws.tickets + a.p.ticket_topk, (unsigned)B, &t.flag)) return true;
     const int W = (B + 63) / 64;
-    unsigned long long *mk = W == 1 ? t.mask : masks;  // [E][W]
+    unsigned long long *mk = masks;  // [E][W]
     auto sel_e = [&](int i) { return __ldcg(a.ws.idx + i); };
     for (int i = tid; i < E * W; i += blockDim.x) mk[i] = 0ull;
     __syncthreads();
@@ -366,7 +375,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int e = 4 * tid + i;
-        if (e < E) t.off[e] = off;
+        if (e < E) offs[e] = off;
         if (cnt[i] > 0) {
             a.ws.active_e[j] = e;
             a.ws.active_cnt[j] = cnt[i];
@@ -381,7 +390,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned rt_done = 0u
         const int ex = sel_e(i), tb = i / K;
         if (ex < 0 || ex >= E) continue;
         const unsigned long long *m = mk + ex * W;
-        int pos = t.off[ex] + __popcll(m[tb / 64] & ((1ull << (tb % 64)) - 1ull));
+        int pos = offs[ex] + __popcll(m[tb / 64] & ((1ull << (tb % 64)) - 1ull));
         for (int w = 0; w < tb / 64; ++w) pos += __popcll(m[w]);
         a.ws.entries[pos] = i;
     }
@@ -686,10 +695,10 @@ DEVI bool item_up(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
 // shared expert.  gate/up: 128 rows of I_s (gate, then up) x K range of H; down: 128 rows of H
 // x K range of I_s.  Tokens are staged as fp16 with a per-token exponent over the K range.
 
-template <bool FUSED, int NT>
+template <bool FUSED, int NT, int MAXB = kMaxBatch>
 DEVI void item_sgu(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag) {
-    __shared__ int s_shift[kMaxBatch];
-    __shared__ unsigned s_amax[kMaxBatch];
+    __shared__ int s_shift[MAXB];
+    __shared__ unsigned s_amax[MAXB];
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     const int H = a.d.H, Is = a.d.Is, B = a.B, maxB = a.d.max_batch;
     const int rb = bid / a.p.sgu.splits, ks = bid % a.p.sgu.splits;
@@ -756,10 +765,10 @@ DEVI void item_sgu(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_
     }
 }
 
-template <bool FUSED, int NT, bool SPLIT>
+template <bool FUSED, int NT, bool SPLIT, int MAXB = kMaxBatch>
 DEVI bool item_sd(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_flag, int *s_ok) {
-    __shared__ int s_shift[kMaxBatch];
-    __shared__ unsigned s_amax[kMaxBatch];
+    __shared__ int s_shift[MAXB];
+    __shared__ unsigned s_amax[MAXB];
     if (FUSED && !cta_wait_geq(a, a.ws.ctl + CTL_SGU_DONE, (unsigned)a.p.sgu.blocks, s_ok)) return false;
     uint16_t *xs = reinterpret_cast<uint16_t *>(smem);
     const int H = a.d.H, Is = a.d.Is, B = a.B, maxB = a.d.max_batch;

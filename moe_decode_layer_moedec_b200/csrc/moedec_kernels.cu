@@ -42,9 +42,9 @@ __global__ void __launch_bounds__(256) k_router_dn(StepArgs a) {
 
 // top-k: one CTA of 256 threads per token; the last one builds the expert buckets
 __global__ void __launch_bounds__(256) k_topk(StepArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];  // token masks of the bucket builder above 64 tokens
+    extern __shared__ __align__(16) unsigned char smem[];  // candidate and bucket lists
     __shared__ TopkSmem t;
-    item_topk<false>(a, blockIdx.x, t, 0u, nullptr, nullptr, nullptr, reinterpret_cast<unsigned long long *>(smem));
+    item_topk<false>(a, blockIdx.x, t, smem);
 }
 
 // routed experts: every warp takes a contiguous range of (expert, 16-row) warp items
@@ -136,8 +136,7 @@ cudaError_t launch_router_dn(const StepArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_topk(const StepArgs &a, cudaStream_t s) {
-    const size_t sm = a.B > 64 ? (size_t)a.d.E * ((a.B + 63) / 64) * 8 : 0;
-    k_topk<<<a.B, 256, sm, s>>>(a);
+    k_topk<<<a.B, 256, topk_lists_smem(a.d.E, a.B), s>>>(a);
     return cudaGetLastError();
 }
 
