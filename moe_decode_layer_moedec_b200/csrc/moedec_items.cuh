@@ -280,9 +280,9 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
     }
     stamp(1);
     // Selection on packed words (score bits << 32 | ~expert): a larger word ranks first (higher
-    // score, then lower expert index), 0 is no expert.  Each warp takes its K best, best first, by
-    // K rounds of a warp maximum whose holder drops the word; warp 0 then ranks the warps'
-    // candidates the same way and so emits the top K in rank order.
+    // score, then lower expert index), 0 is no expert.  Each warp takes its K best by K rounds of
+    // a warp maximum whose holder drops the word; the warps' candidates are then ranked by
+    // counting, which yields the top K in rank order.
     const int lane = tid & 31, warp = tid >> 5, nw = (int)(blockDim.x >> 5);
     unsigned long long P[4];
 #pragma unroll
@@ -295,23 +295,24 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
     }
     __syncthreads();
     stamp(2);
-    if (warp == 0) {
-        unsigned long long C[8];  // nw * K <= 8 * 32 candidates
-#pragma unroll
-        for (int i = 0; i < 8; ++i) C[i] = lane + 32 * i < nw * K ? cand[lane + 32 * i] : 0ull;
-        float S = 0.0f;  // sum of the selected scores in rank order
-        for (int r = 0; r < K; ++r) {
-            const unsigned long long m = warp_take_best(C);
-            if (lane == 0) {
-                const float sc = __uint_as_float((unsigned)(m >> 32));
-                t.rank_e[r] = (int)(0xffffffffu - (unsigned)(m & 0xffffffffull));
-                t.rank_s[r] = sc;
-                S += sc;
-            }
+    // The warps' candidates ranked at once: a candidate's rank is the number of larger candidates
+    // (the packed words are unique, 0 is none), so the K best land in rank order.  (Selecting
+    // them by K more rounds of a warp maximum costs K dependent shuffle chains.)
+    const int nc = nw * K;
+    for (int c = tid; c < nc; c += blockDim.x) {
+        const unsigned long long m = cand[c];
+        int rank = 0;
+        for (int j = 0; j < nc; ++j) rank += cand[j] > m ? 1 : 0;
+        if (rank < K && m != 0ull) {
+            t.rank_e[rank] = (int)(0xffffffffu - (unsigned)(m & 0xffffffffull));
+            t.rank_s[rank] = __uint_as_float((unsigned)(m >> 32));
         }
-        S = __shfl_sync(0xffffffffu, S, 0);
-        __syncwarp();
-        stamp(3);
+    }
+    __syncthreads();
+    stamp(3);
+    if (warp == 0) {
+        float S = 0.0f;  // sum of the selected scores in rank order
+        for (int r = 0; r < K; ++r) S += t.rank_s[r];
         if (lane < K) {
             a.ws.idx[(size_t)b * K + lane] = t.rank_e[lane];
             a.ws.wts[(size_t)b * K + lane] = t.rank_s[lane] / S;
