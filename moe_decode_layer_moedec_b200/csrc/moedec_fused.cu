@@ -32,7 +32,9 @@ enum Queue { Q_ROUTER = 0, Q_TOPK, Q_DN, Q_SGU, Q_EGU, Q_SD, Q_EDOWN, Q_UP, Q_CO
 // groups of that width.  Up to 64 tokens the kernel runs two CTAs per SM (128 registers per
 // thread: 16 warps per SM hide the latency of the MXFP4 decode and MMA chains that 8 warps at
 // 255 registers cannot), with 8-token expert groups and routing tables for 64 x 32 selections;
-// above 64 tokens one CTA per SM, 16-token expert groups and tables for 8192 selections.
+// above 64 tokens one CTA per SM, 16-token expert groups and tables for 8192 selections.  (Two CTAs
+// per SM above 64 tokens with the rings, which need no tables, ran B = 256 in 2,468 against
+// 1,970 us: the dense parts' 32-token groups cost more than the 16 ring warps per SM gained.)
 template <int TIER>
 struct Tier;
 template <> struct Tier<0> {

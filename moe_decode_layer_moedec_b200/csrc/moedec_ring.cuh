@@ -272,6 +272,9 @@ DEVI bool ring_rows(const StepArgs &a, const ExpertMaps &maps, int na, const Seg
     const uint32_t wring = smem_u32(ring) + (uint32_t)(warp * NSW * kRingBytes);
     const uint32_t xsa = smem_u32(xs);
     const int pitch_b = 2 * (K + kRingXPad);
+    uint32_t swo[8];  // this lane's offsets of word q of each 16-byte block chunk (128-byte swizzle)
+#pragma unroll
+    for (int b = 0; b < 8; ++b) swo[b] = (uint32_t)(g * 128 + ((b ^ g) << 4) + 4 * q);
     RingUnit *info = rs.unit[warp];
 
     // issue cursor (the same in every lane): group igi with its range end is1, unit iu, line il,
@@ -381,8 +384,8 @@ DEVI bool ring_rows(const StepArgs &a, const ExpertMaps &maps, int na, const Seg
                 uint32_t w0[8], w1[8];
 #pragma unroll
                 for (int b = 0; b < 8; ++b) {
-                    w0[b] = lds_u32(base + g * 128 + ((b ^ g) << 4) + 4 * q);
-                    w1[b] = lds_u32(base + 1024 + g * 128 + ((b ^ g) << 4) + 4 * q);
+                    w0[b] = lds_u32(base + swo[b]);
+                    w1[b] = lds_u32(base + 1024 + swo[b]);
                 }
                 ++pos;
                 __syncwarp();
