@@ -78,6 +78,10 @@ typedef enum moedec_status {
                                           in shared memory and stream its weights through registers,
                                           instead of the per-warp TMA weight rings (the default when
                                           latent/256 and expert_inter/256 are 1, 2, 4 or 8) */
+#define MOEDEC_FLAG_TEST_STALL_EXPERTS 128u /* tests only: the TMA-ring expert gate/up phase never
+                                          counts its units, so the expert down phase's wait for them
+                                          runs out after 20 ms and the step reports
+                                          MOEDEC_ERR_TIMEOUT (no GPU fault, no hang) */
 #define MOEDEC_TRACE_STAMPS 16         /* stamps per CTA */
 
 typedef struct moedec_config {

@@ -24,6 +24,7 @@ FLAG_MULTI_KERNEL = 8
 FLAG_TRACE = 16
 FLAG_STREAM = 32
 FLAG_NO_TMA_RING = 64
+FLAG_TEST_STALL_EXPERTS = 128
 TRACE_STAMPS = 16
 STATUS = {0: "MOEDEC_OK", -1: "MOEDEC_ERR_INVALID_ARG", -2: "MOEDEC_ERR_UNSUPPORTED", -3: "MOEDEC_ERR_CUDA",
           -4: "MOEDEC_ERR_OOM", -5: "MOEDEC_ERR_TIMEOUT", -6: "MOEDEC_ERR_DEVICE"}

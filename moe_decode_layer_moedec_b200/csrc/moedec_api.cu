@@ -314,7 +314,7 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     p.s_up = small_split(d.L, 32, kSmallSplitUp);
     stream_plan(d, p.st, p.ctl_tk + p.ctl_tk_words);
     p.ctl_words = p.st.words;
-    p.wait_limit_ns = (c.flags & MOEDEC_FLAG_TEST_STALL) ? 20000000LL : 1000000000LL;
+    p.wait_limit_ns = (c.flags & (MOEDEC_FLAG_TEST_STALL | MOEDEC_FLAG_TEST_STALL_EXPERTS)) ? 20000000LL : 1000000000LL;
 
     int rc = MOEDEC_OK;
     cudaError_t e = cudaGetDevice(&h->device);

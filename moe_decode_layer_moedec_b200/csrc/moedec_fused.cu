@@ -192,8 +192,9 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
         });
     }
     stamp(6);
-    // 5: shared down
-    cta_queue(Q_SD, n_sd, [&](int it) { return item_sd<true, T::NTS, T::SPLITS, T::MAXB>(a, it, smem, &s_flag, &s_ok); });
+    // 5: shared down (above 64 tokens after the expert down phase, see 7)
+    if constexpr (TIER != 4)
+        cta_queue(Q_SD, n_sd, [&](int it) { return item_sd<true, T::NTS, T::SPLITS, T::MAXB>(a, it, smem, &s_flag, &s_ok); });
     stamp(7);
     // 6: expert down: the same plan over L / 128 blocks per expert; each segment waits for its
     // expert's gate/up tiles
@@ -217,9 +218,15 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
         }
         alive = __syncthreads_and(ok ? 1 : 0) != 0;
     }
+    // 7: above 64 tokens the shared down comes after the expert down phase, where the CTAs that
+    // finish early take its items while the others complete their ranges (W_up needs all of ylat
+    // first, sh only in its last splits): B = 256 1,960 -> 1,907 us; at 16 and 64 tokens it
+    // measured neutral and 1 % slower
+    if constexpr (TIER == 4)
+        cta_queue(Q_SD, n_sd, [&](int it) { return item_sd<true, T::NTS, T::SPLITS, T::MAXB>(a, it, smem, &s_flag, &s_ok); });
     stamp(8);
     if (alive) prefetch_next_router(a, blockIdx.x, gridDim.x);
-    // 7: W_up and the output
+    // 8: W_up and the output
     cta_queue(Q_UP, n_up, [&](int it) { return item_up<true, T::NTU>(a, it, smem, &s_flag, &s_ok); });
     stamp(9);
     // leave; the last CTA out clears the control block for the next step

@@ -18,7 +18,8 @@
 
 namespace moedec {
 
-constexpr unsigned kFlagTestStall = 4u;  // MOEDEC_FLAG_TEST_STALL (see include/moedec.h)
+constexpr unsigned kFlagTestStall = 4u;           // MOEDEC_FLAG_TEST_STALL (see include/moedec.h)
+constexpr unsigned kFlagTestStallExperts = 128u;  // MOEDEC_FLAG_TEST_STALL_EXPERTS
 
 // ---------------------------------------------------------------------------------------------
 // device-side synchronisation of the fused step

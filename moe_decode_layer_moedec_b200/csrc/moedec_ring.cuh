@@ -422,7 +422,7 @@ DEVI bool ring_rows(const StepArgs &a, const ExpertMaps &maps, int na, const Seg
             else ring_rows_epi_down(a, rs, gr, t, acc, ntok, split);
             ++units_done;
         }
-        if (GU && units_done) warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, units_done);
+        if (GU && units_done && !(a.flags & kFlagTestStallExperts)) warp_signal_add(a.ws.ctl + a.p.ctl_gu + j, units_done);
     }
     if (!ok) {
         // copies still in flight must land before the ring's shared memory is used again

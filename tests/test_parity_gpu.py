@@ -303,6 +303,25 @@ def test_fused_wait_timeout_is_reported_and_context_stays_usable(tiny, schedule)
     _check_step(w, W, synth.tokens(w, batch=2), layer)
 
 
+@pytest.mark.parametrize("B", [2, 9, 65])
+def test_ring_wait_timeout_is_reported_and_context_stays_usable(tiny, B):
+    # MOEDEC_FLAG_TEST_STALL_EXPERTS: the TMA-ring gate/up phase never counts its units, so the
+    # expert down phase's bounded wait for them runs out (20 ms); every CTA drains its ring and
+    # leaves, and the step reports MOEDEC_ERR_TIMEOUT (B = 2: small-batch step, 9 and 65: split-K)
+    from moe_decode_layer_moedec_b200 import FLAG_TEST_STALL_EXPERTS, MoedecError
+    w, W, W_dev = tiny
+    stalled = _make_layer(w, W_dev, max_batch=B, flags=FLAG_TEST_STALL_EXPERTS)
+    assert stalled.tma_ring()
+    x = to_device(synth.tokens(w, batch=B))
+    for _ in range(2):  # the control block was cleared on the way out: it stalls again, no hang
+        stalled.step(x)
+        with pytest.raises(MoedecError, match="TIMEOUT"):
+            stalled.routing(B)
+    stalled.close()
+    layer = _make_layer(w, W_dev, max_batch=B)
+    _check_step(w, W, synth.tokens(w, batch=B), layer, label=f"tiny B{B} after a ring timeout")
+
+
 @pytest.mark.parametrize("batch,schedule", [(2, "stream"), (3, "fused"), (9, "fused")])
 def test_fused_and_multi_agree(tiny, batch, schedule):
     # batch 2 runs the streaming kernel, batch 3 the small-batch fused kernel, batch 9 the split-K one
