@@ -62,6 +62,9 @@ def parse():
     p.add_argument("--ncu", action="store_true",
                    help="profiling case for ncu: --steps eager steps over --layers resident layers, no timing")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU oracle sample length")
+    p.add_argument("--ep-emulate", type=int, default=0, metavar="G",
+                   help="time the expert-parallel step's ranks (G shards of every layer) one at a time on "
+                        "this GPU, and the exchange kernels; prints its own JSON line")
     return p.parse_args()
 
 
@@ -458,6 +461,76 @@ def fp4_stream():
     subprocess.check_call([exe])
 
 
+def ep_emulated(args, w, n_layers, local_rank):
+    """Each rank of a G-way expert-parallel split of the workload's layers, timed alone on this GPU
+    (graph replays of K partial steps over the resident layers, CUDA events, median of the reps),
+    and the exchange (publish + combine over G partials, with flags already set, so no waiting).
+    On a node of G GPUs the ranks run at once; the exchange there reads peer memory over NVLink,
+    which this one-GPU measurement does not include."""
+    import torch
+    from moe_decode_layer_moedec_b200 import FLAG_SKIP_SCALE_CHECK, LayerDims, ep
+    d, B, G = w.dims, w.batch, args.ep_emulate
+    dims = LayerDims(d.hidden, d.latent, d.n_experts, d.top_k, d.expert_inter, d.shared_inter, 1)
+    full, dev_weights = load_layers(w, n_layers, "fused", local_rank, 0)
+    for L_ in full:
+        L_.close()
+    groups = [ep.EmulatedExpertParallel(dims, Wd, G, max_batch=B, flags=FLAG_SKIP_SCALE_CHECK) for Wd in dev_weights]
+    x = torch.from_numpy(synth.tokens(w).view(np.int16)).to(f"cuda:{local_rank}")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for g in groups:
+            g.step(x, stream=stream)
+    torch.cuda.synchronize()
+    for g in groups:
+        check_device_errors(g.layers, B, stream)
+
+    def timed(fn):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream, capture_error_mode="thread_local"):
+            for i in range(args.steps):
+                fn(i)
+        for _ in range(max(args.warmup, 3)):
+            with torch.cuda.stream(stream):
+                gr.replay()
+        ts = []
+        for _ in range(args.reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            with torch.cuda.stream(stream):
+                gr.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        del gr
+        return 1e3 * statistics.median(ts) / args.steps
+
+    n = len(groups)
+    per_rank = []
+    for r in range(G):
+        per_rank.append(timed(lambda i, r=r: groups[i % n].layers[r].step_partial(x, groups[i % n].parts[r, 0],
+                                                                                   stream=stream)))
+    out = torch.empty((B, d.hidden), dtype=torch.int16, device=x.device)
+
+    def exchange(i):
+        g = groups[i % n]
+        e = g.clock.epoch  # already published by every rank: the combine does not wait
+        g.layers[0].ep_publish([g._flag_ptr(q, 0) for q in range(G)], e, stream=stream)
+        g.layers[0].ep_combine([g.parts[q, e % 2].data_ptr() for q in range(G)], g._flag_ptr(0, 0), e, B, out,
+                               stream=stream)
+    xch = timed(exchange)
+    for g in groups:
+        check_device_errors(g.layers, B, stream)
+        g.close()
+    line = {"metric": "ep_emulated", "workload": w.name, "world": G, "batch": B, "layers": n,
+            "steps": args.steps, "reps": args.reps,
+            "per_rank_partial_us": [round(v, 2) for v in per_rank],
+            "exchange_us": round(xch, 2), "slowest_rank_plus_exchange_us": round(max(per_rank) + xch, 2),
+            "note": "ranks timed one at a time on one GPU; the exchange reads local memory, so NVLink "
+                    "transfer time is not included"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.fp4_stream:
@@ -481,6 +554,10 @@ def main():
     n_layers = default_layers(w, args.layers)
     if args.ncu:
         return profile_case(args, w, n_layers, local_rank, rank)
+    if args.ep_emulate:
+        if world > 1:
+            raise SystemExit("--ep-emulate runs on one GPU")
+        return ep_emulated(args, w, n_layers, local_rank)
     peak, peak_src = measured_peak_hbm()
     layers, dev_weights = load_layers(w, n_layers, args.schedule, local_rank, rank)
     x_host = torch.from_numpy(synth.tokens(w).view(np.int16)).pin_memory()

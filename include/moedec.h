@@ -147,6 +147,82 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
  */
 MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint16_t *out, void *stream);
 
+/*
+ * Expert parallelism.  A layer can be split over G ranks (one GPU each): rank r creates a shard
+ * handle that holds the routed experts [expert_begin, expert_begin + expert_count) of the
+ * n_experts the router scores, and a slice of the shared expert's inner width.  Router, top-k and
+ * the H -> L projection run on every rank (identical routing everywhere); each rank runs only its
+ * own experts and its shared slice, and the layer's output is the bf16 rounding of the sum over
+ * ranks of their fp32 partial outputs
+ *   partial_r[b] = W_up ylat_r[b] + SD_r( silu(SG_r x[b]) * (SU_r x[b]) ),
+ * ylat_r summing the routed terms of rank r's experts only.  This follows from the step's
+ * definition above: both terms are linear in the experts and in the shared expert's inner index.
+ * The pages run this MoE tensor-parallel over the GPUs of one NVLink domain, with partial results
+ * in buffers that every GPU can reach and one fused reduction ("快是可以生成的，可信只能证明（vLLM
+ * 重写 Kimi K3 解码路径…）", section 他们换掉了什么); moedec_ep_publish / moedec_ep_combine are
+ * that exchange over peer memory.
+ *
+ * moedec_create_shard: like moedec_create, with cfg->n_experts the layer's total E and
+ *   expert_begin >= 0, expert_count >= 1, expert_begin + expert_count <= E.  The gate/up/down
+ *   code and scale arrays hold expert_count experts (the first is expert expert_begin), in the
+ *   layouts above with E replaced by expert_count.  cfg->shared_inter and the sh_* arrays describe
+ *   this rank's slice of the shared expert: rows [s0, s0 + I_s') of SG and SU, and columns
+ *   [s0, s0 + I_s') of SD stored as their own dense [H][I_s'/2] and [H][I_s'/32] arrays (I_s' a
+ *   multiple of 128, or n_shared = 0 on a rank without a slice).  MOEDEC_FLAG_STREAM is not
+ *   supported for shards (UNSUPPORTED).  Errors as moedec_create, plus INVALID_ARG for the range.
+ * moedec_step_partial: one step of a shard (or of a whole layer) that writes
+ *   partial fp32 [batch][H], device, 16-byte aligned, must not overlap x,
+ *   with W_up ylat + sh before any rounding, instead of the bf16 output.  Errors as moedec_step.
+ */
+MOEDEC_API int moedec_create_shard(const moedec_config *cfg, const moedec_weights *w, int32_t expert_begin,
+                                   int32_t expert_count, moedec_handle **out);
+MOEDEC_API int moedec_step_partial(moedec_handle *h, const uint16_t *x, int batch, float *partial, void *stream);
+
+#define MOEDEC_EP_MAX_WORLD 16
+#define MOEDEC_IPC_HANDLE_BYTES 64
+
+/*
+ * The exchange of an expert-parallel step, on rank r of `world` (1..MOEDEC_EP_MAX_WORLD).  Every
+ * rank owns a flag array uint32 [world] (zeroed once, never reset) and two partial buffers fp32
+ * [max_batch][H] used alternately by step parity; the ranks exchange their addresses once (peer
+ * pointers: moedec_ipc_export / moedec_ipc_open).  Step e (e = 1, 2, ...) on rank r is, on one
+ * stream:
+ *   moedec_step_partial(h, x, B, part_r[e % 2], s);
+ *   moedec_ep_publish(h, slots, world, e, s);   slots[q] = &flags_q[r] (host array of device pointers)
+ *   moedec_ep_combine(h, parts, flags_r, world, e, B, out, s);   parts[g] = part_g[e % 2]
+ * moedec_ep_publish launches one thread that makes all prior work of the stream visible at system
+ *   scope and release-stores e into each slot.
+ * moedec_ep_combine launches a kernel whose blocks wait until flags[g] >= e for every g (acquire,
+ *   system scope; bounded like the step's waits, a timeout is reported as MOEDEC_ERR_TIMEOUT by the
+ *   next synchronising call of h and leaves out unwritten), then write
+ *   out[b][j] = bf16(((parts[0][b][j] + parts[1][b][j]) + ...) + parts[world-1][b][j]) (fp32 sums in
+ *   rank order, one round-to-nearest-even), so every rank gets the same bits.  flags may be NULL:
+ *   no wait (the caller orders the partials itself, e.g. world = 1 after a library all-reduce).
+ *   parts: host array of `world` device pointers, 16-byte aligned; out: bf16 [batch][H], device,
+ *   16-byte aligned.
+ * The two-buffer rotation is what makes reuse safe: rank r overwrites part_r[p] in step e + 2 only
+ * after its combine of step e + 1, which waited for every rank's publish of e + 1, issued after
+ * that rank's combine of step e had read part_r[p].
+ * Errors: INVALID_ARG (NULL, misaligned, world out of range, batch < 0), UNSUPPORTED (batch >
+ * max_batch), CUDA (launch).
+ */
+MOEDEC_API int moedec_ep_publish(moedec_handle *h, uint32_t *const *slots, int world, uint32_t epoch, void *stream);
+MOEDEC_API int moedec_ep_combine(moedec_handle *h, const float *const *parts, const uint32_t *flags, int world,
+                                 uint32_t epoch, int batch, uint16_t *out, void *stream);
+
+/*
+ * CUDA IPC of device memory, for handing a rank's flag array and partial buffers to the other
+ * processes of its node.  moedec_ipc_export writes MOEDEC_IPC_HANDLE_BYTES bytes into the host
+ * buffer `handle` for the whole device allocation that contains `ptr`, and the byte offset of ptr
+ * inside it into the host word *offset; moedec_ipc_open maps such a handle exported by another
+ * process into this one (peer access enabled lazily) and returns the allocation's base, to which
+ * the importer adds the offset; moedec_ipc_close unmaps that base.  A process cannot open its own
+ * handles.  Errors: INVALID_ARG (NULL), CUDA.
+ */
+MOEDEC_API int moedec_ipc_export(const void *ptr, void *handle, uint64_t *offset);
+MOEDEC_API int moedec_ipc_open(const void *handle, void **ptr);
+MOEDEC_API int moedec_ipc_close(void *ptr);
+
 /* Release the workspace, side stream and events (synchronises the side stream). NULL is a no-op. */
 MOEDEC_API int moedec_destroy(moedec_handle *h);
 

@@ -26,6 +26,8 @@ FLAG_STREAM = 32
 FLAG_NO_TMA_RING = 64
 FLAG_TEST_STALL_EXPERTS = 128
 TRACE_STAMPS = 16
+EP_MAX_WORLD = 16
+IPC_HANDLE_BYTES = 64
 STATUS = {0: "MOEDEC_OK", -1: "MOEDEC_ERR_INVALID_ARG", -2: "MOEDEC_ERR_UNSUPPORTED", -3: "MOEDEC_ERR_CUDA",
           -4: "MOEDEC_ERR_OOM", -5: "MOEDEC_ERR_TIMEOUT", -6: "MOEDEC_ERR_DEVICE"}
 WEIGHT_NAMES = ("router", "w_down_lat", "w_up_lat", "gate_q", "gate_s", "up_q", "up_s", "down_q", "down_s",
@@ -89,6 +91,20 @@ def _load():
     lib.moedec_kernels_per_step.restype = i32
     lib.moedec_last_cuda_error.argtypes = [vp]
     lib.moedec_last_cuda_error.restype = ctypes.c_char_p
+    lib.moedec_create_shard.argtypes = [ctypes.POINTER(_Config), ctypes.POINTER(_Weights), i32, i32, ctypes.POINTER(vp)]
+    lib.moedec_create_shard.restype = i32
+    lib.moedec_step_partial.argtypes = [vp, vp, i32, vp, vp]
+    lib.moedec_step_partial.restype = i32
+    lib.moedec_ep_publish.argtypes = [vp, ctypes.POINTER(vp), i32, ctypes.c_uint32, vp]
+    lib.moedec_ep_publish.restype = i32
+    lib.moedec_ep_combine.argtypes = [vp, ctypes.POINTER(vp), vp, i32, ctypes.c_uint32, i32, vp, vp]
+    lib.moedec_ep_combine.restype = i32
+    lib.moedec_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint64)]
+    lib.moedec_ipc_export.restype = i32
+    lib.moedec_ipc_open.argtypes = [vp, ctypes.POINTER(vp)]
+    lib.moedec_ipc_open.restype = i32
+    lib.moedec_ipc_close.argtypes = [vp]
+    lib.moedec_ipc_close.restype = i32
     lib.moedec_status_string.argtypes = [i32]
     lib.moedec_status_string.restype = ctypes.c_char_p
     return lib
@@ -125,12 +141,18 @@ class MoeDecodeLayer:
     `weights` maps the names in WEIGHT_NAMES to contiguous CUDA tensors: bf16 matrices as
     torch.bfloat16 or torch.uint16/int16 bit patterns, MXFP4 codes and E8M0 scales as uint8.
     The tensors are borrowed: keep them alive and unchanged while the layer exists.
+
+    With `expert_range=(begin, count)` the handle is one shard of an expert-parallel layer
+    (moedec_create_shard): `dims.n_experts` is the layer's total, the expert arrays hold experts
+    begin .. begin+count-1 only, and `dims.shared_inter` / the sh_* arrays are this shard's slice
+    of the shared expert.  Such a shard gives its fp32 partial output with `step_partial`.
     """
 
-    def __init__(self, dims: LayerDims, weights: dict, max_batch: int, flags: int = 0):
+    def __init__(self, dims: LayerDims, weights: dict, max_batch: int, flags: int = 0, expert_range=None):
         self.dims = dims
         self.max_batch = max_batch
         self.flags = flags
+        self.expert_range = None if expert_range is None else (int(expert_range[0]), int(expert_range[1]))
         self._weights = {n: weights.get(n) for n in WEIGHT_NAMES}  # keep the tensors alive
         for n, t in self._weights.items():
             if t is not None and not t.is_contiguous():
@@ -139,9 +161,13 @@ class MoeDecodeLayer:
                       dims.shared_inter, dims.n_shared, max_batch, flags)
         w = _Weights(*[_ptr(self._weights[n]) for n in WEIGHT_NAMES])
         h = ctypes.c_void_p()
-        rc = lib.moedec_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))
+        if self.expert_range is None:
+            rc = lib.moedec_create(ctypes.byref(cfg), ctypes.byref(w), ctypes.byref(h))
+        else:
+            rc = lib.moedec_create_shard(ctypes.byref(cfg), ctypes.byref(w), self.expert_range[0],
+                                         self.expert_range[1], ctypes.byref(h))
         if rc != 0:
-            raise MoedecError("moedec_create", rc)
+            raise MoedecError("moedec_create" if self.expert_range is None else "moedec_create_shard", rc)
         self._h = h
 
     def _check(self, call: str, rc: int):
@@ -157,6 +183,35 @@ class MoeDecodeLayer:
             out = torch.empty((B, self.dims.hidden), dtype=x.dtype, device=x.device)
         assert x.is_contiguous() and out.is_contiguous()
         self._check("moedec_step", lib.moedec_step(self._h, _ptr(x), B, _ptr(out), _stream_ptr(stream)))
+        return out
+
+    def step_partial(self, x, partial=None, stream=None):
+        """partial[b] = W_up ylat[b] + sh[b] in fp32, before rounding (this handle's experts and
+        shared slice only when it is a shard); asynchronous on `stream`."""
+        import torch
+        B = x.shape[0]
+        if partial is None:
+            partial = torch.empty((B, self.dims.hidden), dtype=torch.float32, device=x.device)
+        assert x.is_contiguous() and partial.is_contiguous() and partial.dtype == torch.float32
+        assert partial.numel() >= B * self.dims.hidden
+        self._check("moedec_step_partial",
+                    lib.moedec_step_partial(self._h, _ptr(x), B, _ptr(partial), _stream_ptr(stream)))
+        return partial
+
+    def ep_publish(self, slot_ptrs, epoch: int, stream=None):
+        """Release-store `epoch` into each device address of `slot_ptrs` (this rank's flag word in
+        every rank's flag array) after the work already on `stream`."""
+        arr = (ctypes.c_void_p * len(slot_ptrs))(*[int(p) for p in slot_ptrs])
+        self._check("moedec_ep_publish",
+                    lib.moedec_ep_publish(self._h, arr, len(slot_ptrs), epoch & 0xffffffff, _stream_ptr(stream)))
+
+    def ep_combine(self, part_ptrs, flags_ptr: int, epoch: int, batch: int, out, stream=None):
+        """out = bf16(sum of the ranks' fp32 partials, rank order) once every flag word at
+        `flags_ptr` (one per rank; 0 for no wait) has reached `epoch`."""
+        arr = (ctypes.c_void_p * len(part_ptrs))(*[int(p) for p in part_ptrs])
+        self._check("moedec_ep_combine",
+                    lib.moedec_ep_combine(self._h, arr, int(flags_ptr) or None, len(part_ptrs), epoch & 0xffffffff,
+                                          batch, _ptr(out), _stream_ptr(stream)))
         return out
 
     def step_ptr(self, x_ptr: int, batch: int, out_ptr: int, stream_ptr: int):
@@ -274,3 +329,33 @@ def router_logits_noalloc(router, x, logits=None, stream=None):
     if rc != 0:
         raise MoedecError("moedec_router_logits_noalloc", rc)
     return logits
+
+
+def ipc_export(ptr: int) -> tuple[bytes, int]:
+    """CUDA IPC handle (IPC_HANDLE_BYTES bytes) of the device allocation that contains `ptr`, and
+    the offset of `ptr` inside it."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    off = ctypes.c_uint64()
+    rc = lib.moedec_ipc_export(int(ptr), buf, ctypes.byref(off))
+    if rc != 0:
+        raise MoedecError("moedec_ipc_export", rc)
+    return buf.raw, int(off.value)
+
+
+def ipc_open(handle: bytes) -> int:
+    """Map an allocation exported by another process; returns its base address here (add the
+    exporter's offset)."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("IPC handle must be %d bytes" % IPC_HANDLE_BYTES)
+    buf = ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES)
+    p = ctypes.c_void_p()
+    rc = lib.moedec_ipc_open(buf, ctypes.byref(p))
+    if rc != 0:
+        raise MoedecError("moedec_ipc_open", rc)
+    return int(p.value)
+
+
+def ipc_close(ptr: int) -> None:
+    rc = lib.moedec_ipc_close(int(ptr))
+    if rc != 0:
+        raise MoedecError("moedec_ipc_close", rc)

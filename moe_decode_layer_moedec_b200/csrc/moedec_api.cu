@@ -98,9 +98,9 @@ void make_expert_maps(moedec_handle *h) {
         return;
     }
     const TensorMapEncodeFn enc = reinterpret_cast<TensorMapEncodeFn>(fn);
-    const bool ok = encode_rows(enc, &m.gate, h->w.gate_q, (uint64_t)d.L / 2, (uint64_t)d.E * d.I) &&
-                    encode_rows(enc, &m.up, h->w.up_q, (uint64_t)d.L / 2, (uint64_t)d.E * d.I) &&
-                    encode_rows(enc, &m.down, h->w.down_q, (uint64_t)d.I / 2, (uint64_t)d.E * d.L);
+    const bool ok = encode_rows(enc, &m.gate, h->w.gate_q, (uint64_t)d.L / 2, (uint64_t)d.ne * d.I) &&
+                    encode_rows(enc, &m.up, h->w.up_q, (uint64_t)d.L / 2, (uint64_t)d.ne * d.I) &&
+                    encode_rows(enc, &m.down, h->w.down_q, (uint64_t)d.I / 2, (uint64_t)d.ne * d.L);
     m.ok = ok ? 1 : 0;
 }
 
@@ -174,8 +174,8 @@ int check_scales(moedec_handle *h) {
         const uint8_t *p;
         size_t n;
     } arrs[] = {
-        {h->w.gate_s, (size_t)d.E * d.I * (d.L / 32)}, {h->w.up_s, (size_t)d.E * d.I * (d.L / 32)},
-        {h->w.down_s, (size_t)d.E * d.L * (d.I / 32)}, {h->w.sh_gate_s, d.n_shared ? (size_t)d.Is * (d.H / 32) : 0},
+        {h->w.gate_s, (size_t)d.ne * d.I * (d.L / 32)}, {h->w.up_s, (size_t)d.ne * d.I * (d.L / 32)},
+        {h->w.down_s, (size_t)d.ne * d.L * (d.I / 32)}, {h->w.sh_gate_s, d.n_shared ? (size_t)d.Is * (d.H / 32) : 0},
         {h->w.sh_up_s, d.n_shared ? (size_t)d.Is * (d.H / 32) : 0}, {h->w.sh_down_s, d.n_shared ? (size_t)d.H * (d.Is / 32) : 0},
     };
     unsigned host_bad = 0;
@@ -258,11 +258,17 @@ MOEDEC_API const char *moedec_status_string(int status) {
 
 MOEDEC_API const char *moedec_last_cuda_error(moedec_handle *h) { return h ? h->cuda_error : ""; }
 
-MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, moedec_handle **out) {
+}  // extern "C"
+
+namespace {
+
+int create_handle(const moedec_config *cfg, const moedec_weights *w, int e0, int ne, moedec_handle **out) {
     if (!out) return MOEDEC_ERR_INVALID_ARG;
     *out = nullptr;
     if (!cfg || !w || cfg->abi_version != MOEDEC_ABI_VERSION) return MOEDEC_ERR_INVALID_ARG;
     const moedec_config &c = *cfg;
+    if (e0 < 0 || ne < 1 || e0 + ne > c.n_experts) return MOEDEC_ERR_INVALID_ARG;
+    if (ne != c.n_experts && (c.flags & MOEDEC_FLAG_STREAM)) return MOEDEC_ERR_UNSUPPORTED;
     if (c.hidden <= 0 || c.latent <= 0 || c.n_experts <= 0 || c.top_k <= 0 || c.expert_inter <= 0 || c.max_batch <= 0 ||
         (c.n_shared != 0 && c.n_shared != 1) || (c.n_shared && c.shared_inter <= 0))
         return MOEDEC_ERR_INVALID_ARG;
@@ -282,7 +288,7 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     if (!h) return MOEDEC_ERR_OOM;
     h->cfg = c;
     h->d = Dims{c.hidden, c.latent, c.n_experts, c.top_k, c.expert_inter, c.n_shared ? c.shared_inter : 128,
-                c.n_shared, c.max_batch};
+                c.n_shared, c.max_batch, e0, ne};
     h->w = Weights{w->router, w->w_down_lat, w->w_up_lat, w->gate_q, w->gate_s, w->up_q, w->up_s, w->down_q, w->down_s,
                    w->sh_gate_q, w->sh_gate_s, w->sh_up_q, w->sh_up_s, w->sh_down_q, w->sh_down_s};
     const Dims &d = h->d;
@@ -346,6 +352,19 @@ MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, 
     return MOEDEC_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+MOEDEC_API int moedec_create(const moedec_config *cfg, const moedec_weights *w, moedec_handle **out) {
+    return create_handle(cfg, w, 0, cfg ? cfg->n_experts : 0, out);
+}
+
+MOEDEC_API int moedec_create_shard(const moedec_config *cfg, const moedec_weights *w, int32_t expert_begin,
+                                   int32_t expert_count, moedec_handle **out) {
+    return create_handle(cfg, w, expert_begin, expert_count, out);
+}
+
 MOEDEC_API int moedec_destroy(moedec_handle *h) {
     if (!h) return MOEDEC_OK;
     if (h->side) cudaStreamSynchronize(h->side);
@@ -363,14 +382,20 @@ MOEDEC_API int moedec_destroy(moedec_handle *h) {
     return MOEDEC_OK;
 }
 
-MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint16_t *out, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// One step into bf16 out (out_f32 == nullptr) or into the fp32 partial out_f32 (out == nullptr).
+int step_impl(moedec_handle *h, const uint16_t *x, int batch, uint16_t *out, float *out_f32, void *stream) {
     if (!h || batch < 0) return MOEDEC_ERR_INVALID_ARG;
     if (batch > h->d.max_batch) return MOEDEC_ERR_UNSUPPORTED;
     if (batch == 0) return MOEDEC_OK;
-    if (!x || !out || !aligned16(x) || !aligned16(out)) return MOEDEC_ERR_INVALID_ARG;
-    const size_t bytes = (size_t)batch * h->d.H * 2;
-    const char *xb = reinterpret_cast<const char *>(x), *ob = reinterpret_cast<const char *>(out);
-    if (xb < ob + bytes && ob < xb + bytes) return MOEDEC_ERR_INVALID_ARG;
+    void *dst = out ? static_cast<void *>(out) : static_cast<void *>(out_f32);
+    if (!x || !dst || !aligned16(x) || !aligned16(dst)) return MOEDEC_ERR_INVALID_ARG;
+    const size_t xbytes = (size_t)batch * h->d.H * 2, obytes = (size_t)batch * h->d.H * (out ? 2 : 4);
+    const char *xb = reinterpret_cast<const char *>(x), *ob = reinterpret_cast<const char *>(dst);
+    if (xb < ob + obytes && ob < xb + xbytes) return MOEDEC_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     StepArgs a;
     a.d = h->d;
@@ -380,19 +405,22 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     a.next_router = h->next_router;
     a.x = x;
     a.out = out;
+    a.out_f32 = out_f32;
     a.B = batch;
     a.flags = h->cfg.flags;
     cudaError_t e = cudaSuccess;
     const int variant = batch <= 4 ? 0 : 1;
     if (!(h->cfg.flags & MOEDEC_FLAG_MULTI_KERNEL)) {
-        if ((h->cfg.flags & MOEDEC_FLAG_STREAM) && stream_supports(h->d, batch))
+        // the streaming schedule writes bf16 only: a partial step takes the small-batch kernel
+        const bool stream_sched = (h->cfg.flags & MOEDEC_FLAG_STREAM) && !out_f32 && stream_supports(h->d, batch);
+        if (stream_sched)
             e = timed(h, K_FUSED_STREAM, s, [&] { return launch_stream(a, s, h->n_sm); });
         else if (fused_small_supports(h->d, batch))
             e = timed(h, K_FUSED_SMALL, s, [&] { return launch_fused_small(a, h->maps, s, h->n_sm); });
         else
             e = timed(h, K_FUSED, s, [&] { return launch_fused(a, h->maps, s, h->n_sm); });
         if (e != cudaSuccess) return record_cuda(h, e);
-        h->launches[variant] += (uint64_t)moedec_kernels_per_step(h, batch);
+        h->launches[variant] += stream_sched ? (uint64_t)kStreamLaunches : 1u;
         h->last_batch = batch;
         return MOEDEC_OK;
     }
@@ -414,6 +442,90 @@ MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint1
     h->launches[variant] += (uint64_t)kernels_per_step(h->d);
     h->last_batch = batch;
     return MOEDEC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+MOEDEC_API int moedec_step(moedec_handle *h, const uint16_t *x, int batch, uint16_t *out, void *stream) {
+    return step_impl(h, x, batch, out, nullptr, stream);
+}
+
+MOEDEC_API int moedec_step_partial(moedec_handle *h, const uint16_t *x, int batch, float *partial, void *stream) {
+    return step_impl(h, x, batch, nullptr, partial, stream);
+}
+
+MOEDEC_API int moedec_ep_publish(moedec_handle *h, uint32_t *const *slots, int world, uint32_t epoch, void *stream) {
+    if (!h || !slots || world < 1 || world > kEpMaxWorld) return MOEDEC_ERR_INVALID_ARG;
+    EpSlots sl{};
+    for (int g = 0; g < world; ++g) {
+        if (!slots[g] || reinterpret_cast<uintptr_t>(slots[g]) % 4) return MOEDEC_ERR_INVALID_ARG;
+        sl.p[g] = slots[g];
+    }
+    const cudaError_t e = launch_ep_publish(sl, world, epoch, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOEDEC_OK : record_cuda(h, e);
+}
+
+MOEDEC_API int moedec_ep_combine(moedec_handle *h, const float *const *parts, const uint32_t *flags, int world,
+                                 uint32_t epoch, int batch, uint16_t *out, void *stream) {
+    if (!h || !parts || world < 1 || world > kEpMaxWorld || batch < 0) return MOEDEC_ERR_INVALID_ARG;
+    if (batch > h->d.max_batch) return MOEDEC_ERR_UNSUPPORTED;
+    if (batch == 0) return MOEDEC_OK;
+    if (!out || !aligned16(out) || (flags && reinterpret_cast<uintptr_t>(flags) % 4)) return MOEDEC_ERR_INVALID_ARG;
+    EpParts pp{};
+    for (int g = 0; g < world; ++g) {
+        if (!parts[g] || !aligned16(parts[g])) return MOEDEC_ERR_INVALID_ARG;
+        pp.p[g] = parts[g];
+    }
+    const cudaError_t e = launch_ep_combine(pp, flags, world, epoch, (size_t)batch * h->d.H, out, h->ws.err,
+                                            h->p.wait_limit_ns, h->n_sm, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MOEDEC_OK : record_cuda(h, e);
+}
+
+MOEDEC_API int moedec_ipc_export(const void *ptr, void *handle, uint64_t *offset) {
+    if (!ptr || !handle || !offset) return MOEDEC_ERR_INVALID_ARG;
+    // the handle names the whole allocation that contains ptr (an allocator may hand out pieces
+    // of a larger one), so the offset of ptr inside it travels with the handle
+    typedef CUresult (*AddressRangeFn)(CUdeviceptr *, size_t *, CUdeviceptr);
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+        cudaGetLastError();
+        return MOEDEC_ERR_CUDA;
+    }
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (reinterpret_cast<AddressRangeFn>(fn)(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+        return MOEDEC_ERR_CUDA;
+    cudaIpcMemHandle_t m;
+    if (cudaIpcGetMemHandle(&m, reinterpret_cast<void *>(base)) != cudaSuccess) {
+        cudaGetLastError();
+        return MOEDEC_ERR_CUDA;
+    }
+    static_assert(sizeof(m) == MOEDEC_IPC_HANDLE_BYTES, "IPC handle size");
+    memcpy(handle, &m, sizeof(m));
+    *offset = (uint64_t)(reinterpret_cast<CUdeviceptr>(ptr) - base);
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_ipc_open(const void *handle, void **ptr) {
+    if (!handle || !ptr) return MOEDEC_ERR_INVALID_ARG;
+    *ptr = nullptr;
+    cudaIpcMemHandle_t m;
+    memcpy(&m, handle, sizeof(m));
+    if (cudaIpcOpenMemHandle(ptr, m, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) {
+        cudaGetLastError();
+        *ptr = nullptr;
+        return MOEDEC_ERR_CUDA;
+    }
+    return MOEDEC_OK;
+}
+
+MOEDEC_API int moedec_ipc_close(void *ptr) {
+    if (!ptr) return MOEDEC_ERR_INVALID_ARG;
+    return cudaIpcCloseMemHandle(ptr) == cudaSuccess ? MOEDEC_OK : MOEDEC_ERR_CUDA;
 }
 
 MOEDEC_API int moedec_set_next(moedec_handle *h, const moedec_handle *next) {

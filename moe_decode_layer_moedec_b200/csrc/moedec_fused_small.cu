@@ -504,7 +504,8 @@ DEVI bool w_up(const StepArgs &a, int item, const uint16_t *ys) {
         for (int h2 = 0; h2 < 2; ++h2) {
             const int r = row0 + g + 8 * h2;
             if (a.ws.up_tap) a.ws.up_tap[(size_t)q * H + r] = sv[h2];
-            a.out[(size_t)q * H + r] = f32_to_bf16_rne(sv[h2] + shv[h2]);
+            if (a.out_f32) a.out_f32[(size_t)q * H + r] = sv[h2] + shv[h2];
+            else a.out[(size_t)q * H + r] = f32_to_bf16_rne(sv[h2] + shv[h2]);
         }
     }
     return true;

@@ -29,8 +29,11 @@ constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmall
 constexpr int kSmallMaxBatch = 4;  // tokens of the small-batch step
 constexpr int kTraceStamps = 16;     // MOEDEC_TRACE_STAMPS
 
+// e0, ne: the experts whose weights this handle holds, [e0, e0 + ne) of the E the router scores
+// (all of them, e0 = 0 and ne = E, unless the handle is one shard of an expert-parallel layer);
+// the expert weight arrays are indexed by e - e0.
 struct Dims {
-    int H, L, E, k, I, Is, n_shared, max_batch;
+    int H, L, E, k, I, Is, n_shared, max_batch, e0, ne;
 };
 
 struct Weights {
@@ -140,6 +143,7 @@ struct StepArgs {
     Plan p;
     const uint16_t *x;  // [B][H]
     uint16_t *out;      // [B][H]
+    float *out_f32;     // [B][H] fp32 W_up ylat + sh before rounding (partial step of a shard), or nullptr
     int B;
     unsigned flags;     // MOEDEC_FLAG_* of the handle
 };
@@ -185,6 +189,17 @@ bool fused_small_supports(const Dims &d, int B);
 cudaError_t launch_fused_small(const StepArgs &a, const ExpertMaps &maps, cudaStream_t s, int n_sm);
 cudaError_t init_fused_small_attributes();
 int kernels_per_step(const Dims &d);
+// exchange step of an expert-parallel layer (moedec_ep.cu)
+constexpr int kEpMaxWorld = 16;
+struct EpSlots {
+    unsigned *p[kEpMaxWorld];  // this rank's flag word in each rank's flag array (peer pointers)
+};
+struct EpParts {
+    const float *p[kEpMaxWorld];  // each rank's fp32 partial output [B][H] (peer pointers)
+};
+cudaError_t launch_ep_publish(const EpSlots &slots, int world, unsigned epoch, cudaStream_t s);
+cudaError_t launch_ep_combine(const EpParts &parts, const unsigned *flags, int world, unsigned epoch, size_t n,
+                              uint16_t *out, unsigned *err, long long wait_ns, int n_sm, cudaStream_t s);
 cudaError_t init_kernel_attributes();
 
 }  // namespace moedec

@@ -324,20 +324,29 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
             reinterpret_cast<float4 *>(zero_rows + (size_t)b * a.d.L)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
     stamp(4);
+    // A shard of an expert-parallel layer keeps only the selections of its own experts
+    // [e0, e0 + ne) (bucketed by local index e - e0); the W_up items still wait for B K counts per
+    // ylat block, so the selections of other shards' experts are counted here at once.
+    const int e0 = a.d.e0, e1 = a.d.e0 + a.d.ne;
     if (B == 1) {
         // one token: its K distinct experts are the buckets (one entry each), in expert order
         if (warp == 0) {
-            const int e = lane < K ? t.rank_e[lane] : 0x7fffffff;
+            const int er = lane < K ? t.rank_e[lane] : -1;
+            const bool local = er >= e0 && er < e1;
+            const int e = local ? er : 0x7fffffff;
             int pos = 0;
             for (int j = 0; j < K; ++j) pos += __shfl_sync(0xffffffffu, e, j) < e ? 1 : 0;
-            if (lane < K) {
-                a.ws.active_e[pos] = e;
+            const int n_local = __popc(__ballot_sync(0xffffffffu, local));
+            if (local) {
+                a.ws.active_e[pos] = e - e0;
                 a.ws.active_cnt[pos] = 1;
                 a.ws.active_off[pos] = pos;
                 a.ws.entries[pos] = lane;
-                a.ws.a_amax[lane] = 0u;
             }
-            if (lane == 0) *a.ws.n_active = K;
+            if (lane < K) a.ws.a_amax[lane] = 0u;
+            if (lane == 0) *a.ws.n_active = n_local;
+            if (FUSED && n_local < K)
+                for (int i = lane; i < a.d.L / 16; i += 32) atomicAdd(a.ws.ctl + a.p.ctl_ylat + i, (unsigned)(K - n_local));
         }
         stamp(6);
         if (FUSED) cta_signal_add(a.ws.ctl + CTL_ROUTE_READY, 1u);
@@ -355,8 +364,8 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
     __syncthreads();
     for (int i = tid; i < B * K; i += blockDim.x) {
         const int ex = sel_e(i), tb = i / K;
-        if (ex >= 0 && ex < E) atomicOr(&mk[ex * W + tb / 64], 1ull << (tb % 64));
-        else atomicOr(a.ws.err, kErrBucket);
+        if (ex < 0 || ex >= E) atomicOr(a.ws.err, kErrBucket);
+        else if (ex >= e0 && ex < e1) atomicOr(&mk[ex * W + tb / 64], 1ull << (tb % 64));
         a.ws.a_amax[i] = 0u;
     }
     __syncthreads();
@@ -379,7 +388,7 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
         const int e = 4 * tid + i;
         if (e < E) offs[e] = off;
         if (cnt[i] > 0) {
-            a.ws.active_e[j] = e;
+            a.ws.active_e[j] = e - e0;
             a.ws.active_cnt[j] = cnt[i];
             a.ws.active_off[j] = off;
             ++j;
@@ -387,10 +396,12 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
         off += cnt[i];
     }
     if (tid == 0) *a.ws.n_active = n_act;
+    if (FUSED && n_ent < B * K)
+        for (int i = tid; i < a.d.L / 16; i += blockDim.x) atomicAdd(a.ws.ctl + a.p.ctl_ylat + i, (unsigned)(B * K - n_ent));
     __syncthreads();
     for (int i = tid; i < B * K; i += blockDim.x) {
         const int ex = sel_e(i), tb = i / K;
-        if (ex < 0 || ex >= E) continue;
+        if (ex < e0 || ex >= e1) continue;
         const unsigned long long *m = mk + ex * W;
         int pos = offs[ex] + __popcll(m[tb / 64] & ((1ull << (tb % 64)) - 1ull));
         for (int w = 0; w < tb / 64; ++w) pos += __popcll(m[w]);
@@ -402,15 +413,19 @@ DEVI bool item_topk(const StepArgs &a, int b, TopkSmem &t, unsigned char *lists,
     return true;
 }
 
-// ylat[b][l] = sum_r w[b][r] y[b*K + r][l] in slot order (all loads issued before the sum)
+// ylat[b][l] = sum_r w[b][r] y[b*K + r][l] in slot order (all loads issued before the sum); a
+// shard of an expert-parallel layer sums the slots of its own experts only
 DEVI float combine_value(const StepArgs &a, int b, int l) {
     const int L = a.d.L, K = a.d.k;
+    const bool all = a.d.ne == a.d.E;
     float wv[kMaxTopK], yv[kMaxTopK];
 #pragma unroll
     for (int r = 0; r < kMaxTopK; ++r)
         if (r < K) {
-            wv[r] = __ldcg(a.ws.wts + (size_t)b * K + r);
-            yv[r] = __ldcg(a.ws.y + ((size_t)b * K + r) * L + l);
+            const int e = all ? 0 : __ldcg(a.ws.idx + (size_t)b * K + r) - a.d.e0;
+            const bool local = all || (e >= 0 && e < a.d.ne);
+            wv[r] = local ? __ldcg(a.ws.wts + (size_t)b * K + r) : 0.0f;
+            yv[r] = local ? __ldcg(a.ws.y + ((size_t)b * K + r) * L + l) : 0.0f;
         }
     float s = 0.0f;
 #pragma unroll
@@ -686,7 +701,8 @@ DEVI bool item_up(const StepArgs &a, int bid, unsigned char *smem, unsigned *s_f
             for (int j = 0; j < NP; ++j)
                 if (ok[j]) {
                     if (a.ws.up_tap) a.ws.up_tap[o[j]] = sum[j];
-                    a.out[o[j]] = f32_to_bf16_rne(sum[j] + shv[j]);
+                    if (a.out_f32) a.out_f32[o[j]] = sum[j] + shv[j];
+                    else a.out[o[j]] = f32_to_bf16_rne(sum[j] + shv[j]);
                 }
         }
     }

@@ -1,6 +1,8 @@
 """Helpers shared by the GPU tests: upload seeded weights, run the layer, compare with the oracle."""
 from __future__ import annotations
 
+import dataclasses
+
 import numpy as np
 
 import synth
@@ -90,3 +92,33 @@ def run_layer(layer, x_np: np.ndarray):
     torch.cuda.synchronize()
     return (bf16_tensor_to_f32(out), idx.cpu().numpy(), w.cpu().numpy(),
             {k: v.cpu().numpy() for k, v in taps.items()})
+
+
+def oracle_layer_of_shard(wd: synth.Dims, W: dict, shard):
+    """The oracle's dims, weights and n_shared for one shard: the shard's arrays (from
+    ep.shard_weights) in a full-size layer whose other experts have zero codes."""
+    from moe_decode_layer_moedec_b200 import LayerDims
+    from moe_decode_layer_moedec_b200 import ep
+    d = LayerDims(wd.hidden, wd.latent, wd.n_experts, wd.top_k, wd.expert_inter, wd.shared_inter, 1)
+    sd, SW = ep.shard_weights(d, W, shard)
+    O = {n: W[n] for n in ("router", "w_down_lat", "w_up_lat")}
+    e0, e1 = shard.expert_begin, shard.expert_begin + shard.expert_count
+    for n in ("gate_q", "up_q", "down_q"):
+        a = np.zeros_like(W[n])
+        a[e0:e1] = SW[n]
+        O[n] = a
+    for n in ("gate_s", "up_s", "down_s"):
+        a = np.full_like(W[n], 127)
+        a[e0:e1] = SW[n]
+        O[n] = a
+    if sd.n_shared:
+        for n in ("sh_gate_q", "sh_gate_s", "sh_up_q", "sh_up_s", "sh_down_q", "sh_down_s"):
+            O[n] = np.ascontiguousarray(SW[n])
+        od = dataclasses.replace(wd, shared_inter=shard.shared_count)
+    else:  # no slice: the oracle is told there is no shared expert (its arrays are not read)
+        od = dataclasses.replace(wd, shared_inter=128)
+        H = wd.hidden
+        for n, shape in (("sh_gate_q", (128, H // 2)), ("sh_gate_s", (128, H // 32)), ("sh_up_q", (128, H // 2)),
+                         ("sh_up_s", (128, H // 32)), ("sh_down_q", (H, 64)), ("sh_down_s", (H, 4))):
+            O[n] = np.zeros(shape, dtype=np.uint8)
+    return od, O, sd.n_shared
