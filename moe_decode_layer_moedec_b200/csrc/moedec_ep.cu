@@ -9,10 +9,10 @@
 // reduction ("快是可以生成的，可信只能证明（vLLM 重写 Kimi K3 解码路径…）", section 他们换掉了什么);
 // here the same exchange is two small kernels over peer memory:
 //
-//   k_ep_publish  after rank r's partial step (stream order): one thread fences at system scope
-//                 and release-stores the step's epoch into flag slot r of every rank's flag array.
-//   k_ep_combine  every block waits (bounded, %globaltimer) until all G flag words of this rank
-//                 reach the epoch (acquire, system scope), then sums the G partials element by
+//   k_ep_publish  after rank r's partial step (stream order): lane g of one warp fences at system
+//                 scope and release-stores the step's epoch into flag slot r of rank g's flag array.
+//   k_ep_combine  in every block, thread g waits (bounded, %globaltimer) until flag word g of this
+//                 rank reaches the epoch (acquire, system scope), then the block sums the G partials element by
 //                 element in rank order in fp32 and rounds once to bf16.  The partials are read
 //                 with loads that bypass the non-coherent caches (ld.global.cv), since a peer
 //                 may have written them while this kernel was already resident.
@@ -47,34 +47,31 @@ DEVI void st_release_sys(unsigned *p, unsigned v) {
     asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+// one warp: lane g fences and release-stores into rank g's flag array (the stores go out together)
 __global__ void k_ep_publish(EpSlots slots, int world, unsigned epoch) {
-    if (threadIdx.x == 0 && blockIdx.x == 0) {
+    const int g = threadIdx.x;
+    if (blockIdx.x == 0 && g < world) {
         __threadfence_system();
-        for (int g = 0; g < world; ++g) st_release_sys(slots.p[g], epoch);
+        st_release_sys(slots.p[g], epoch);
     }
 }
 
 __global__ void __launch_bounds__(256) k_ep_combine(EpParts parts, const unsigned *flags, int world, unsigned epoch,
                                                     size_t n4, uint16_t *out, unsigned *err, long long wait_ns) {
-    __shared__ int s_ok;
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        if (flags) {
-            const unsigned long long t0 = ep_now_ns();
-            for (int g = 0; g < world && ok; ++g)
-                while ((int)(ld_acquire_sys(flags + g) - epoch) < 0) {
-                    if ((long long)(ep_now_ns() - t0) > wait_ns) {
-                        atomicOr(err, kErrTimeout);
-                        ok = 0;
-                        break;
-                    }
-                    __nanosleep(64);
-                }
+    // thread g polls rank g's flag word (all ranks' flags at once, not one after another)
+    int ok = 1;
+    if (flags && threadIdx.x < world) {
+        const unsigned long long t0 = ep_now_ns();
+        while ((int)(ld_acquire_sys(flags + threadIdx.x) - epoch) < 0) {
+            if ((long long)(ep_now_ns() - t0) > wait_ns) {
+                atomicOr(err, kErrTimeout);
+                ok = 0;
+                break;
+            }
+            __nanosleep(32);
         }
-        s_ok = ok;
     }
-    __syncthreads();
-    if (!s_ok) return;
+    if (!__syncthreads_and(ok)) return;
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         float4 s = __ldcv(reinterpret_cast<const float4 *>(parts.p[0]) + i);
         for (int g = 1; g < world; ++g) {
