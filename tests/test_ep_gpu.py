@@ -139,6 +139,31 @@ def test_ep_combine_times_out_without_flags(tiny):
         grp.close()
 
 
+def test_step_partial_of_a_whole_layer_takes_the_small_batch_kernel():
+    # the streaming schedule writes bf16 only: a partial step of a handle created with
+    # MOEDEC_FLAG_STREAM runs the small-batch kernel instead (one launch, not four).  The mid-size
+    # layer: every dimension a multiple of 512, so its full steps do take the streaming schedule
+    from moe_decode_layer_moedec_b200 import FLAG_STREAM, MoeDecodeLayer
+    w = synth.WORKLOADS["mid_b2"]
+    W = synth.layer_weights(w, 0)
+    W_dev = upload_weights(W)
+    layer = MoeDecodeLayer(layer_dims(w.dims), W_dev, max_batch=2, flags=FLAG_STREAM)
+    launches = lambda: sum(layer.launch_counts().values())
+    try:
+        for B in (1, 2):
+            x_np = synth.tokens(w, step=7, batch=B)
+            before = launches()
+            part = layer.step_partial(to_device(x_np))
+            assert launches() - before == 1
+            set_config(f"partial mid B{B} stream flag")
+            assert_close(part.cpu().numpy(), oracle.step(w.dims, W, x_np)["out"], f"partial mid B{B}")
+            before = launches()
+            layer.step(to_device(x_np))
+            assert launches() - before == layer.kernels_per_step(B) == 4
+    finally:
+        layer.close()
+
+
 def test_ipc_export_names_the_allocation_and_the_offset():
     import torch
     from moe_decode_layer_moedec_b200 import IPC_HANDLE_BYTES, ipc_export
