@@ -180,13 +180,17 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(rows)}
 
 
+# the files that decide what a kernel reads and writes: its code, and moedec_api.cu, which sizes
+# its work items (the plan of K splits)
 KERNEL_SOURCES = {
     "fused_step_stream": ["moedec_stream.cu", "moedec_items.cuh", "moedec_tiles.cuh", "moedec_device.cuh",
-                          "moedec_router.cuh", "moedec_internal.h"],
+                          "moedec_router.cuh", "moedec_internal.h", "moedec_api.cu"],
     "fused_step_small": ["moedec_fused_small.cu", "moedec_ring.cuh", "moedec_experts.cuh", "moedec_items.cuh",
-                         "moedec_tiles.cuh", "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h"],
+                         "moedec_tiles.cuh", "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h",
+                         "moedec_api.cu"],
     "fused_step_splitk": ["moedec_fused.cu", "moedec_ring.cuh", "moedec_experts.cuh", "moedec_items.cuh",
-                          "moedec_tiles.cuh", "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h"],
+                          "moedec_tiles.cuh", "moedec_device.cuh", "moedec_router.cuh", "moedec_internal.h",
+                          "moedec_api.cu"],
 }
 
 

@@ -297,6 +297,13 @@ int create_handle(const moedec_config *cfg, const moedec_weights *w, int e0, int
     p.dn = split(d.L, kDenseRows, d.H);
     p.up = split(d.H, kDenseRows, d.L);
     p.sgu = split(d.Is, kDenseRows, d.H);
+    // K ranges of 1024 for the shared gate/up when H allows: half the items and half the splits
+    // that the last CTA of a row block adds up (its reduction was the tail that delayed a few
+    // CTAs' start of the expert phase; B = 16 280.2 -> 277.2 us)
+    if (d.H % 1024 == 0) {
+        p.sgu.krange = 1024;
+        p.sgu.splits = d.H / 1024;
+    }
     p.sd = split(d.H, kDenseRows, d.Is);
     p.ticket_rt = 0;
     p.ticket_dn = p.ticket_rt + p.rt.blocks;
