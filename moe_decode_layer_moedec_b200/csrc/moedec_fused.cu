@@ -156,7 +156,17 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
         cta_queue(Q_DN, n_dn, [&](int it) { item_dn<true, T::NTX, T::MAXB>(a, it, smem, &s_flag); return true; });
         stamp(3);
         // 3: shared gate/up
-        cta_queue(Q_SGU, n_sgu, [&](int it) { item_sgu<true, T::NTX, T::MAXB>(a, it, smem, &s_flag); return true; });
+        cta_queue(Q_SGU, n_sgu, [&](int it) {
+            if constexpr (TIER == 3) {  // record the CTA (see the expert gate/up ranges below)
+                if (threadIdx.x == 0 && gridDim.x <= 32 * kSguBitWords) {
+                    atomicOr(ctl + CTL_SGU_BITS + blockIdx.x / 32, 1u << (blockIdx.x % 32));
+                    __threadfence();
+                    atomicAdd(ctl + CTL_SGU_REC, 1u);
+                }
+            }
+            item_sgu<true, T::NTX, T::MAXB>(a, it, smem, &s_flag);
+            return true;
+        });
     }
     stamp(4);
     // 4: expert gate/up: routing and all of h must be final; the CTA's static range of the
@@ -176,7 +186,29 @@ __global__ void __launch_bounds__(256, Tier<TIER>::MINB) k_fused(StepArgs a, con
         __syncthreads();
         int lo, hi;
         range((a.d.I / 8) * segp.ngroups, lo, hi);
-        const bool ok = ring_rows<true, NSW>(a, maps, n_act, segp, rs, ring_gr, ring, ring_xs, lo, hi, ring_pos);
+        if constexpr (TIER == 3) {
+            // At 17-64 tokens the CTAs that took a shared gate/up item enter this phase late (those
+            // items run into the expert streams), so they get 6/8 of an equal share of its units.
+            // Every CTA reads the same final bitmap: the ranges still partition [0, n).
+            if (n_sgu && gridDim.x <= 32 * kSguBitWords) {
+                alive = cta_wait_geq(a, ctl + CTL_SGU_REC, (unsigned)n_sgu, &s_ok);
+                const int c = blockIdx.x, G = gridDim.x;
+                int before = 0, total = 0;
+                for (int w = 0; w < (G + 31) / 32; ++w) {
+                    const unsigned bits = __ldcg(ctl + CTL_SGU_BITS + w);
+                    total += __popc(bits);
+                    if (w < c / 32) before += __popc(bits);
+                    else if (w == c / 32) before += __popc(bits & ((1u << (c % 32)) - 1u));
+                }
+                const bool mine = (__ldcg(ctl + CTL_SGU_BITS + c / 32) >> (c % 32)) & 1u;
+                constexpr long long WN = 8, WS = 6;
+                const long long wpre = WN * c - (WN - WS) * before, wtot = WN * G - (WN - WS) * total;
+                const long long n = (long long)(a.d.I / 8) * segp.ngroups;
+                lo = (int)(n * wpre / wtot);
+                hi = (int)(n * (wpre + (mine ? WS : WN)) / wtot);
+            }
+        }
+        const bool ok = alive && ring_rows<true, NSW>(a, maps, n_act, segp, rs, ring_gr, ring, ring_xs, lo, hi, ring_pos);
         alive = __syncthreads_and(ok ? 1 : 0) != 0;
     } else if (alive) {
         cta_load_routing(a, route);

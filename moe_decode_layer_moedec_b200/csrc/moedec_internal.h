@@ -27,6 +27,7 @@ constexpr int kSmallSharedPer64 = 8;
 constexpr int kSmallSplitRt = 16, kSmallSplitDn = 16, kSmallSplitSgu = 8, kSmallSplitEgu = 2, kSmallSplitSd = 1,
               kSmallSplitUp = 4;
 constexpr int kSmallMaxBatch = 4;  // tokens of the small-batch step
+constexpr int kSguBitWords = 16;   // CTL_SGU_BITS words: grids up to 512 CTAs
 constexpr int kTraceStamps = 16;     // MOEDEC_TRACE_STAMPS
 
 // e0, ne: the experts whose weights this handle holds, [e0, e0 + ne) of the E the router scores
@@ -92,7 +93,9 @@ enum CtlWord {
     CTL_TOPK_TICKET,    // tokens whose top-k is written
     CTL_EXIT,           // CTAs that left the fused kernel
     CTL_ABORT,          // set when a bounded wait gave up; every CTA then leaves
-    CTL_FIXED = 16
+    CTL_SGU_REC = 16,   // shared gate/up items whose CTA is recorded in CTL_SGU_BITS (split-K, 17-64 tokens)
+    CTL_SGU_BITS = 17,  // [kSguBitWords] one bit per CTA that took a shared gate/up item
+    CTL_FIXED = 33
 };
 
 // Device workspace of one handle (all sized for max_batch).
