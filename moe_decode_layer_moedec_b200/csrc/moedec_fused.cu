@@ -56,7 +56,7 @@ template <> struct Tier<2> {
     using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
 };
 template <> struct Tier<3> {
-    static constexpr int NTX = 4, NTS = 4, NTU = 4, MINB = 2;
+    static constexpr int NTX = 4, NTS = 4, NTU = 8, MINB = 2;
     static constexpr int MAXB = 64;
     static constexpr bool SPLITS = false;
     using RT = RouteTables<kMaxExperts, 64 * kMaxTopK>;
