@@ -519,8 +519,8 @@ def ep_emulated(args, w, n_layers, local_rank):
     def exchange(i):
         g = groups[i % n]
         e = g.clock.epoch  # already published by every rank: the combine does not wait
-        g.layers[0].ep_publish([g._flag_ptr(q, 0) for q in range(G)], e, stream=stream)
-        g.layers[0].ep_combine([g.parts[q, e % 2].data_ptr() for q in range(G)], g._flag_ptr(0, 0), e, B, out,
+        g.layers[0].ep_publish([g.flag_ptr(q, 0) for q in range(G)], e, stream=stream)
+        g.layers[0].ep_combine([g.parts[q, e % 2].data_ptr() for q in range(G)], g.flag_ptr(0, 0), e, B, out,
                                stream=stream)
     xch = timed(exchange)
     for g in groups:

@@ -135,7 +135,8 @@ class EmulatedExpertParallel:
         self.flags = torch.zeros((world, world), dtype=torch.int32, device="cuda")
         self.clock = EpochCounter()
 
-    def _flag_ptr(self, owner: int, slot: int) -> int:
+    def flag_ptr(self, owner: int, slot: int) -> int:
+        """Device address of flag word `slot` (the publishing rank) in rank `owner`'s flag array."""
         return self.flags.data_ptr() + 4 * (owner * self.world + slot)
 
     def step(self, x, stream=None):
@@ -147,11 +148,11 @@ class EmulatedExpertParallel:
         for r, layer in enumerate(self.layers):
             layer.step_partial(x, self.parts[r, parity], stream)
         for r, layer in enumerate(self.layers):
-            layer.ep_publish([self._flag_ptr(q, r) for q in range(self.world)], epoch, stream)
+            layer.ep_publish([self.flag_ptr(q, r) for q in range(self.world)], epoch, stream)
         outs = []
         for r, layer in enumerate(self.layers):
             out = torch.empty((B, self.dims.hidden), dtype=x.dtype, device=x.device)
-            layer.ep_combine([self.parts[g, parity].data_ptr() for g in range(self.world)], self._flag_ptr(r, 0),
+            layer.ep_combine([self.parts[g, parity].data_ptr() for g in range(self.world)], self.flag_ptr(r, 0),
                              epoch, B, out, stream)
             outs.append(out)
         return outs, [self.parts[r, parity, :B] for r in range(self.world)]

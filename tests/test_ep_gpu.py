@@ -126,9 +126,9 @@ def test_ep_combine_times_out_without_flags(tiny):
         epoch, parity = grp.clock.next()
         for r, layer in enumerate(grp.layers):
             layer.step_partial(x, grp.parts[r, parity])
-        grp.layers[0].ep_publish([grp._flag_ptr(q, 0) for q in range(2)], epoch)
+        grp.layers[0].ep_publish([grp.flag_ptr(q, 0) for q in range(2)], epoch)
         out = torch.full((B, w.dims.hidden), 0x40E0, dtype=torch.int16, device="cuda")  # bf16 7.0
-        grp.layers[0].ep_combine([grp.parts[g, parity].data_ptr() for g in range(2)], grp._flag_ptr(0, 0), epoch, B,
+        grp.layers[0].ep_combine([grp.parts[g, parity].data_ptr() for g in range(2)], grp.flag_ptr(0, 0), epoch, B,
                                  out)
         with pytest.raises(MoedecError, match="TIMEOUT"):
             grp.layers[0].routing(B)
