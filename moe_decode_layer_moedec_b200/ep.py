@@ -162,6 +162,36 @@ class EmulatedExpertParallel:
             layer.close()
 
 
+def peer_addresses(rank: int, handles: list, local: tuple, open_fn):
+    """This process's addresses of every rank's partial buffers and flag array.
+
+    handles[g] = ((parts_handle, parts_offset), (flags_handle, flags_offset)) as rank g exported
+    them; local = (parts_ptr, flags_ptr) of this rank; open_fn maps an exported handle to the base
+    address of its allocation here.  A handle is opened once even when both buffers of a rank lie
+    in one allocation.  Returns (parts[g], flags[g], opened bases to close later)."""
+    parts, flags, opened = [], [], []
+    for g, ((hp, op), (hf, of)) in enumerate(handles):
+        if g == rank:
+            parts.append(local[0])
+            flags.append(local[1])
+            continue
+        bp = open_fn(hp)
+        opened.append(bp)
+        if hf == hp:
+            bf = bp
+        else:
+            bf = open_fn(hf)
+            opened.append(bf)
+        parts.append(bp + op)
+        flags.append(bf + of)
+    return parts, flags, opened
+
+
+def publish_slots(rank: int, peer_flags: list) -> list:
+    """The flag word that rank `rank` release-stores into, in every rank's flag array (u32 words)."""
+    return [f + 4 * rank for f in peer_flags]
+
+
 def exchange(obj, group=None) -> list:
     """Every rank's `obj`, in rank order (one all_gather_object over the process group)."""
     import torch.distributed as dist
@@ -192,22 +222,8 @@ class ExpertParallelLayer:
         self.flags = torch.zeros((self.world,), dtype=torch.int32, device="cuda")
         torch.cuda.synchronize()
         handles = exchange((ipc_export(self.parts.data_ptr()), ipc_export(self.flags.data_ptr())), group)
-        self._opened = []
-        self.peer_parts, self.peer_flags = [], []
-        for g, ((hp, op), (hf, of)) in enumerate(handles):
-            if g == self.rank:
-                self.peer_parts.append(self.parts.data_ptr())
-                self.peer_flags.append(self.flags.data_ptr())
-                continue
-            bp = ipc_open(hp)
-            self._opened.append(bp)
-            if hf == hp:  # both buffers in one allocation of the exporter
-                bf = bp
-            else:
-                bf = ipc_open(hf)
-                self._opened.append(bf)
-            self.peer_parts.append(bp + op)
-            self.peer_flags.append(bf + of)
+        self.peer_parts, self.peer_flags, self._opened = peer_addresses(
+            self.rank, handles, (self.parts.data_ptr(), self.flags.data_ptr()), ipc_open)
         self.clock = EpochCounter()
         self._part_bytes = max_batch * H * 4
 
@@ -218,7 +234,7 @@ class ExpertParallelLayer:
             out = torch.empty((B, self.dims.hidden), dtype=x.dtype, device=x.device)
         epoch, parity = self.clock.next()
         self.layer.step_partial(x, self.parts[parity], stream)
-        self.layer.ep_publish([f + 4 * self.rank for f in self.peer_flags], epoch, stream)
+        self.layer.ep_publish(publish_slots(self.rank, self.peer_flags), epoch, stream)
         self.layer.ep_combine([p + parity * self._part_bytes for p in self.peer_parts], self.flags.data_ptr(),
                               epoch, B, out, stream)
         return out

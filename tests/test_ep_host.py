@@ -6,8 +6,10 @@ tests pin the host side of that against the oracle.  Each shard's weights come f
 `ep.shard_weights`.  They are put back into a full-size layer whose other experts have zero
 codes (an E2M1 code 0 is +0, so those experts add exactly nothing).  The oracle's outputs of the
 shards, summed, must equal its output for the whole layer (fp64, so up to rounding), and every
-shard must route the same.  The world-size-2 test runs the same over two gloo processes, with the
-partition agreed through `ep.exchange`.
+shard must route the same.  The world-size-2 tests run the same over two gloo processes, with the
+partition agreed through `ep.exchange`, and map each other's exchange buffers from exported
+handles (a fake IPC opener stands in for the GPU: the addresses, the offsets, one opening per
+allocation, and the flag slot each rank publishes into).
 """
 import dataclasses
 import datetime
@@ -186,3 +188,64 @@ def test_two_gloo_ranks_reassemble_the_layer_output():
         assert np.abs(total - full["out"]).max() <= 1e-12 * scale
         assert np.abs(reduced - full["out"]).max() <= 1e-12 * scale
     assert np.array_equal(got[0][2], got[1][2])  # the same rank-order sum on both ranks
+
+
+def _fake_handle(kind: str, rank: int) -> bytes:
+    return (kind.encode() + bytes([rank])).ljust(64, b"\0")
+
+
+def _fake_base(handle: bytes) -> int:
+    return 0x1000_0000 * (handle[1] + 1) + (0x100_0000 if handle[:1] == b"F" else 0)
+
+
+def _rank_main_peers(rank: int, world: int, port: int, q) -> None:
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        # rank 0: both buffers in one allocation (one handle, two offsets); rank 1: two allocations
+        parts = (_fake_handle("P", rank), 256 * (rank + 1))
+        flags = (_fake_handle("P", rank), 4096) if rank == 0 else (_fake_handle("F", rank), 64)
+        handles = ep.exchange((parts, flags))
+        opened_calls = []
+
+        def fake_open(h):
+            opened_calls.append(h)
+            return _fake_base(h)
+        local = (0xAAAA_0000 + rank, 0xBBBB_0000 + rank)
+        pp, pf, opened = ep.peer_addresses(rank, handles, local, fake_open)
+        q.put((rank, pp, pf, opened, opened_calls, ep.publish_slots(rank, pf)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_map_each_others_exchange_buffers():
+    import torch.multiprocessing as mp
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main_peers, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    got = {g[0]: g[1:] for g in (q.get(timeout=10) for _ in range(world))}
+    # rank 0 sees rank 1's two allocations, each opened once, at base + offset
+    pp, pf, opened, calls, slots = got[0]
+    assert pp[0] == 0xAAAA_0000 and pf[0] == 0xBBBB_0000
+    assert pp[1] == _fake_base(_fake_handle("P", 1)) + 512 and pf[1] == _fake_base(_fake_handle("F", 1)) + 64
+    assert calls == [_fake_handle("P", 1), _fake_handle("F", 1)] and len(opened) == 2
+    assert slots == [pf[0], pf[1]]
+    # rank 1 sees rank 0's single allocation opened once, with the two offsets
+    pp, pf, opened, calls, slots = got[1]
+    assert pp[1] == 0xAAAA_0001 and pf[1] == 0xBBBB_0001
+    base = _fake_base(_fake_handle("P", 0))
+    assert pp[0] == base + 256 and pf[0] == base + 4096
+    assert calls == [_fake_handle("P", 0)] and opened == [base]
+    assert slots == [pf[0] + 4, pf[1] + 4]
